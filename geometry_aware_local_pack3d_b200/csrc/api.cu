@@ -1,0 +1,129 @@
+// C ABI of the PACK3D operator: argument checks and dispatch to the kernels.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace p3d {
+thread_local int g_launches = 0;
+
+cudaError_t summarize_dispatch(const pack3d_index& ix, const void* k, const void* v, int dtype,
+                               int64_t bh, void* ksum, void* vsum, cudaStream_t s);
+cudaError_t fwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, int dtype, int64_t bh, float scale, int excl,
+                              void* o, float* lse_loc, float* lse_glob, void* o_loc,
+                              void* o_glob, cudaStream_t s);
+cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, const void* o_loc, const void* o_glob,
+                              const float* lse_loc, const float* lse_glob, const void* dO,
+                              int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
+                              void* dv, void* dgate, void* ws, cudaStream_t s);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh);
+}  // namespace p3d
+
+using namespace p3d;
+
+namespace {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int heads) {
+  if (!idx || !idx->coord || !idx->nbr || !idx->members || !idx->rope)
+    return PACK3D_ERR_INVALID_ARG;
+  if (dtype != PACK3D_F32 && dtype != PACK3D_BF16) return PACK3D_ERR_INVALID_ARG;
+  if (batch <= 0 || heads <= 0) return PACK3D_ERR_INVALID_ARG;
+  if ((int64_t)batch * heads > 65535) return PACK3D_ERR_UNSUPPORTED;
+  if (idx->geom.head_dim != 48 && idx->geom.head_dim != 96) return PACK3D_ERR_UNSUPPORTED;
+  return PACK3D_OK;
+}
+
+pack3d_status check_rows(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (!p) return PACK3D_ERR_INVALID_ARG;
+    if (!aligned16(p)) return PACK3D_ERR_ALIGN;
+  }
+  return PACK3D_OK;
+}
+
+pack3d_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
+}  // namespace
+
+extern "C" const char* pack3d_strerror(pack3d_status s) {
+  switch (s) {
+    case PACK3D_OK: return "ok";
+    case PACK3D_ERR_INVALID_ARG: return "invalid argument";
+    case PACK3D_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PACK3D_ERR_DUP_COORD: return "two tokens carry the same coordinate";
+    case PACK3D_ERR_COORD_RANGE: return "coordinate outside the grid";
+    case PACK3D_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PACK3D_ERR_TIMEOUT: return "device-side wait timed out";
+    case PACK3D_ERR_CUDA: return "CUDA runtime error";
+    case PACK3D_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+extern "C" int pack3d_last_launch_count(void) { return g_launches; }
+
+extern "C" pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const void* v,
+                                          int dtype, int batch, int heads, void* ksum,
+                                          void* vsum, void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({k, v, ksum, vsum})) != PACK3D_OK) return st;
+  return cuda_status(summarize_dispatch(*idx, k, v, dtype, (int64_t)batch * heads, ksum, vsum,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void* k,
+                                         const void* v, const void* gate, const void* ksum,
+                                         const void* vsum, int dtype, int batch, int heads,
+                                         float scale, uint32_t flags, void* o, float* lse_loc,
+                                         float* lse_glob, void* o_loc, void* o_glob,
+                                         void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({q, k, v, ksum, vsum, o})) != PACK3D_OK) return st;
+  if (!gate) return PACK3D_ERR_INVALID_ARG;
+  if ((o_loc && !aligned16(o_loc)) || (o_glob && !aligned16(o_glob))) return PACK3D_ERR_ALIGN;
+  if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
+  const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
+  const int64_t bh = (int64_t)batch * heads;
+  return cuda_status(fwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, dtype, bh, scale, excl,
+                                       o, lse_loc, lse_glob, o_loc, o_glob,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch,
+                                             int heads) {
+  if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;
+  return bwd_workspace_bytes(*idx, (int64_t)batch * heads);
+}
+
+extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
+                                         const void* v, const void* gate, const void* ksum,
+                                         const void* vsum, const void* o_loc,
+                                         const void* o_glob, const float* lse_loc,
+                                         const float* lse_glob, const void* dO, int dtype,
+                                         int batch, int heads, float scale, uint32_t flags,
+                                         void* dq, void* dk, void* dv, void* dgate,
+                                         void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({q, k, v, ksum, vsum, o_loc, o_glob, dO, dq, dk, dv})) != PACK3D_OK)
+    return st;
+  if (!gate || !dgate || !lse_loc || !lse_glob || !workspace) return PACK3D_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return PACK3D_ERR_ALIGN;
+  if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
+  const int64_t bh = (int64_t)batch * heads;
+  if (workspace_bytes < bwd_workspace_bytes(*idx, bh)) return PACK3D_ERR_WORKSPACE;
+  const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
+  return cuda_status(bwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc,
+                                       lse_glob, dO, dtype, bh, scale, excl, dq, dk, dv, dgate,
+                                       workspace, static_cast<cudaStream_t>(stream)));
+}

@@ -1,0 +1,550 @@
+// PACK3D attention on CUDA cores in float32: the general path for every supported dtype and
+// head_dim (float32 I/O always runs here), forward and backward.
+//
+// Forward (project page "Geometry Matters in Packed 3D Attention", Chapter 3 Contracts 1-3;
+// paper summary §3.2, §3.3, §3.5):
+//   k_local_fwd   one thread per query: exact softmax over the <= 27 coordinate neighbours,
+//                 keys rotated on the fly from the rotation table, offsets in canonical order.
+//   k_global_fwd  one thread per query: online softmax over all summaries, staged through
+//                 shared memory in chunks (every thread reads the same summary: broadcast),
+//                 optional exclude_near mask, and the sigmoid mixer fused in the epilogue.
+// Backward (paper summary §3.4), one warp per row, lanes over head dims:
+//   k_bwd_prep    rotated q, k; dgate; D_loc = <g dO, o_loc>, D_glob = <(1-g) dO, o_glob>.
+//   k_bwd_dsum    dK_sum[m] = sum_i dS_im q~_i and dV_sum[m] = sum_i P_im (1-g_i) dO_i.
+//   k_bwd_dq      dq = R(c)^T (sum_j dS_ij k~_j + sum_m dS_im K_sum[m]).
+//   k_bwd_dkv     dk, dv gathered over the key's own neighbourhood (the 3x3x3 relation is
+//                 symmetric, so no scatter/atomics) plus 1/|S| of its block's summary grads.
+// Every reduction order depends on coordinates (offset order, canonical slots, summary ids),
+// never on memory slots, except the sums over all queries in k_bwd_dsum.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "vec.cuh"
+
+namespace p3d {
+
+// ------------------------------------------------------------------------------ helpers
+template <typename T, int D>
+__device__ __forceinline__ void load_row(const T* __restrict__ p, float (&x)[D]) {
+  constexpr int E = Vec<T>::E;
+#pragma unroll
+  for (int c = 0; c < D / E; ++c) {
+    float t[E];
+    Vec<T>::load(p + c * E, t);
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[c * E + e] = t[e];
+  }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void store_row(T* p, const float (&x)[D]) {
+  constexpr int E = Vec<T>::E;
+#pragma unroll
+  for (int c = 0; c < D / E; ++c) {
+    float t[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) t[e] = x[c * E + e];
+    Vec<T>::store(p + c * E, t);
+  }
+}
+
+// x <- R(c) x (sign = +1) or R(c)^T x (sign = -1), rotation table in global memory.
+template <int D>
+__device__ __forceinline__ void rotate_row(const pack3d_index& ix, const Coord& c,
+                                           float (&x)[D], float sign) {
+  constexpr int DA = D / 3;
+#pragma unroll
+  for (int e = 0; e < D; e += 2) {
+    const int axis = e / DA, p = (e % DA) / 2;
+    const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+    const float sn = sign * cs.y;
+    const float x0 = x[e], x1 = x[e + 1];
+    x[e] = x0 * cs.x - x1 * sn;
+    x[e + 1] = x0 * sn + x1 * cs.x;
+  }
+}
+
+// ------------------------------------------------------------------------ local forward
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_local_fwd(pack3d_index ix, const T* __restrict__ q,
+                                                   const T* __restrict__ k,
+                                                   const T* __restrict__ v, float scale,
+                                                   T* __restrict__ o_loc,
+                                                   float* __restrict__ lse_loc) {
+  const int64_t bh = blockIdx.y;
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= ix.n) return;
+  const int64_t rowbase = bh * ix.n;
+  const Coord ci = decode(ix.coord[i]);
+  float qr[D];
+  load_row<T, D>(q + (rowbase + i) * D, qr);
+  rotate_row<D>(ix, ci, qr, 1.f);
+
+  const float sl2 = scale * kLog2e;
+  float s[kNbr];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int o = 0; o < kNbr; ++o) {
+    const int j = ix.nbr[i * kNbr + o];
+    s[o] = -INFINITY;
+    if (j < 0) continue;
+    float kr[D];
+    load_row<T, D>(k + (rowbase + j) * D, kr);
+    rotate_row<D>(ix, decode(ix.coord[j]), kr, 1.f);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < D; ++e) dot = fmaf(qr[e], kr[e], dot);
+    s[o] = dot * sl2;
+    mx = fmaxf(mx, s[o]);
+  }
+  float l = 0.f;
+  float acc[D];
+#pragma unroll
+  for (int e = 0; e < D; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int o = 0; o < kNbr; ++o) {
+    const int j = ix.nbr[i * kNbr + o];
+    if (j < 0) continue;
+    const float p = exp2f(s[o] - mx);
+    l += p;
+    float vr[D];
+    load_row<T, D>(v + (rowbase + j) * D, vr);
+#pragma unroll
+    for (int e = 0; e < D; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
+  }
+  const float inv = 1.f / l;  // the query itself is always a neighbour: l >= 1
+#pragma unroll
+  for (int e = 0; e < D; ++e) acc[e] *= inv;
+  store_row<T, D>(o_loc + (rowbase + i) * D, acc);
+  if (lse_loc) lse_loc[rowbase + i] = (mx + log2f(l)) * kLn2;
+}
+
+// ------------------------------------------------------------------ global forward + mixer
+template <typename T, int D, int CH>
+__global__ void __launch_bounds__(128) k_global_fwd(
+    pack3d_index ix, const T* __restrict__ q, const T* __restrict__ ksum,
+    const T* __restrict__ vsum, const T* __restrict__ gate, const T* o_loc_in, float scale,
+    int exclude_near, T* o, float* __restrict__ lse_glob, T* __restrict__ o_glob_out) {
+  __shared__ float sk[CH][D];
+  __shared__ float sv[CH][D];
+  const int64_t bh = blockIdx.y;
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const bool live = i < ix.n;
+  const int64_t rowbase = bh * ix.n;
+  const int M = (int)ix.m;
+  Coord ci{0, 0, 0};
+  float qr[D];
+  if (live) {
+    ci = decode(ix.coord[i]);
+    load_row<T, D>(q + (rowbase + i) * D, qr);
+    rotate_row<D>(ix, ci, qr, 1.f);
+  }
+  const float sl2 = scale * kLog2e;
+  float mx = -INFINITY, l = 0.f;
+  float acc[D];
+#pragma unroll
+  for (int e = 0; e < D; ++e) acc[e] = 0.f;
+
+  const T* kb = ksum + bh * (int64_t)M * D;
+  const T* vb = vsum + bh * (int64_t)M * D;
+  for (int m0 = 0; m0 < M; m0 += CH) {
+    const int cnt = min(CH, M - m0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < cnt * D; t += blockDim.x) {
+      sk[t / D][t % D] = to_f(kb[(int64_t)m0 * D + t]);
+      sv[t / D][t % D] = to_f(vb[(int64_t)m0 * D + t]);
+    }
+    __syncthreads();
+    if (!live) continue;
+    for (int mm = 0; mm < cnt; ++mm) {
+      if (exclude_near && block_is_near(ix, m0 + mm, ci)) continue;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < D; ++e) dot = fmaf(qr[e], sk[mm][e], dot);
+      const float sc = dot * sl2;
+      if (sc > mx) {
+        const float corr = exp2f(mx - sc);  // exp2(-inf) = 0 on the first hit
+        l *= corr;
+#pragma unroll
+        for (int e = 0; e < D; ++e) acc[e] *= corr;
+        mx = sc;
+      }
+      const float p = exp2f(sc - mx);
+      l += p;
+#pragma unroll
+      for (int e = 0; e < D; ++e) acc[e] = fmaf(p, sv[mm][e], acc[e]);
+    }
+  }
+  if (!live) return;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < D; ++e) acc[e] *= inv;
+  if (lse_glob) lse_glob[rowbase + i] = l > 0.f ? (mx + log2f(l)) * kLn2 : -INFINITY;
+  if (o_glob_out) store_row<T, D>(o_glob_out + (rowbase + i) * D, acc);
+  // mixer (paper summary §3.3): o = g o_loc + (1 - g) o_glob, g = sigmoid(a)
+  const float a = to_f(gate[rowbase + i]);
+  const float g = 1.f / (1.f + expf(-a));
+  float ol[D];
+  load_row<T, D>(o_loc_in + (rowbase + i) * D, ol);
+#pragma unroll
+  for (int e = 0; e < D; ++e) acc[e] = g * ol[e] + (1.f - g) * acc[e];
+  store_row<T, D>(o + (rowbase + i) * D, acc);
+}
+
+// ------------------------------------------------------------------------------ backward
+// Warp-per-row layout: lane owns dims e = lane + 32 * t, t < KT.
+template <int D> struct WarpRow {
+  static constexpr int KT = (D + 31) / 32;
+  float x[KT];
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void wr_load(const T* __restrict__ p, WarpRow<D>& r, int lane) {
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    r.x[t] = e < D ? to_f(p[e]) : 0.f;
+  }
+}
+template <int D>
+__device__ __forceinline__ void wr_load_f(const float* __restrict__ p, WarpRow<D>& r, int lane) {
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    r.x[t] = e < D ? p[e] : 0.f;
+  }
+}
+template <typename T, int D>
+__device__ __forceinline__ void wr_store(T* p, const WarpRow<D>& r, int lane) {
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    if (e < D) p[e] = from_f<T>(r.x[t]);
+  }
+}
+template <int D>
+__device__ __forceinline__ float wr_dot(const WarpRow<D>& a, const WarpRow<D>& b) {
+  float s = 0.f;
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) s = fmaf(a.x[t], b.x[t], s);
+  return warp_sum(s);
+}
+// r <- R(c) r or R(c)^T r; the pair partner of dim e is e ^ 1, held by lane ^ 1.
+template <int D>
+__device__ __forceinline__ void wr_rotate(const pack3d_index& ix, const Coord& c, WarpRow<D>& r,
+                                          int lane, float sign) {
+  constexpr int DA = D / 3;
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    const float partner = __shfl_xor_sync(0xffffffffu, r.x[t], 1);
+    if (e < D) {
+      const int axis = e / DA, p = (e % DA) / 2;
+      const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+      const float sn = sign * cs.y;
+      // even e: x0' = x0 c - x1 s ; odd e: x1' = x0 s + x1 c
+      r.x[t] = (e & 1) ? fmaf(partner, sn, r.x[t] * cs.x) : fmaf(-partner, sn, r.x[t] * cs.x);
+    }
+  }
+}
+
+struct BwdWork {
+  float* qr;    // [BH, N, D]
+  float* kr;    // [BH, N, D]
+  float* Dl;    // [BH, N]
+  float* Dg;    // [BH, N]
+  float* dks;   // [BH, M, D]
+  float* dvs;   // [BH, M, D]
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __restrict__ q,
+                                                  const T* __restrict__ k,
+                                                  const T* __restrict__ gate,
+                                                  const T* __restrict__ o_loc,
+                                                  const T* __restrict__ o_glob,
+                                                  const T* __restrict__ dO, int64_t rows,
+                                                  BwdWork w, T* __restrict__ dgate) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t i = row % ix.n;
+  const Coord c = decode(ix.coord[i]);
+  WarpRow<D> a, b, d;
+  wr_load<T, D>(q + row * D, a, lane);
+  wr_rotate<D>(ix, c, a, lane, 1.f);
+  wr_load<T, D>(k + row * D, b, lane);
+  wr_rotate<D>(ix, c, b, lane, 1.f);
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    if (e < D) {
+      w.qr[row * D + e] = a.x[t];
+      w.kr[row * D + e] = b.x[t];
+    }
+  }
+  wr_load<T, D>(dO + row * D, d, lane);
+  wr_load<T, D>(o_loc + row * D, a, lane);
+  wr_load<T, D>(o_glob + row * D, b, lane);
+  const float dl = wr_dot<D>(d, a), dgl = wr_dot<D>(d, b);
+  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
+  if (lane == 0) {
+    dgate[row] = from_f<T>((dl - dgl) * g * (1.f - g));
+    w.Dl[row] = g * dl;
+    w.Dg[row] = (1.f - g) * dgl;
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __restrict__ ksum,
+                                                  const T* __restrict__ vsum,
+                                                  const T* __restrict__ gate,
+                                                  const T* __restrict__ dO,
+                                                  const float* __restrict__ lse_glob,
+                                                  float scale, int exclude_near, int64_t bh_count,
+                                                  BwdWork w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t M = ix.m;
+  if (task >= bh_count * M) return;
+  const int64_t bh = task / M;
+  const int m = (int)(task % M);
+  WarpRow<D> km, vm, ak, av, x, d;
+  wr_load<T, D>(ksum + task * D, km, lane);
+  wr_load<T, D>(vsum + task * D, vm, lane);
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
+  for (int64_t i = 0; i < ix.n; ++i) {
+    const int64_t row = bh * ix.n + i;
+    const float lse = lse_glob[row];
+    if (lse == -INFINITY) continue;
+    if (exclude_near && block_is_near(ix, m, decode(ix.coord[i]))) continue;
+    wr_load_f<D>(w.qr + row * D, x, lane);
+    wr_load<T, D>(dO + row * D, d, lane);
+    const float g1 = 1.f - 1.f / (1.f + expf(-to_f(gate[row])));
+    const float s = wr_dot<D>(x, km) * scale;
+    const float p = expf(s - lse);
+    const float dp = g1 * wr_dot<D>(d, vm);
+    const float ds = p * (dp - w.Dg[row]) * scale;
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) {
+      ak.x[t] = fmaf(ds, x.x[t], ak.x[t]);
+      av.x[t] = fmaf(p * g1, d.x[t], av.x[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    if (e < D) {
+      w.dks[task * D + e] = ak.x[t];
+      w.dvs[task * D + e] = av.x[t];
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __restrict__ v,
+                                                const T* __restrict__ ksum,
+                                                const T* __restrict__ vsum,
+                                                const T* __restrict__ gate,
+                                                const T* __restrict__ dO,
+                                                const float* __restrict__ lse_loc,
+                                                const float* __restrict__ lse_glob, float scale,
+                                                int exclude_near, int64_t rows, BwdWork w,
+                                                T* __restrict__ dq) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t bh = row / ix.n, i = row % ix.n;
+  const int64_t rowbase = bh * ix.n;
+  const Coord c = decode(ix.coord[i]);
+  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
+  WarpRow<D> qr, d, acc, x, y;
+  wr_load_f<D>(w.qr + row * D, qr, lane);
+  wr_load<T, D>(dO + row * D, d, lane);
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = 0.f;
+  // local branch
+  const float ll = lse_loc[row], Dl = w.Dl[row];
+  for (int o = 0; o < kNbr; ++o) {
+    const int j = ix.nbr[i * kNbr + o];
+    if (j < 0) continue;
+    wr_load_f<D>(w.kr + (rowbase + j) * D, x, lane);
+    wr_load<T, D>(v + (rowbase + j) * D, y, lane);
+    const float p = expf(wr_dot<D>(qr, x) * scale - ll);
+    const float ds = p * (g * wr_dot<D>(d, y) - Dl) * scale;
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = fmaf(ds, x.x[t], acc.x[t]);
+  }
+  // global branch
+  const float lg = lse_glob[row], Dg = w.Dg[row];
+  if (lg != -INFINITY) {
+    const int M = (int)ix.m;
+    for (int m = 0; m < M; ++m) {
+      if (exclude_near && block_is_near(ix, m, c)) continue;
+      wr_load<T, D>(ksum + (bh * M + m) * D, x, lane);
+      wr_load<T, D>(vsum + (bh * M + m) * D, y, lane);
+      const float p = expf(wr_dot<D>(qr, x) * scale - lg);
+      const float ds = p * ((1.f - g) * wr_dot<D>(d, y) - Dg) * scale;
+#pragma unroll
+      for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = fmaf(ds, x.x[t], acc.x[t]);
+    }
+  }
+  wr_rotate<D>(ix, c, acc, lane, -1.f);
+  wr_store<T, D>(dq + row * D, acc, lane);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __restrict__ v,
+                                                 const T* __restrict__ gate,
+                                                 const T* __restrict__ dO,
+                                                 const float* __restrict__ lse_loc, float scale,
+                                                 int64_t rows, BwdWork w, T* __restrict__ dk,
+                                                 T* __restrict__ dv) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t bh = row / ix.n, j = row % ix.n;
+  const int64_t rowbase = bh * ix.n;
+  const Coord c = decode(ix.coord[j]);
+  WarpRow<D> kr, vj, ak, av, x, d;
+  wr_load_f<D>(w.kr + row * D, kr, lane);
+  wr_load<T, D>(v + row * D, vj, lane);
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
+  // j is a neighbour of query i exactly when i is a neighbour of j
+  for (int o = 0; o < kNbr; ++o) {
+    const int i = ix.nbr[j * kNbr + o];
+    if (i < 0) continue;
+    const int64_t ri = rowbase + i;
+    wr_load_f<D>(w.qr + ri * D, x, lane);
+    wr_load<T, D>(dO + ri * D, d, lane);
+    const float g = 1.f / (1.f + expf(-to_f(gate[ri])));
+    const float p = expf(wr_dot<D>(x, kr) * scale - lse_loc[ri]);
+    const float ds = p * (g * wr_dot<D>(d, vj) - w.Dl[ri]) * scale;
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) {
+      ak.x[t] = fmaf(ds, x.x[t], ak.x[t]);
+      av.x[t] = fmaf(p * g, d.x[t], av.x[t]);
+    }
+  }
+  // un-pool: 1/|S| of the block summary's gradient
+  const int b = ix.block_of[j];
+  const float inv = 1.f / (float)ix.count[b];
+  wr_load_f<D>(w.dks + (bh * ix.m + b) * D, x, lane);
+  wr_load_f<D>(w.dvs + (bh * ix.m + b) * D, d, lane);
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    ak.x[t] = fmaf(x.x[t], inv, ak.x[t]);
+    av.x[t] = fmaf(d.x[t], inv, av.x[t]);
+  }
+  wr_rotate<D>(ix, c, ak, lane, -1.f);
+  wr_store<T, D>(dk + row * D, ak, lane);
+  wr_store<T, D>(dv + row * D, av, lane);
+}
+
+// ------------------------------------------------------------------------------ launchers
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh) {
+  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t D = ix.geom.head_dim;
+  return 2 * a(sizeof(float) * bh * ix.n * D) + 2 * a(sizeof(float) * bh * ix.n) +
+         2 * a(sizeof(float) * bh * ix.m * D);
+}
+
+static BwdWork carve(const pack3d_index& ix, int64_t bh, void* ws) {
+  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t D = ix.geom.head_dim;
+  char* p = static_cast<char*>(ws);
+  BwdWork w;
+  w.qr = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n * D);
+  w.kr = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n * D);
+  w.Dl = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n);
+  w.Dg = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n);
+  w.dks = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.m * D);
+  w.dvs = reinterpret_cast<float*>(p);
+  return w;
+}
+
+template <typename T, int D>
+cudaError_t fwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
+                     const void* gate, const void* ksum, const void* vsum, int64_t bh,
+                     float scale, int excl, void* o, float* lse_loc, float* lse_glob,
+                     void* o_loc, void* o_glob, cudaStream_t s) {
+  const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
+  T* ol = static_cast<T*>(o_loc ? o_loc : o);  // the local output may live in `o` until mixed
+  k_local_fwd<T, D><<<grid, 128, 0, s>>>(ix, static_cast<const T*>(q), static_cast<const T*>(k),
+                                          static_cast<const T*>(v), scale, ol, lse_loc);
+  k_global_fwd<T, D, 32><<<grid, 128, 0, s>>>(
+      ix, static_cast<const T*>(q), static_cast<const T*>(ksum), static_cast<const T*>(vsum),
+      static_cast<const T*>(gate), ol, scale, excl, static_cast<T*>(o), lse_glob,
+      static_cast<T*>(o_glob));
+  count_launch(2);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
+                     const void* gate, const void* ksum, const void* vsum, const void* o_loc,
+                     const void* o_glob, const float* lse_loc, const float* lse_glob,
+                     const void* dO, int64_t bh, float scale, int excl, void* dq, void* dk,
+                     void* dv, void* dgate, void* ws, cudaStream_t s) {
+  const BwdWork w = carve(ix, bh, ws);
+  const int64_t rows = bh * ix.n;
+  const unsigned rb = (unsigned)((rows + 3) / 4);
+  const unsigned mb = (unsigned)((bh * ix.m + 3) / 4);
+  const T* tq = static_cast<const T*>(q);
+  const T* tk = static_cast<const T*>(k);
+  const T* tv = static_cast<const T*>(v);
+  const T* tg = static_cast<const T*>(gate);
+  const T* tdo = static_cast<const T*>(dO);
+  k_bwd_prep<T, D><<<rb, 128, 0, s>>>(ix, tq, tk, tg, static_cast<const T*>(o_loc),
+                                       static_cast<const T*>(o_glob), tdo, rows, w,
+                                       static_cast<T*>(dgate));
+  k_bwd_dsum<T, D><<<mb, 128, 0, s>>>(ix, static_cast<const T*>(ksum),
+                                       static_cast<const T*>(vsum), tg, tdo, lse_glob, scale,
+                                       excl, bh, w);
+  k_bwd_dq<T, D><<<rb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
+                                     static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
+                                     scale, excl, rows, w, static_cast<T*>(dq));
+  k_bwd_dkv<T, D><<<rb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, w,
+                                      static_cast<T*>(dk), static_cast<T*>(dv));
+  count_launch(4);
+  return cudaGetLastError();
+}
+
+cudaError_t fwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, int dtype, int64_t bh, float scale, int excl,
+                              void* o, float* lse_loc, float* lse_glob, void* o_loc,
+                              void* o_glob, cudaStream_t s) {
+  const int d = ix.geom.head_dim;
+#define P3D_FWD(T, D) \
+  fwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, bh, scale, excl, o, lse_loc, lse_glob, o_loc, o_glob, s)
+  if (dtype == PACK3D_BF16) return d == 96 ? P3D_FWD(__nv_bfloat16, 96) : P3D_FWD(__nv_bfloat16, 48);
+  return d == 96 ? P3D_FWD(float, 96) : P3D_FWD(float, 48);
+#undef P3D_FWD
+}
+
+cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, const void* o_loc, const void* o_glob,
+                              const float* lse_loc, const float* lse_glob, const void* dO,
+                              int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
+                              void* dv, void* dgate, void* ws, cudaStream_t s) {
+  const int d = ix.geom.head_dim;
+#define P3D_BWD(T, D)                                                                         \
+  bwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc, lse_glob, dO, bh, scale, \
+                 excl, dq, dk, dv, dgate, ws, s)
+  if (dtype == PACK3D_BF16) return d == 96 ? P3D_BWD(__nv_bfloat16, 96) : P3D_BWD(__nv_bfloat16, 48);
+  return d == 96 ? P3D_BWD(float, 96) : P3D_BWD(float, 48);
+#undef P3D_BWD
+}
+
+}  // namespace p3d

@@ -1,0 +1,58 @@
+// Shared device helpers of the PACK3D CUDA path (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pack3d.h"
+
+namespace p3d {
+
+constexpr int kNbr = 27;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// status word slots (pack3d_index::status[0])
+constexpr int kStatusFirstError = 0;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+struct Coord {
+  int z, y, x;
+};
+__device__ __forceinline__ Coord decode(int32_t c) {
+  return Coord{c >> 20, (c >> 10) & 1023, c & 1023};
+}
+__device__ __forceinline__ int coord_axis(const Coord& c, int a) {
+  return a == 0 ? c.z : (a == 1 ? c.y : c.x);
+}
+
+// Records the first device-detected error in the status word (never traps).
+__device__ __forceinline__ void set_status(int32_t* status, int code) {
+  if (status) atomicCAS(status + kStatusFirstError, 0, code);
+}
+
+// (cos, sin) of coordinate value `cv` for rotation pair p of an axis third.
+__device__ __forceinline__ float2 rope_cs(const float* rope, int pairs, int cv, int p) {
+  return reinterpret_cast<const float2*>(rope)[cv * pairs + p];
+}
+
+// Is summary `m` (block box) within Chebyshev distance 1 of coordinate c?
+__device__ __forceinline__ bool block_is_near(const pack3d_index& ix, int m, const Coord& c) {
+  const int nbx = ix.geom.gx / ix.geom.bx, nby = ix.geom.gy / ix.geom.by;
+  const int mx = m % nbx, my = (m / nbx) % nby, mz = m / (nbx * nby);
+  const int lz = mz * ix.geom.bz, ly = my * ix.geom.by, lx = mx * ix.geom.bx;
+  return lz <= c.z + 1 && lz + ix.geom.bz - 1 >= c.z - 1 && ly <= c.y + 1 &&
+         ly + ix.geom.by - 1 >= c.y - 1 && lx <= c.x + 1 && lx + ix.geom.bx - 1 >= c.x - 1;
+}
+
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + __expf(-a)); }
+
+}  // namespace p3d

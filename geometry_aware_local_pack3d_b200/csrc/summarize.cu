@@ -1,0 +1,116 @@
+// Rotate-then-pool block summaries (project page "Geometry Matters in Packed 3D Attention",
+// Chapter 3 "Rotate first, then pool"; paper summary §3.2 and §B.5).
+//
+//   ksum[b,h,m] = (1/|S_m|) sum_{s} R(c_j) k[b,h,j],   vsum[b,h,m] = (1/|S_m|) sum_{s} v[b,h,j]
+//   with j = members[m][s], s the canonical slot.
+//
+// HBM-bound: every k and v row is read exactly once with 16-byte vector loads. One warp per
+// summary: lane l handles 16-byte chunk (l % C) of member rows s = l / C, l / C + R, ...
+// (C chunks per row, R = 32 / C rows per pass); the R partial sums are then combined in fixed
+// order with warp shuffles. The summation order depends on canonical slots only, never on
+// memory slots, so a coordinate-carrying repack gives bit-identical summaries.
+#include "common.cuh"
+#include "launch.h"
+#include "vec.cuh"
+
+namespace p3d {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __restrict__ k,
+                                                   const T* __restrict__ v, int64_t bh_count,
+                                                   T* __restrict__ ksum, T* __restrict__ vsum) {
+  constexpr int E = Vec<T>::E;
+  constexpr int C = D / E;       // chunks per row
+  constexpr int R = 32 / C;      // member rows per pass
+  constexpr int DA = D / 3;      // axis third
+  static_assert(DA % E == 0, "a 16-byte chunk must stay inside one axis third");
+  const int lane = threadIdx.x & 31;
+  const int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t M = ix.m;
+  if (task >= bh_count * M) return;
+  const int64_t bh = task / M;
+  const int m = (int)(task % M);
+  const int vol = ix.block_volume;
+  const int r = lane / C, c = lane % C;
+  const bool active = r < R;
+  const int axis = (c * E) / DA;
+  const int p0 = ((c * E) % DA) / 2;
+
+  float ak[E], av[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) ak[e] = av[e] = 0.f;
+
+  const T* kb = k + bh * ix.n * D;
+  const T* vb = v + bh * ix.n * D;
+  if (active) {
+#pragma unroll 4
+    for (int s = r; s < vol; s += R) {
+      const int j = ix.members[(int64_t)m * vol + s];
+      if (j < 0) continue;
+      const Coord cj = decode(ix.coord[j]);
+      const int cv = coord_axis(cj, axis);
+      float xk[E], xv[E];
+      Vec<T>::load(kb + (int64_t)j * D + c * E, xk);
+      Vec<T>::load(vb + (int64_t)j * D + c * E, xv);
+#pragma unroll
+      for (int e = 0; e < E; e += 2) {
+        const float2 cs = rope_cs(ix.rope, ix.rope_pairs, cv, p0 + e / 2);
+        ak[e] += xk[e] * cs.x - xk[e + 1] * cs.y;
+        ak[e + 1] += xk[e] * cs.y + xk[e + 1] * cs.x;
+        av[e] += xv[e];
+        av[e + 1] += xv[e + 1];
+      }
+    }
+  }
+  // combine the R partial sums in the fixed order r = 0, 1, ..., R-1 (each lane's own
+  // partials are read, never a value already combined in an earlier step)
+  float pk[E], pv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    pk[e] = ak[e];
+    pv[e] = av[e];
+  }
+#pragma unroll
+  for (int rr = 1; rr < R; ++rr) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      ak[e] += __shfl_sync(0xffffffffu, pk[e], (lane + rr * C) & 31);
+      av[e] += __shfl_sync(0xffffffffu, pv[e], (lane + rr * C) & 31);
+    }
+  }
+  if (r == 0) {
+    const int cnt = ix.count[m];
+    const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      ak[e] *= inv;
+      av[e] *= inv;
+    }
+    Vec<T>::store(ksum + (bh * M + m) * D + c * E, ak);
+    Vec<T>::store(vsum + (bh * M + m) * D + c * E, av);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_summarize(const pack3d_index& ix, const void* k, const void* v, int64_t bh,
+                             void* ksum, void* vsum, cudaStream_t s) {
+  const int64_t tasks = bh * ix.m;
+  const unsigned blocks = (unsigned)((tasks + 3) / 4);
+  k_summarize<T, D><<<blocks, 128, 0, s>>>(ix, static_cast<const T*>(k), static_cast<const T*>(v),
+                                            bh, static_cast<T*>(ksum), static_cast<T*>(vsum));
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t summarize_dispatch(const pack3d_index& ix, const void* k, const void* v, int dtype,
+                               int64_t bh, void* ksum, void* vsum, cudaStream_t s) {
+  const int d = ix.geom.head_dim;
+  if (dtype == PACK3D_BF16) {
+    if (d == 96) return launch_summarize<__nv_bfloat16, 96>(ix, k, v, bh, ksum, vsum, s);
+    return launch_summarize<__nv_bfloat16, 48>(ix, k, v, bh, ksum, vsum, s);
+  }
+  if (d == 96) return launch_summarize<float, 96>(ix, k, v, bh, ksum, vsum, s);
+  return launch_summarize<float, 48>(ix, k, v, bh, ksum, vsum, s);
+}
+
+}  // namespace p3d

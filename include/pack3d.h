@@ -1,0 +1,175 @@
+/*
+ * pack3d.h -- C ABI of the PACK3D attention operator (sm_100a).
+ *
+ * PACK3D ("Geometry Matters in Packed 3D Attention", Khan, Subrahmanya, Manjunath, NeurIPS
+ * 2026) attends over a 3D token grid whose tokens sit in memory in an arbitrary order
+ * (raster, Morton, block-contiguous, random). Each token keeps its integer grid coordinate
+ * c = (z, y, x) and every operation is indexed by that coordinate, never by the memory slot
+ * (project page amilworks.github.io/Pack3D, Chapter 1 and Chapter 3 Contracts 1-3). The
+ * operator has four parts:
+ *   - axial RoPE of q and k at c (head_dim split in three axis thirds z, y, x; base 10000);
+ *   - exact softmax attention over the 3x3x3 coordinate neighbourhood (<= 27 tokens);
+ *   - a global branch: rotated keys and values mean-pooled over contiguous 3D blocks into
+ *     summaries, and a softmax of each query over all summaries (optionally dropping the
+ *     summaries whose block meets the query's neighbourhood);
+ *   - a tokenwise mixer o = g * o_local + (1 - g) * o_global, g = sigmoid(gate logit).
+ *
+ * Conventions shared by every call:
+ *   - Tensors are dense, row-major [B, H, N, d] with N in MEMORY order (the packing);
+ *     gate logits are [B, H, N]; lse outputs are float32 [B, H, N]. Summaries are
+ *     [B, H, M, d] with M = number of blocks, block ids raster over the block grid.
+ *   - dtype: PACK3D_F32 or PACK3D_BF16 for q, k, v, gate, summaries, outputs and gradients.
+ *     All accumulation, softmax and logsumexp run in float32.
+ *   - Pointers marked "device" must be device (or managed) memory of the current device;
+ *     "host" pointers are host memory. The library never allocates device memory and never
+ *     takes ownership of a pointer; all buffers belong to the caller.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are asynchronous on
+ *     that stream unless stated otherwise. Argument errors are returned synchronously before
+ *     any launch; a launch failure returns PACK3D_ERR_CUDA.
+ *   - d (head_dim) must be 48 or 96 (a multiple of 6 is required by axial RoPE; other values
+ *     return PACK3D_ERR_UNSUPPORTED). The grid must be fully populated (N = Gz*Gy*Gx) and
+ *     divisible by the block extents.
+ */
+#ifndef PACK3D_H
+#define PACK3D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PACK3D_OK = 0,
+  PACK3D_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent arguments */
+  PACK3D_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build (d, partial grid) */
+  PACK3D_ERR_DUP_COORD = 3,     /* two tokens carry the same coordinate */
+  PACK3D_ERR_COORD_RANGE = 4,   /* a coordinate (or raster id) lies outside the grid */
+  PACK3D_ERR_ALIGN = 5,         /* a pointer is not 16-byte aligned */
+  PACK3D_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (status word) */
+  PACK3D_ERR_CUDA = 7,          /* a CUDA runtime call or kernel launch failed */
+  PACK3D_ERR_WORKSPACE = 8      /* caller's buffer smaller than the size query returned */
+} pack3d_status;
+
+typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
+
+/* attn_fwd / attn_bwd flag: drop, for each query, the summaries whose block box meets the
+ * cube [c-1, c+1]^3 around the query's coordinate. */
+#define PACK3D_EXCLUDE_NEAR 1u
+
+/* Geometry of a packed field: grid extents, block (summary) extents, RoPE plan. */
+typedef struct {
+  int32_t gz, gy, gx;   /* grid extents, each in [1, 1024] */
+  int32_t bz, by, bx;   /* block extents, each dividing the grid extent */
+  int32_t head_dim;     /* d: 48 or 96 */
+  float rope_base;      /* RoPE base per axis (10000 on the pages) */
+} pack3d_geom;
+
+/* Index tables of one packed field (one geometry, one packing). Filled by
+ * pack3d_build_index; all pointers point into the caller's device buffer `buf`.
+ * Coordinates are stored packed as (z << 20) | (y << 10) | x. */
+typedef struct {
+  pack3d_geom geom;
+  int64_t n;              /* tokens N = Gz*Gy*Gx */
+  int64_t m;              /* summaries M = (Gz/bz)*(Gy/by)*(Gx/bx) */
+  int32_t block_volume;   /* v = bz*by*bx */
+  int32_t rope_pairs;     /* d / 6 rotation pairs per axis */
+  int32_t rope_rows;      /* max(Gz, Gy, Gx): coordinates covered by the rotation table */
+  int32_t reserved;
+  int32_t* coord;         /* device [N]      packed coordinate of the token at each slot */
+  int32_t* inv;           /* device [Gz*Gy*Gx] memory slot of each raster site (-1: none) */
+  int32_t* nbr;           /* device [N, 27]  slot of c + delta_o, o = 9(dz+1)+3(dy+1)+(dx+1);
+                             -1 outside the grid */
+  int32_t* block_of;      /* device [N]      block id of each token */
+  int32_t* slot_of;       /* device [N]      canonical slot inside its block (raster) */
+  int32_t* members;       /* device [M, v]   slot of the member at each canonical slot */
+  int32_t* count;         /* device [M]      members present */
+  float* rope;            /* device [rope_rows, rope_pairs, 2] (cos, sin) of c * theta_p */
+  int32_t* status;        /* device [4]      status words written by kernels */
+} pack3d_index;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pack3d_strerror(pack3d_status s);
+
+/* Bytes of device memory pack3d_build_index needs for `n` tokens of geometry `g`
+ * (0 if the geometry is invalid). Host-only; launches nothing. */
+size_t pack3d_index_bytes(const pack3d_geom* g, int64_t n);
+
+/* Build the coordinate -> slot inverse map, the 27-neighbour table, the block-membership
+ * tables and the RoPE rotation table of a packed field.
+ *   Project page Ch.3 Contract 1 (neighbourhoods by coordinate, not adjacency in memory),
+ *   Ch.4 Proposition 2 (coordinates, edges, memberships and within-block slots travel with
+ *   each token); paper summary §B.1.
+ * g        host   geometry.
+ * coords   device int32 [n, 3] (z, y, x) of the token at each memory slot, or NULL;
+ * perm     device int64 [n] raster id (z*Gy + y)*Gx + x of the token at each slot, or NULL.
+ *          Exactly one of coords / perm must be non-NULL.
+ * buf      device buffer of at least pack3d_index_bytes(g, n) bytes, 256-byte aligned; it
+ *          holds every table and must outlive `out`'s use.
+ * out      host   filled with the table pointers and sizes.
+ * Errors: INVALID_ARG, UNSUPPORTED (n != Gz*Gy*Gx, d not 48/96), WORKSPACE, ALIGN, and --
+ * after one stream synchronisation at the end of the call -- DUP_COORD or COORD_RANGE
+ * detected by the kernels. */
+pack3d_status pack3d_build_index(const pack3d_geom* g, const int32_t* coords,
+                                 const int64_t* perm, int64_t n, void* buf, size_t buf_bytes,
+                                 pack3d_index* out, void* stream);
+
+/* Rotate-then-pool block summaries: ksum[m] = mean over members j of R(c_j) k_j and
+ * vsum[m] = mean of v_j, summed in canonical-slot order (project page Ch.3 "Rotate first,
+ * then pool"; paper summary §3.2, §B.5).
+ * k, v       device [B, H, N, d] dtype;  ksum, vsum device [B, H, M, d] dtype (outputs). */
+pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const void* v,
+                               int dtype, int batch, int heads, void* ksum, void* vsum,
+                               void* stream);
+
+/* PACK3D forward: local branch + global branch over (ksum, vsum) + sigmoid mixer
+ * (project page Ch.3 Contracts 1-3; paper summary §3.2, §3.3, §3.5).
+ * q, k, v    device [B, H, N, d] dtype;  gate device [B, H, N] dtype (logits a).
+ * ksum, vsum device [B, H, M, d] dtype from pack3d_summarize of the same k, v.
+ * scale      softmax scale tau (both branches); pass 1/sqrt(d) for the usual choice.
+ * flags      0 or PACK3D_EXCLUDE_NEAR.
+ * o          device [B, H, N, d] dtype (output).
+ * lse_loc, lse_glob  device float32 [B, H, N] or NULL: natural-log logsumexp of each
+ *            branch's logits (-inf where every summary is excluded).
+ * o_loc, o_glob      device [B, H, N, d] dtype or NULL: the two normalised branch outputs
+ *            (what the backward needs). A query whose summaries are all excluded has
+ *            o_glob = 0. */
+pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, int dtype, int batch, int heads, float scale,
+                              uint32_t flags, void* o, float* lse_loc, float* lse_glob,
+                              void* o_loc, void* o_glob, void* stream);
+
+/* Bytes of device workspace pack3d_attn_bwd needs. Host-only. */
+size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch, int heads);
+
+/* PACK3D backward: gradients of sum(dO * o) through the mixer, both softmax branches, the
+ * mean pooling and the axial RoPE (paper summary §3.4: the backward follows the forward's
+ * streamed access pattern).
+ * Inputs as in pack3d_attn_fwd plus the forward's saved o_loc, o_glob (dtype), lse_loc,
+ * lse_glob (float32) and the upstream gradient dO [B, H, N, d] dtype.
+ * Outputs dq, dk, dv [B, H, N, d] dtype and dgate [B, H, N] dtype (gradient w.r.t. the gate
+ * logit). workspace: device, >= pack3d_bwd_workspace_bytes bytes, 256-byte aligned;
+ * contents on entry are ignored. */
+pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
+                              const void* v, const void* gate, const void* ksum,
+                              const void* vsum, const void* o_loc, const void* o_glob,
+                              const float* lse_loc, const float* lse_glob, const void* dO,
+                              int dtype, int batch, int heads, float scale, uint32_t flags,
+                              void* dq, void* dk, void* dv, void* dgate, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Reads (after synchronising `stream`) and clears the index's device status word: OK, or
+ * the first device-detected error (DUP_COORD, COORD_RANGE, TIMEOUT). */
+pack3d_status pack3d_device_status(const pack3d_index* idx, void* stream);
+
+/* Kernel launches issued by the last pack3d_summarize / attn_fwd / attn_bwd call made on
+ * this host thread (for launch accounting). */
+int pack3d_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PACK3D_H */

@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle.
+
+Bar: index tables bit-exact; float32 I/O max-abs-err <= 1e-4; bfloat16 I/O max-abs-err <= 2e-2
+and relative L2 <= 5e-3 (o, lse, dq, dk, dv, dgate); coordinate-carrying repacks give outputs
+that are exact permutations of the raster output.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import inputs
+from oracle import pack3d_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-4
+BF16_ABS, BF16_REL = 2e-2, 5e-3
+
+
+def p3d():
+    import geometry_aware_local_pack3d_b200 as m
+    return m
+
+
+def assert_close(got, ref, dtype, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got), fin), f"{what}: non-finite pattern differs"
+    err = np.abs(got[fin] - ref[fin])
+    mx = float(err.max()) if err.size else 0.0
+    if dtype == "fp32":
+        assert mx <= F32_TOL, f"{what}: max-abs-err {mx:.3e} > {F32_TOL}"
+    else:
+        rel = float(np.linalg.norm(got[fin] - ref[fin]) / max(np.linalg.norm(ref[fin]), 1e-30))
+        assert mx <= BF16_ABS, f"{what}: max-abs-err {mx:.3e} > {BF16_ABS}"
+        assert rel <= BF16_REL, f"{what}: rel-L2 {rel:.3e} > {BF16_REL}"
+
+
+def tdtype(dt):
+    return torch.bfloat16 if dt == "bf16" else torch.float32
+
+
+def gpu_index(w, d, via="coords"):
+    m = p3d()
+    geom = m.make_geom(w["grid"], w["block"], d)
+    if via == "coords":
+        return m.pack3d_build_index(geom, coords=torch.from_numpy(w["coords"]).cuda())
+    return m.pack3d_build_index(geom, perm=torch.from_numpy(np.asarray(w["perm"])).cuda())
+
+
+def gpu_forward(w, exclude_near, save=False, ix=None):
+    m = p3d()
+    dt = tdtype(w["dtype"])
+    ix = ix or gpu_index(w, w["d"])
+    q, k, v, a = (w[n].to(dt).cuda().contiguous() for n in "qkva")
+    ksum, vsum = m.pack3d_summarize(ix, k, v)
+    out = m.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=exclude_near,
+                            save_for_backward=True if save else False)
+    torch.cuda.synchronize()
+    out.update(ksum=ksum, vsum=vsum, ix=ix, q=q, k=k, v=v, a=a)
+    return out
+
+
+def small(grid, block, B, H, d, dtype, packing, exclude_near=False, qkv_std=1.0, seed=0):
+    cfg = dict(grid=grid, block=block, batch=B, heads=H, d=d, dtype=dtype, packing=packing,
+               qkv_std=qkv_std, exclude_near=exclude_near)
+    return inputs.make_workload(cfg, seed=seed)
+
+
+def np64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+# ----------------------------------------------------------------------------- index tables
+def compare_tables(ix, w, ref):
+    n = len(w["coords"])
+    M, vol = ref["members"].shape
+    c = w["coords"].astype(np.int64)
+    packed = (c[:, 0] << 20) | (c[:, 1] << 10) | c[:, 2]
+    assert np.array_equal(ix.table("coord", (n,)).cpu().numpy(), packed)
+    assert np.array_equal(ix.table("inv", (len(ref["inv"]),)).cpu().numpy(), ref["inv"])
+    assert np.array_equal(ix.table("nbr", (n, 27)).cpu().numpy(), ref["nbr"])
+    assert np.array_equal(ix.table("block_of", (n,)).cpu().numpy(), ref["block_of"])
+    assert np.array_equal(ix.table("slot_of", (n,)).cpu().numpy(), ref["slot_of"])
+    assert np.array_equal(ix.table("members", (M, vol)).cpu().numpy(), ref["members"])
+    assert np.array_equal(ix.table("count", (M,)).cpu().numpy(), ref["count"])
+
+
+@pytest.mark.parametrize("grid,block", [((8, 8, 8), (2, 2, 2)), ((6, 10, 12), (3, 2, 4)),
+                                        ((1, 5, 7), (1, 5, 7))])
+@pytest.mark.parametrize("kind", inputs.PACKINGS)
+def test_index_tables_bit_exact(grid, block, kind):
+    if kind == "raster_block" and any(g % b for g, b in zip(grid, block)):
+        pytest.skip("block packing needs divisible grid")
+    w = small(grid, block, 1, 1, 48, "fp32", kind)
+    ref = orc.build_index(w["coords"], grid, block)
+    compare_tables(gpu_index(w, 48), w, ref)
+    compare_tables(gpu_index(w, 48, via="perm"), w, ref)
+
+
+@pytest.mark.parametrize("kind", inputs.PACKINGS)
+def test_index_tables_bit_exact_65k_field(kind):
+    w = dict(inputs.WORKLOADS["field65k_repack_bf16"])
+    perm = inputs.packing(kind, w["grid"], w["block"], seed=1)
+    w.update(perm=perm, coords=inputs.coords_of(perm, w["grid"]))
+    ref = orc.build_index(w["coords"], w["grid"], w["block"])
+    compare_tables(gpu_index(w, 96), w, ref)
+
+
+def test_rope_table_matches_theta_plan():
+    w = small((4, 6, 9), (1, 1, 1), 1, 1, 96, "fp32", "raster")
+    ix = gpu_index(w, 96)
+    tab = ix.rope_table().cpu().numpy().astype(np.float64)
+    theta = orc.rope_theta(96)
+    ang = np.arange(9)[:, None] * theta[None, :]
+    assert np.abs(tab[..., 0] - np.cos(ang)).max() < 1e-6
+    assert np.abs(tab[..., 1] - np.sin(ang)).max() < 1e-6
+
+
+def test_index_errors_are_reported():
+    m = p3d()
+    geom = m.make_geom((2, 2, 2), (1, 1, 1), 48)
+    c = torch.from_numpy(inputs.coords_of(np.arange(8), (2, 2, 2))).cuda()
+    dup = c.clone()
+    dup[3] = dup[5]
+    with pytest.raises(m.Pack3DError) as e:
+        m.pack3d_build_index(geom, coords=dup)
+    assert e.value.status == 3
+    bad = c.clone()
+    bad[2, 1] = 2
+    with pytest.raises(m.Pack3DError) as e:
+        m.pack3d_build_index(geom, coords=bad)
+    assert e.value.status == 4
+    with pytest.raises(m.Pack3DError) as e:
+        m.pack3d_build_index(geom, perm=torch.tensor([0, 1, 2, 3, 4, 5, 6, 8]).cuda())
+    assert e.value.status == 4
+    # the library stays usable after reported errors
+    m.pack3d_build_index(geom, coords=c)
+
+
+# -------------------------------------------------------------------------------- forward
+@pytest.mark.parametrize("dtype,d", [("fp32", 48), ("fp32", 96), ("bf16", 48), ("bf16", 96)])
+def test_summaries(dtype, d):
+    w = small((4, 8, 8), (2, 4, 4), 2, 2, d, dtype, "random")
+    g = gpu_forward(w, False)
+    ix = orc.build_index(w["coords"], w["grid"], w["block"])
+    ks, vs = orc.summaries(orc.rope(w["k"].numpy(), w["coords"]), w["v"].numpy(), ix["members"])
+    assert_close(np64(g["ksum"]), ks, dtype, "ksum")
+    assert_close(np64(g["vsum"]), vs, dtype, "vsum")
+
+
+def full_compare(w, exclude_near, what=""):
+    g = gpu_forward(w, exclude_near, save=True)
+    ref = orc.forward(w["q"].numpy(), w["k"].numpy(), w["v"].numpy(), w["a"].numpy(),
+                      w["coords"], w["grid"], w["block"], exclude_near=exclude_near)
+    for key in ("o", "o_loc", "o_glob", "lse_loc", "lse_glob"):
+        assert_close(np64(g[key]), ref[key], w["dtype"], f"{what}{key}")
+    return g, ref
+
+
+def test_forward_tiny_field_fp32():
+    # the 8x8x8 / 2x2x2 field of the two-indices lab, fp32, d48, raster
+    w = inputs.make_workload("tiny_8x8x8_fp32")
+    full_compare(w, False)
+
+
+@pytest.mark.parametrize("kind", inputs.PACKINGS)
+@pytest.mark.parametrize("exclude_near", [False, True])
+def test_forward_bf16_d96_packings(kind, exclude_near):
+    w = small((8, 8, 16), (4, 4, 4), 1, 2, 96, "bf16", kind, qkv_std=96 ** -0.5)
+    full_compare(w, exclude_near, f"{kind}/{exclude_near}/")
+
+
+@pytest.mark.parametrize("dtype,d", [("fp32", 96), ("bf16", 48), ("fp32", 48)])
+def test_forward_other_dtypes(dtype, d):
+    w = small((6, 8, 10), (3, 2, 5), 2, 1, d, dtype, "morton")
+    full_compare(w, True, f"{dtype}/{d}/")
+
+
+def test_forward_all_summaries_excluded():
+    w = small((4, 4, 4), (2, 2, 2), 1, 2, 48, "fp32", "random")
+    g, ref = full_compare(w, True)
+    lse = g["lse_glob"].cpu().numpy()
+    assert np.isneginf(lse).sum() == np.isneginf(ref["lse_glob"]).sum() > 0
+    assert np.all(g["o_glob"].cpu().numpy()[np.isneginf(lse)] == 0)
+
+
+def test_forward_unit_blocks_and_thin_grid():
+    w = small((1, 6, 5), (1, 1, 1), 1, 1, 48, "fp32", "random")
+    full_compare(w, False)
+    full_compare(w, True)
+
+
+def sampled_rows(n, count, seed=0):
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 63, 64, 127, 128, n - 129, n - 128, n - 1]
+    return np.unique(np.concatenate([rng.choice(n, count, replace=False), edge]))
+
+
+def sampled_compare(w, exclude_near, heads=((0, 0), (-1, -1)), count=96):
+    g = gpu_forward(w, exclude_near, save=True)
+    idx = orc.build_index(w["coords"], w["grid"], w["block"])
+    rows = sampled_rows(len(w["coords"]), count)
+    for (b, h) in heads:
+        sl = lambda t: t[b:b + 1 if b != -1 else None, h:h + 1 if h != -1 else None].numpy()  # noqa: E731
+        ref = orc.forward(sl(w["q"]), sl(w["k"]), sl(w["v"]), sl(w["a"]), w["coords"], w["grid"],
+                          w["block"], exclude_near=exclude_near, index=idx, rows=rows)
+        for key in ("o", "lse_loc", "lse_glob", "o_loc", "o_glob"):
+            gv = g[key][b, h][rows] if key.startswith("o") else g[key][b, h][rows]
+            assert_close(np64(gv), ref[key][0, 0], w["dtype"], f"{key}[{b},{h}]")
+        assert_close(np64(g["ksum"][b, h]), ref["ksum"][0, 0], w["dtype"], "ksum")
+    return g
+
+
+def test_forward_65k_field_sampled():
+    sampled_compare(inputs.make_workload("field65k_bf16"), False)
+
+
+def test_forward_262k_field_sampled():
+    sampled_compare(inputs.make_workload("field262k_bf16"), False, heads=((0, 3),), count=64)
+
+
+def test_repacking_equivariance_is_exact_65k_field():
+    # four coordinate-carrying packings: outputs are exact permutations of the raster output
+    outs = {}
+    for kind in inputs.PACKINGS:
+        w = inputs.make_workload("field65k_repack_bf16", packing_kind=kind)
+        g = gpu_forward(w, True)
+        outs[kind] = inputs.unpack(g["o"].cpu(), w["perm"])
+        del g
+    for kind in inputs.PACKINGS:
+        assert torch.equal(outs[kind], outs["raster"]), kind
+    # and the raster output itself meets the oracle on sampled rows
+    w = inputs.make_workload("field65k_repack_bf16", packing_kind="random")
+    sampled_compare(w, True, heads=((1, 5),), count=48)
+
+
+# ------------------------------------------------------------------------------- backward
+def gpu_backward(w, exclude_near):
+    m = p3d()
+    g = gpu_forward(w, exclude_near, save=True)
+    dO = inputs.pack(inputs.upstream_grad(w["batch"], w["heads"], w["grid"], w["d"]), w["perm"])
+    if w["dtype"] == "bf16":
+        dO = dO.to(torch.bfloat16).to(torch.float32)
+    dOd = dO.to(tdtype(w["dtype"])).cuda().contiguous()
+    gr = m.pack3d_attn_bwd(g["ix"], g["q"], g["k"], g["v"], g["a"], g["ksum"], g["vsum"], g, dOd,
+                           exclude_near=exclude_near)
+    torch.cuda.synchronize()
+    return gr, dO
+
+
+@pytest.mark.parametrize("dtype,d,exclude_near", [("fp32", 48, False), ("fp32", 96, True),
+                                                  ("bf16", 96, True), ("bf16", 48, False)])
+def test_backward_full(dtype, d, exclude_near):
+    w = small((4, 4, 8), (2, 2, 4), 1, 2, d, dtype, "random",
+              qkv_std=1.0 if dtype == "fp32" else d ** -0.5)
+    gr, dO = gpu_backward(w, exclude_near)
+    ref = orc.backward(w["q"].numpy(), w["k"].numpy(), w["v"].numpy(), w["a"].numpy(),
+                       dO.numpy(), w["coords"], w["grid"], w["block"], exclude_near=exclude_near)
+    for key, rk in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dgate", "da")):
+        assert_close(np64(gr[key]), ref[rk], dtype, key)
+
+
+def test_backward_65k_field_sampled():
+    w = inputs.make_workload("field65k_fwdbwd_bf16")
+    gr, dO = gpu_backward(w, False)
+    b, h = 1, 6
+    sl = lambda t: t[b:b + 1, h:h + 1].numpy()  # noqa: E731
+    rows = sampled_rows(len(w["coords"]), 24)
+    idx = orc.build_index(w["coords"], w["grid"], w["block"])
+    ref = orc.backward_rows(sl(w["q"]), sl(w["k"]), sl(w["v"]), sl(w["a"]), sl(dO), w["coords"],
+                            w["grid"], w["block"], qrows=rows, krows=rows, index=idx)
+    assert_close(np64(gr["dq"][b, h][rows]), ref["dq"][0, 0], "bf16", "dq")
+    assert_close(np64(gr["dgate"][b, h][rows]), ref["da"][0, 0], "bf16", "dgate")
+    assert_close(np64(gr["dk"][b, h][rows]), ref["dk"][0, 0], "bf16", "dk")
+    assert_close(np64(gr["dv"][b, h][rows]), ref["dv"][0, 0], "bf16", "dv")
