@@ -1,5 +1,7 @@
 // C ABI of the PACK3D operator: argument checks and dispatch to the kernels.
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -21,6 +23,13 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
                               void* dv, void* dgate, void* ws, cudaStream_t s);
 size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh);
+cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                                const void* v, int dtype, int64_t bh, float scale, void* o_loc,
+                                float* lse_loc, cudaStream_t s);
+cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
+                               const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
+                               float scale, int excl, void* o, float* lse_glob, void* o_glob,
+                               cudaStream_t s);
 }  // namespace p3d
 
 using namespace p3d;
@@ -47,6 +56,17 @@ pack3d_status check_rows(std::initializer_list<const void*> ptrs) {
 }
 
 pack3d_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
+
+// bf16 runs the global branch on tcgen05 tensor cores unless PACK3D_BF16_PATH=simt selects the
+// CUDA-core kernels (both compute the whole operator).
+bool bf16_tensor_path() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("PACK3D_BF16_PATH");
+    v = (e && strcmp(e, "simt") == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
 }  // namespace
 
 extern "C" const char* pack3d_strerror(pack3d_status s) {
@@ -92,6 +112,16 @@ extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q,
   if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
   const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
   const int64_t bh = (int64_t)batch * heads;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == PACK3D_BF16 && bf16_tensor_path()) {
+    // local branch first (its normalised output goes to o_loc, or to o until it is mixed),
+    // then the tensor-core global branch with the mixer in its epilogue
+    void* ol = o_loc ? o_loc : o;
+    cudaError_t e = local_simt_dispatch(*idx, q, k, v, dtype, bh, scale, ol, lse_loc, s);
+    if (e != cudaSuccess) return PACK3D_ERR_CUDA;
+    return cuda_status(global_tc_dispatch(*idx, q, gate, ksum, vsum, ol, bh, scale, excl, o,
+                                          lse_glob, o_glob, s));
+  }
   return cuda_status(fwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, dtype, bh, scale, excl,
                                        o, lse_loc, lse_glob, o_loc, o_glob,
                                        static_cast<cudaStream_t>(stream)));

@@ -532,6 +532,25 @@ cudaError_t fwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
 #undef P3D_FWD
 }
 
+cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                                const void* v, int dtype, int64_t bh, float scale, void* o_loc,
+                                float* lse_loc, cudaStream_t s) {
+  const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
+  const int d = ix.geom.head_dim;
+#define P3D_LOC(T, D)                                                                         \
+  k_local_fwd<T, D><<<grid, 128, 0, s>>>(ix, static_cast<const T*>(q), static_cast<const T*>(k), \
+                                          static_cast<const T*>(v), scale, static_cast<T*>(o_loc), \
+                                          lse_loc)
+  if (dtype == PACK3D_BF16) {
+    if (d == 96) P3D_LOC(__nv_bfloat16, 96); else P3D_LOC(__nv_bfloat16, 48);
+  } else {
+    if (d == 96) P3D_LOC(float, 96); else P3D_LOC(float, 48);
+  }
+#undef P3D_LOC
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
                               const void* v, const void* gate, const void* ksum,
                               const void* vsum, const void* o_loc, const void* o_glob,

@@ -1,0 +1,538 @@
+// Global branch of PACK3D attention on tcgen05 tensor cores, with the sigmoid mixer fused into
+// the epilogue (bf16 I/O, head_dim 48 or 96).
+//
+// Project page "Geometry Matters in Packed 3D Attention", Chapter 3 Contract 2: every query
+// attends to all block summaries; paper summary §3.5: a streamed online softmax, no dense
+// token x summary score matrix in memory; §3.3: o = g o_loc + (1 - g) o_glob, g = sigmoid(a).
+//
+// Work unit: 256 consecutive memory rows of one (batch, head) = two 128-row query tiles that
+// share every summary chunk (halves the L2 reads of the summaries). Persistent CTAs walk the
+// units round-robin. Warp roles (384 threads):
+//   warps 0-3  softmax of tile 0 (thread = row, TMEM lanes 0..127)
+//   warps 4-7  softmax of tile 1
+//   warps 8-9  query producer: coalesced 16-byte loads of q, axial RoPE, bf16 rows into the
+//              K-major shared-memory A operand (double-buffered across units)
+//   warp 10    MMA issuer (one thread) and TMEM owner
+//   warp 11    TMA producer: 128-summary chunks of ksum / vsum into a 2-stage ring
+// Per chunk j and tile t:  S_t = q~_t K_j^T (SS MMA, fp32 in TMEM) -> softmax threads turn S_t
+// into P_t = exp2(s - m) in bf16, written over S_t in TMEM -> O_t += P_t V_j (TS MMA).
+// The running max uses a lazy rescale: O_t is corrected in TMEM only when a row's max grows by
+// more than 2^8, so the common case touches O once at the end.
+// The summary order is the same for every query (block ids ascending) and rows never interact,
+// so a coordinate-carrying repack permutes the output bit for bit.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+
+namespace p3d {
+
+namespace gtc {
+constexpr int kRows = 128;        // rows per tile
+constexpr int kTiles = 2;         // tiles per unit
+constexpr int kChunk = 128;       // summaries per chunk
+constexpr int kStages = 2;        // summary ring depth
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D> struct Smem {
+  static constexpr int kTileBytes = kRows * D * 2;       // one q tile / one summary chunk
+  static constexpr int kQ = 0;                           // [2 buffers][2 tiles]
+  static constexpr int kK = kQ + 2 * kTiles * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kBytes = kBar + 256;
+};
+
+// barrier slots
+enum {
+  B_QFULL = 0,   // [2]
+  B_QEMPTY = 2,  // [2]
+  B_KVFULL = 4,  // [kStages]
+  B_KVEMPTY = 6, // [kStages]
+  B_SFULL = 8,   // [2] per tile
+  B_PFULL = 10,  // [2]
+  B_OFULL = 12,  // [2]
+  B_OFREE = 14,  // [2]
+  B_DONE = 16,
+  B_COUNT = 17
+};
+
+struct Params {
+  pack3d_index ix;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* gate;
+  const __nv_bfloat16* o_loc;  // may alias o
+  __nv_bfloat16* o;
+  __nv_bfloat16* o_glob;       // optional
+  float* lse_glob;             // optional
+  float scale_log2;            // tau * log2(e)
+  int exclude_near;
+  int64_t units;               // (batch*heads) * units_per_bh
+  int units_per_bh;
+  int n_chunks;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct Abort {
+  volatile int* flag;
+  int32_t* status;
+  __device__ bool wait(uint64_t* bar, uint32_t parity) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!tc::mbar_try_wait(bar, parity)) {
+      if (*flag) return false;
+      if (clock64() - t0 > 4000000000LL) {
+        *flag = 1;
+        set_status(status, PACK3D_ERR_TIMEOUT);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+}  // namespace gtc
+
+template <int D>
+__global__ void __launch_bounds__(gtc::kThreads, 1)
+    k_global_tc(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                const gtc::Params P) {
+  using namespace gtc;
+  using S = Smem<D>;
+  constexpr int KC = D / 8;  // 16-byte chunks per row
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  Abort ab{abort_flag, P.ix.status};
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars[B_QFULL + i], 64);
+      tc::mbar_init(&bars[B_QEMPTY + i], 1);
+      tc::mbar_init(&bars[B_SFULL + i], 1);
+      tc::mbar_init(&bars[B_PFULL + i], 128);
+      tc::mbar_init(&bars[B_OFULL + i], 1);
+      tc::mbar_init(&bars[B_OFREE + i], 128);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&bars[B_KVFULL + i], 1);
+      tc::mbar_init(&bars[B_KVEMPTY + i], 1);
+    }
+    tc::mbar_init(&bars[B_DONE], 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 10) tc::tmem_alloc(tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int64_t N = P.ix.n;
+  const int M = (int)P.ix.m;
+  const int NC = P.n_chunks;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;
+    const int rin = (warp & 3) * 32 + lane;
+    const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_col = t * 128, o_col = 256 + t * 128;
+    int pc = 0;
+    for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
+      const int64_t bh = u / P.units_per_bh;
+      const int64_t row = (u % P.units_per_bh) * (kRows * kTiles) + t * kRows + rin;
+      const bool valid = row < N;
+      // summaries excluded for this row: blocks meeting the cube [c-1, c+1]^3, kept as block
+      // coordinate ranges [z0,z1] x [y0,y1] x [x0,x1] (empty when exclusion is off)
+      int z0 = 0, z1 = -1, y0 = 0, y1 = -1, x0 = 0, x1 = -1;
+      const int nby = P.ix.geom.gy / P.ix.geom.by, nbx = P.ix.geom.gx / P.ix.geom.bx;
+      if (P.exclude_near && valid) {
+        const Coord c = decode(P.ix.coord[row]);
+        const pack3d_geom& g = P.ix.geom;
+        z0 = max(c.z - 1, 0) / g.bz; z1 = min(c.z + 1, g.gz - 1) / g.bz;
+        y0 = max(c.y - 1, 0) / g.by; y1 = min(c.y + 1, g.gy - 1) / g.by;
+        x0 = max(c.x - 1, 0) / g.bx; x1 = min(c.x + 1, g.gx - 1) / g.bx;
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < NC; ++j) {
+        const uint32_t it = (uint32_t)(pc * NC + j);
+        if (!ab.wait(&bars[B_SFULL + t], it & 1)) break;
+        tc::tc_fence_after();
+        const int m0 = j * kChunk;
+        const int ncol = min(kChunk, M - m0);
+        // exclusion bitmask of this chunk
+        uint32_t xm[4] = {0u, 0u, 0u, 0u};
+        bool any_x = false;
+        for (int mz = z0; mz <= z1; ++mz)
+          for (int my = y0; my <= y1; ++my)
+            for (int mx = x0; mx <= x1; ++mx) {
+              const int cidx = (mz * nby + my) * nbx + mx - m0;
+              if (cidx >= 0 && cidx < kChunk) {
+                const uint32_t bit = 1u << (cidx & 31);
+                const int w = cidx >> 5;
+                xm[0] |= w == 0 ? bit : 0u;
+                xm[1] |= w == 1 ? bit : 0u;
+                xm[2] |= w == 2 ? bit : 0u;
+                xm[3] |= w == 3 ? bit : 0u;
+                any_x = true;
+              }
+            }
+        const bool masked = any_x || ncol < kChunk;
+        // pass 1: row max of this chunk (log2 domain)
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int c0 = 0; c0 < kChunk; c0 += 32) {
+          uint32_t r[32];
+          tc::tmem_ld32(tl + s_col + c0, r);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            float s = __uint_as_float(r[k]) * P.scale_log2;
+            if (masked && (((xm[c0 >> 5] >> k) & 1u) || c0 + k >= ncol)) s = -INFINITY;
+            cmax = fmaxf(cmax, s);
+          }
+        }
+        const float m_new = fmaxf(m_run, cmax);
+        const bool need = m_new > m_run + kRescaleLog2;  // false while everything is masked
+        if (__any_sync(0xffffffffu, need) && j > 0) {
+          // O_t holds sum_{<j} P V with the old max: wait for the previous PV, then rescale
+          if (!ab.wait(&bars[B_OFULL + t], (it - 1) & 1)) break;
+          tc::tc_fence_after();
+          const float f = need ? ex2(m_run - m_new) : 1.f;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            tc::tmem_ld32(tl + o_col + c0, r);
+            tc::tmem_wait_ld();
+            uint32_t a[16], b[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              a[k] = __float_as_uint(__uint_as_float(r[k]) * f);
+              b[k] = __float_as_uint(__uint_as_float(r[16 + k]) * f);
+            }
+            tc::tmem_st16(tl + o_col + c0, a);
+            tc::tmem_st16(tl + o_col + c0 + 16, b);
+          }
+          tc::tmem_wait_st();
+        }
+        if (need) {
+          l_run *= ex2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        // pass 2: P = exp2(s - m) as bf16, written over the first half of S_t
+        float lsum = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kChunk; c0 += 32) {
+          uint32_t r[32];
+          tc::tmem_ld32(tl + s_col + c0, r);
+          tc::tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            float s0 = __uint_as_float(r[k]) * P.scale_log2;
+            float s1 = __uint_as_float(r[k + 1]) * P.scale_log2;
+            if (masked) {
+              if (((xm[c0 >> 5] >> k) & 1u) || c0 + k >= ncol) s0 = -INFINITY;
+              if (((xm[c0 >> 5] >> (k + 1)) & 1u) || c0 + k + 1 >= ncol) s1 = -INFINITY;
+            }
+            const float p0 = ex2(s0 - m_use), p1 = ex2(s1 - m_use);
+            lsum += p0 + p1;
+            p[k >> 1] = tc::pack_bf16(p0, p1);
+          }
+          tc::tmem_st16(tl + s_col + (c0 >> 1), p);
+        }
+        l_run += lsum;
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bars[B_PFULL + t]);
+      }
+      if (*abort_flag) break;
+      // epilogue: o_glob = O / l, lse, mixer
+      const uint32_t last = (uint32_t)(pc * NC + NC - 1);
+      if (!ab.wait(&bars[B_OFULL + t], last & 1)) break;
+      tc::tc_fence_after();
+      // O row -> o_glob = O / l, kept packed as bf16 pairs; TMEM is released right after
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint32_t gp[(D + 31) / 32 * 16];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tc::tmem_ld32(tl + o_col + c0, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          gp[c0 / 2 + k] = tc::pack_bf16(__uint_as_float(r[2 * k]) * inv_l,
+                                         __uint_as_float(r[2 * k + 1]) * inv_l);
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bars[B_OFREE + t]);
+      if (valid) {
+        const int64_t grow = bh * N + row;
+        if (P.lse_glob)
+          P.lse_glob[grow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+        const float a = __bfloat162float(P.gate[grow]);
+        const float g = 1.f / (1.f + __expf(-a));
+        const uint4* ol = reinterpret_cast<const uint4*>(P.o_loc + grow * D);
+        uint4* oo = reinterpret_cast<uint4*>(P.o + grow * D);
+        uint4* og = P.o_glob ? reinterpret_cast<uint4*>(P.o_glob + grow * D) : nullptr;
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+          const uint4 lv = ol[c];
+          const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+          uint32_t outw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t gw = gp[4 * c + k];
+            const float g0 = __uint_as_float(gw << 16), g1 = __uint_as_float(gw & 0xffff0000u);
+            const float l0 = __uint_as_float(lw[k] << 16);
+            const float l1 = __uint_as_float(lw[k] & 0xffff0000u);
+            outw[k] = tc::pack_bf16(g * l0 + (1.f - g) * g0, g * l1 + (1.f - g) * g1);
+          }
+          oo[c] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          if (og) og[c] = make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
+        }
+      }
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------------ query producer
+    const int ptid = tid - 256;  // 64 producer threads
+    constexpr int DA = D / 3;
+    int pc = 0;
+    for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
+      const int b = pc & 1;
+      if (pc >= 2 && !ab.wait(&bars[B_QEMPTY + b], ((pc >> 1) - 1) & 1)) break;
+      const int64_t bh = u / P.units_per_bh;
+      const int64_t row0 = (u % P.units_per_bh) * (kRows * kTiles);
+      uint8_t* qb = smem + S::kQ + b * kTiles * S::kTileBytes;
+      for (int c = ptid; c < kRows * kTiles * KC; c += 64) {
+        const int r = c / KC, kc = c % KC;
+        const int64_t row = row0 + r;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (row < N) {
+          const uint4 x = *reinterpret_cast<const uint4*>(P.q + (bh * N + row) * D + kc * 8);
+          const Coord cc = decode(P.ix.coord[row]);
+          const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
+          const int cv = coord_axis(cc, axis);
+          const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
+          uint32_t xo[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 cs = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, p0 + k);
+            const float e0 = __uint_as_float(xin[k] << 16);
+            const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+            xo[k] = tc::pack_bf16(e0 * cs.x - e1 * cs.y, e0 * cs.y + e1 * cs.x);
+          }
+          w = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+        }
+        const int t = r / kRows, rr = r % kRows;
+        *reinterpret_cast<uint4*>(qb + t * S::kTileBytes + kc * 2048 + (rr >> 3) * 128 +
+                                  (rr & 7) * 16) = w;
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[B_QFULL + b]);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
+      const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
+      int pc = 0;
+      uint32_t kv_it = 0;
+      bool issued = false;
+      for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x, ++pc) {
+        const int b = pc & 1;
+        if (!ab.wait(&bars[B_QFULL + b], (pc >> 1) & 1)) break;
+        tc::tc_fence_after();
+        const uint32_t qaddr = tc::smem_u32(smem + S::kQ + b * kTiles * S::kTileBytes);
+        bool ok = true;
+        for (int j = 0; j < P.n_chunks && ok; ++j, ++kv_it) {
+          const int st = kv_it % kStages;
+          if (!ab.wait(&bars[B_KVFULL + st], (kv_it / kStages) & 1)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t kaddr = tc::smem_u32(smem + S::kK + st * S::kTileBytes);
+          const uint32_t vaddr = tc::smem_u32(smem + S::kV + st * S::kTileBytes);
+          const uint32_t it = (uint32_t)(pc * P.n_chunks + j);
+          for (int t = 0; t < kTiles; ++t) {
+            // S_t / P_t is free once the previous PV on this tile has completed
+            if (it > 0 && !ab.wait(&bars[B_OFULL + t], (it - 1) & 1)) { ok = false; break; }
+            tc::tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint64_t a = tc::smem_desc(qaddr + t * S::kTileBytes + ks * 4096, 2048, 128);
+              const uint64_t bd = tc::smem_desc(kaddr + ks * 4096, 2048, 128);
+              tc::mma_ss(tbase + t * 128, a, bd, id_qk, ks > 0);
+            }
+            tc::tc_commit(&bars[B_SFULL + t]);
+            issued = true;
+          }
+          if (!ok) break;
+          for (int t = 0; t < kTiles; ++t) {
+            if (!ab.wait(&bars[B_PFULL + t], it & 1)) { ok = false; break; }
+            if (j == 0 && pc > 0 && !ab.wait(&bars[B_OFREE + t], (pc - 1) & 1)) { ok = false; break; }
+            tc::tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < kChunk / 16; ++ks) {
+              const uint64_t bd = tc::smem_desc(vaddr + ks * 256, 128, 2048);
+              tc::mma_ts(tbase + 256 + t * 128, tbase + t * 128 + ks * 8, bd, id_pv,
+                         (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            tc::tc_commit(&bars[B_OFULL + t]);
+          }
+          if (!ok) break;
+          tc::tc_commit(&bars[B_KVEMPTY + st]);
+        }
+        if (!ok) break;
+        tc::tc_commit(&bars[B_QEMPTY + b]);
+      }
+      // every MMA issued by this thread has completed before TMEM is released
+      if (issued) {
+        tc::tc_commit(&bars[B_DONE]);
+        tc::mbar_wait(&bars[B_DONE], 0, 4000000000LL);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&map_k);
+      tc::tma_prefetch_desc(&map_v);
+      uint32_t kv_it = 0;
+      for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x) {
+        const int64_t bh = u / P.units_per_bh;
+        bool ok = true;
+        for (int j = 0; j < P.n_chunks; ++j, ++kv_it) {
+          const int st = kv_it % kStages;
+          if (kv_it >= (uint32_t)kStages &&
+              !ab.wait(&bars[B_KVEMPTY + st], ((kv_it / kStages) - 1) & 1)) { ok = false; break; }
+          tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kTileBytes);
+          const int y = (int)(bh * M + j * kChunk);
+          uint8_t* kd = smem + S::kK + st * S::kTileBytes;
+          uint8_t* vd = smem + S::kV + st * S::kTileBytes;
+#pragma unroll
+          for (int kc = 0; kc < KC; ++kc) {
+            tc::tma_load_2d(kd + kc * 2048, &map_k, 8 * kc, y, &bars[B_KVFULL + st]);
+            tc::tma_load_2d(vd + kc * 2048, &map_v, 8 * kc, y, &bars[B_KVFULL + st]);
+          }
+        }
+        if (!ok) break;
+      }
+      // the last loads issued to each stage have landed before the CTA may exit
+      for (uint32_t k = (kv_it > (uint32_t)kStages ? kv_it - kStages : 0); k < kv_it; ++k)
+        tc::mbar_wait(&bars[B_KVFULL + (k % kStages)], (k / kStages) & 1, 4000000000LL);
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 10) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, D] bf16 row-major viewed as 2D; box = 8 columns x 128 rows (one 16-byte column of
+// core matrices), no swizzle.
+bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {8, 128};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+}  // namespace
+
+template <int D>
+cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* gate,
+                             const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
+                             float scale, int excl, void* o, float* lse_glob, void* o_glob,
+                             cudaStream_t s) {
+  using namespace gtc;
+  CUtensorMap mk, mv;
+  if (!encode_rows(&mk, ksum, bh * ix.m, D) || !encode_rows(&mv, vsum, bh * ix.m, D))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_global_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<D>::kBytes) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  Params p;
+  p.ix = ix;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.o_loc = static_cast<const __nv_bfloat16*>(o_loc);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_glob = static_cast<__nv_bfloat16*>(o_glob);
+  p.lse_glob = lse_glob;
+  p.scale_log2 = scale * kLog2e;
+  p.exclude_near = excl;
+  p.units_per_bh = (int)((ix.n + kRows * kTiles - 1) / (kRows * kTiles));
+  p.units = bh * p.units_per_bh;
+  p.n_chunks = (int)((ix.m + kChunk - 1) / kChunk);
+  const int grid = (int)(p.units < sm_count() ? p.units : sm_count());
+  k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mk, mv, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
+                               const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
+                               float scale, int excl, void* o, float* lse_glob, void* o_glob,
+                               cudaStream_t s) {
+  if (ix.geom.head_dim == 96)
+    return launch_global_tc<96>(ix, q, gate, ksum, vsum, o_loc, bh, scale, excl, o, lse_glob,
+                                o_glob, s);
+  return launch_global_tc<48>(ix, q, gate, ksum, vsum, o_loc, bh, scale, excl, o, lse_glob,
+                              o_glob, s);
+}
+
+}  // namespace p3d

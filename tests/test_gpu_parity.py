@@ -277,3 +277,27 @@ def test_backward_65k_field_sampled():
     assert_close(np64(gr["dgate"][b, h][rows]), ref["da"][0, 0], "bf16", "dgate")
     assert_close(np64(gr["dk"][b, h][rows]), ref["dk"][0, 0], "bf16", "dk")
     assert_close(np64(gr["dv"][b, h][rows]), ref["dv"][0, 0], "bf16", "dv")
+
+
+# ------------------------------------------------------------- bf16 tensor-core path edges
+@pytest.mark.parametrize("d", [48, 96])
+def test_bf16_all_summaries_excluded(d):
+    w = small((4, 4, 4), (2, 2, 2), 2, 2, d, "bf16", "random", qkv_std=d ** -0.5)
+    g, ref = full_compare(w, True)
+    lse = g["lse_glob"].cpu().numpy()
+    assert np.isneginf(lse).sum() == np.isneginf(ref["lse_glob"]).sum() > 0
+    assert np.all(g["o_glob"].float().cpu().numpy()[np.isneginf(lse)] == 0)
+
+
+@pytest.mark.parametrize("exclude_near", [False, True])
+def test_bf16_ragged_rows_and_summary_chunks(exclude_near):
+    # N = 1,920 (7.5 units of 256 rows) and M = 240 (one full and one partial chunk of 128)
+    w = small((8, 12, 20), (2, 2, 2), 1, 3, 96, "bf16", "morton", qkv_std=96 ** -0.5)
+    full_compare(w, exclude_near)
+
+
+def test_bf16_thin_grid_unit_blocks():
+    # M = N = 105: every token is its own summary; one partial unit
+    w = small((3, 5, 7), (1, 1, 1), 1, 2, 48, "bf16", "random", qkv_std=48 ** -0.5)
+    full_compare(w, True)
+    full_compare(w, False)
