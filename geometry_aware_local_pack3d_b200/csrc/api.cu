@@ -26,6 +26,9 @@ size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh);
 cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
                                 const void* v, int dtype, int64_t bh, float scale, void* o_loc,
                                 float* lse_loc, cudaStream_t s);
+cudaError_t local_tc_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                              const void* v, int64_t bh, float scale, void* o_loc,
+                              float* lse_loc, cudaStream_t s);
 cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
                                float scale, int excl, void* o, float* lse_glob, void* o_glob,
@@ -117,7 +120,7 @@ extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q,
     // local branch first (its normalised output goes to o_loc, or to o until it is mixed),
     // then the tensor-core global branch with the mixer in its epilogue
     void* ol = o_loc ? o_loc : o;
-    cudaError_t e = local_simt_dispatch(*idx, q, k, v, dtype, bh, scale, ol, lse_loc, s);
+    cudaError_t e = local_tc_dispatch(*idx, q, k, v, bh, scale, ol, lse_loc, s);
     if (e != cudaSuccess) return PACK3D_ERR_CUDA;
     return cuda_status(global_tc_dispatch(*idx, q, gate, ksum, vsum, ol, bh, scale, excl, o,
                                           lse_glob, o_glob, s));

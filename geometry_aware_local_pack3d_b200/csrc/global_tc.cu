@@ -10,8 +10,8 @@
 // units round-robin. Warp roles (384 threads):
 //   warps 0-3  softmax of tile 0 (thread = row, TMEM lanes 0..127)
 //   warps 4-7  softmax of tile 1
-//   warps 8-9  query producer: coalesced 16-byte loads of q, axial RoPE, bf16 rows into the
-//              K-major shared-memory A operand (double-buffered across units)
+//   warps 8-9  query producer: cp.async of q rows into the K-major shared-memory A operand
+//              (double-buffered across units), then axial RoPE applied in place
 //   warp 10    MMA issuer (one thread) and TMEM owner
 //   warp 11    TMA producer: 128-summary chunks of ksum / vsum into a 2-stage ring
 // Per chunk j and tile t:  S_t = q~_t K_j^T (SS MMA, fp32 in TMEM) -> softmax threads turn S_t
@@ -42,7 +42,8 @@ template <int D> struct Smem {
   static constexpr int kQ = 0;                           // [2 buffers][2 tiles]
   static constexpr int kK = kQ + 2 * kTiles * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kCoord = kV + kStages * kTileBytes;   // 256 packed coordinates
+  static constexpr int kBar = kCoord + kRows * kTiles * 4;
   static constexpr int kBytes = kBar + 256;
 };
 
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < NC; ++j) {
         const uint32_t it = (uint32_t)(pc * NC + j);
-        if (!ab.wait(&bars[B_SFULL + t], it & 1)) break;
+        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + t], it & 1))) break;
         tc::tc_fence_after();
         const int m0 = j * kChunk;
         const int ncol = min(kChunk, M - m0);
@@ -188,40 +189,34 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
               }
             }
         const bool masked = any_x || ncol < kChunk;
-        // pass 1: row max of this chunk (log2 domain)
+        // the whole 128-column chunk in registers: row max (log2 domain) ...
+        uint32_t r[kChunk];
+        tc::tmem_ld64(tl + s_col, *reinterpret_cast<uint32_t(*)[64]>(&r[0]));
+        tc::tmem_ld64(tl + s_col + 64, *reinterpret_cast<uint32_t(*)[64]>(&r[64]));
+        tc::tmem_wait_ld();
         float cmax = -INFINITY;
 #pragma unroll
-        for (int c0 = 0; c0 < kChunk; c0 += 32) {
-          uint32_t r[32];
-          tc::tmem_ld32(tl + s_col + c0, r);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            float s = __uint_as_float(r[k]) * P.scale_log2;
-            if (masked && (((xm[c0 >> 5] >> k) & 1u) || c0 + k >= ncol)) s = -INFINITY;
-            cmax = fmaxf(cmax, s);
-          }
+        for (int k = 0; k < kChunk; ++k) {
+          float s = __uint_as_float(r[k]) * P.scale_log2;
+          if (masked && (((xm[k >> 5] >> (k & 31)) & 1u) || k >= ncol)) s = -INFINITY;
+          r[k] = __float_as_uint(s);
+          cmax = fmaxf(cmax, s);
         }
         const float m_new = fmaxf(m_run, cmax);
         const bool need = m_new > m_run + kRescaleLog2;  // false while everything is masked
         if (__any_sync(0xffffffffu, need) && j > 0) {
           // O_t holds sum_{<j} P V with the old max: wait for the previous PV, then rescale
-          if (!ab.wait(&bars[B_OFULL + t], (it - 1) & 1)) break;
+          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_OFULL + t], (it - 1) & 1))) break;
           tc::tc_fence_after();
           const float f = need ? ex2(m_run - m_new) : 1.f;
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t r[32];
-            tc::tmem_ld32(tl + o_col + c0, r);
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tc::tmem_ld16(tl + o_col + c0, o);
             tc::tmem_wait_ld();
-            uint32_t a[16], b[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              a[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-              b[k] = __float_as_uint(__uint_as_float(r[16 + k]) * f);
-            }
-            tc::tmem_st16(tl + o_col + c0, a);
-            tc::tmem_st16(tl + o_col + c0 + 16, b);
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+            tc::tmem_st16(tl + o_col + c0, o);
           }
           tc::tmem_wait_st();
         }
@@ -230,23 +225,15 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           m_run = m_new;
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        // pass 2: P = exp2(s - m) as bf16, written over the first half of S_t
+        // ... then P = exp2(s - m) as bf16 over the first half of S_t
         float lsum = 0.f;
 #pragma unroll
         for (int c0 = 0; c0 < kChunk; c0 += 32) {
-          uint32_t r[32];
-          tc::tmem_ld32(tl + s_col + c0, r);
-          tc::tmem_wait_ld();
           uint32_t p[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            float s0 = __uint_as_float(r[k]) * P.scale_log2;
-            float s1 = __uint_as_float(r[k + 1]) * P.scale_log2;
-            if (masked) {
-              if (((xm[c0 >> 5] >> k) & 1u) || c0 + k >= ncol) s0 = -INFINITY;
-              if (((xm[c0 >> 5] >> (k + 1)) & 1u) || c0 + k + 1 >= ncol) s1 = -INFINITY;
-            }
-            const float p0 = ex2(s0 - m_use), p1 = ex2(s1 - m_use);
+            const float p0 = ex2(__uint_as_float(r[c0 + k]) - m_use);
+            const float p1 = ex2(__uint_as_float(r[c0 + k + 1]) - m_use);
             lsum += p0 + p1;
             p[k >> 1] = tc::pack_bf16(p0, p1);
           }
@@ -260,7 +247,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       if (*abort_flag) break;
       // epilogue: o_glob = O / l, lse, mixer
       const uint32_t last = (uint32_t)(pc * NC + NC - 1);
-      if (!ab.wait(&bars[B_OFULL + t], last & 1)) break;
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_OFULL + t], last & 1))) break;
       tc::tc_fence_after();
       // O row -> o_glob = O / l, kept packed as bf16 pairs; TMEM is released right after
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -306,40 +293,60 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------------ query producer
+    // cp.async the unit's 256 q rows straight into the operand layout (every copy in flight at
+    // once), then rotate each 16-byte piece in place with the row's coordinate.
     const int ptid = tid - 256;  // 64 producer threads
     constexpr int DA = D / 3;
+    int32_t* coord_s = reinterpret_cast<int32_t*>(smem + S::kCoord);
+    volatile int* prod_ok = abort_flag + 1;
     int pc = 0;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int b = pc & 1;
-      if (pc >= 2 && !ab.wait(&bars[B_QEMPTY + b], ((pc >> 1) - 1) & 1)) break;
+      if (pc >= 2) {
+        // one thread waits; the named barrier hands its verdict to both producer warps
+        if (ptid == 0) *prod_ok = ab.wait(&bars[B_QEMPTY + b], ((pc >> 1) - 1) & 1) ? 1 : 0;
+        asm volatile("bar.sync 1, 64;" ::: "memory");
+        if (!*prod_ok) break;
+      }
       const int64_t bh = u / P.units_per_bh;
       const int64_t row0 = (u % P.units_per_bh) * (kRows * kTiles);
       uint8_t* qb = smem + S::kQ + b * kTiles * S::kTileBytes;
+      const __nv_bfloat16* qsrc = P.q + bh * N * D;
       for (int c = ptid; c < kRows * kTiles * KC; c += 64) {
         const int r = c / KC, kc = c % KC;
         const int64_t row = row0 + r;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (row < N) {
-          const uint4 x = *reinterpret_cast<const uint4*>(P.q + (bh * N + row) * D + kc * 8);
-          const Coord cc = decode(P.ix.coord[row]);
-          const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
-          const int cv = coord_axis(cc, axis);
-          const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
-          uint32_t xo[4];
+        const bool ok = row < N;
+        tc::cp_async16(qb + (r >> 7) * S::kTileBytes + kc * 2048 + ((r & 127) >> 3) * 128 +
+                           (r & 7) * 16,
+                       qsrc + (ok ? row : 0) * D + kc * 8, ok);
+      }
+      tc::cp_async_commit();
+      for (int r = ptid; r < kRows * kTiles; r += 64)
+        coord_s[r] = row0 + r < N ? P.ix.coord[row0 + r] : 0;
+      asm volatile("bar.sync 1, 64;" ::: "memory");
+      tc::cp_async_wait_all();
+#pragma unroll 4
+      for (int c = ptid; c < kRows * kTiles * KC; c += 64) {
+        const int r = c / KC, kc = c % KC;
+        uint4* ptr = reinterpret_cast<uint4*>(qb + (r >> 7) * S::kTileBytes + kc * 2048 +
+                                              ((r & 127) >> 3) * 128 + (r & 7) * 16);
+        const uint4 x = *ptr;
+        const Coord cc = decode(coord_s[r]);
+        const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
+        const int cv = coord_axis(cc, axis);
+        const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
+        uint32_t xo[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 cs = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, p0 + k);
-            const float e0 = __uint_as_float(xin[k] << 16);
-            const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
-            xo[k] = tc::pack_bf16(e0 * cs.x - e1 * cs.y, e0 * cs.y + e1 * cs.x);
-          }
-          w = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+        for (int k = 0; k < 4; ++k) {
+          const float2 cs = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, p0 + k);
+          const float e0 = __uint_as_float(xin[k] << 16);
+          const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+          xo[k] = tc::pack_bf16(e0 * cs.x - e1 * cs.y, e0 * cs.y + e1 * cs.x);
         }
-        const int t = r / kRows, rr = r % kRows;
-        *reinterpret_cast<uint4*>(qb + t * S::kTileBytes + kc * 2048 + (rr >> 3) * 128 +
-                                  (rr & 7) * 16) = w;
+        *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
       }
       tc::fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 64;" ::: "memory");  // coord_s is rewritten next unit
       tc::mbar_arrive(&bars[B_QFULL + b]);
     }
   } else if (warp == 10) {
