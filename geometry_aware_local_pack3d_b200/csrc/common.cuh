@@ -55,4 +55,22 @@ __device__ __forceinline__ bool block_is_near(const pack3d_index& ix, int m, con
 
 __device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + __expf(-a)); }
 
+// Phase timestamps for one CTA, compiled in only by a tracing build (P3D_TRACE_ENABLED):
+// the kernels mark their handoffs with P3D_TRACE(slot); normal builds emit nothing.
+#ifdef P3D_TRACE_ENABLED
+static __device__ unsigned long long g_trace[4096];
+#define P3D_TRACE(slot)                                                            \
+  do {                                                                             \
+    if (blockIdx.x == 0) {                                                         \
+      unsigned long long t_;                                                       \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
+      g_trace[(slot) & 4095] = t_;                                                 \
+    }                                                                              \
+  } while (0)
+#else
+#define P3D_TRACE(slot) \
+  do {                  \
+  } while (0)
+#endif
+
 }  // namespace p3d

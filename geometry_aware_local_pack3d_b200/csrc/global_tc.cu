@@ -7,17 +7,19 @@
 //
 // Work unit: 256 consecutive memory rows of one (batch, head) = two 128-row query tiles that
 // share every summary chunk (halves the L2 reads of the summaries). Persistent CTAs walk the
-// units round-robin. Warp roles (384 threads):
-//   warps 0-3  softmax of tile 0 (thread = row, TMEM lanes 0..127)
-//   warps 4-7  softmax of tile 1
-//   warps 8-9  query producer: cp.async of q rows into the K-major shared-memory A operand
-//              (double-buffered across units), then axial RoPE applied in place
-//   warp 10    MMA issuer (one thread) and TMEM owner
-//   warp 11    TMA producer: 128-summary chunks of ksum / vsum into a 2-stage ring
-// Per chunk j and tile t:  S_t = q~_t K_j^T (SS MMA, fp32 in TMEM) -> softmax threads turn S_t
-// into P_t = exp2(s - m) in bf16, written over S_t in TMEM -> O_t += P_t V_j (TS MMA).
-// The running max uses a lazy rescale: O_t is corrected in TMEM only when a row's max grows by
-// more than 2^8, so the common case touches O once at the end.
+// units round-robin. Warp roles (448 threads):
+//   warps 0-3   softmax + epilogue of tile 0 (thread = row, TMEM lanes 0..127)
+//   warps 4-7   softmax + epilogue of tile 1
+//   warps 8-11  query producer: cp.async of q rows into the K-major shared-memory A operand
+//               (double-buffered across units), then axial RoPE applied in place
+//   warp 12     MMA issuer (one thread) and TMEM owner
+//   warp 13     TMA producer: 64-summary chunks of ksum / vsum into a 4-stage ring
+// Per 64-summary chunk j and tile t:  S_t[j%2] = q~_t K_j^T (SS MMA, fp32 in TMEM) -> the
+// softmax threads turn it into P = exp2(s - m) in bf16, written over S in TMEM ->
+// O_t += P V_j (TS MMA). S is double-buffered, and the issuer runs one chunk ahead (QK of
+// chunk j+1 is issued before the PV of chunk j), so the softmax of consecutive chunks runs
+// back to back while the tensor core works in its shadow. The running max uses a lazy
+// rescale: O_t is corrected in TMEM only when a row's max grows by more than 2^8.
 // The summary order is the same for every query (block ids ascending) and rows never interact,
 // so a coordinate-carrying repack permutes the output bit for bit.
 #include <math.h>
@@ -31,34 +33,42 @@ namespace p3d {
 namespace gtc {
 constexpr int kRows = 128;        // rows per tile
 constexpr int kTiles = 2;         // tiles per unit
-constexpr int kChunk = 128;       // summaries per chunk
-constexpr int kStages = 2;        // summary ring depth
-constexpr int kThreads = 384;
+constexpr int kChunk = 64;        // summaries per chunk
+constexpr int kStages = 4;        // summary ring depth
+constexpr int kThreads = 448;
+constexpr int kProd = 128;        // query producer threads
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kRopeSmemBytes = 16384;
+
+// TMEM columns: tile t uses [256 t, 256 t + 256): S buffers at +0 and +64, O at +128.
+__host__ __device__ constexpr uint32_t s_col(int t, int b) { return 256u * t + 64u * b; }
+__host__ __device__ constexpr uint32_t o_col(int t) { return 256u * t + 128u; }
 
 template <int D> struct Smem {
-  static constexpr int kTileBytes = kRows * D * 2;       // one q tile / one summary chunk
-  static constexpr int kQ = 0;                           // [2 buffers][2 tiles]
-  static constexpr int kK = kQ + 2 * kTiles * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kCoord = kV + kStages * kTileBytes;   // 256 packed coordinates
-  static constexpr int kBar = kCoord + kRows * kTiles * 4;
+  static constexpr int kQTile = kRows * D * 2;       // one q tile
+  static constexpr int kCTile = kChunk * D * 2;      // one summary chunk (ksum or vsum)
+  static constexpr int kQ = 0;                       // [2 buffers][2 tiles]
+  static constexpr int kK = kQ + 2 * kTiles * kQTile;
+  static constexpr int kV = kK + kStages * kCTile;
+  static constexpr int kCoord = kV + kStages * kCTile;  // 256 packed coordinates
+  static constexpr int kRope = kCoord + kRows * kTiles * 4;
+  static constexpr int kBar = kRope + kRopeSmemBytes;
   static constexpr int kBytes = kBar + 256;
 };
 
 // barrier slots
 enum {
-  B_QFULL = 0,   // [2]
-  B_QEMPTY = 2,  // [2]
-  B_KVFULL = 4,  // [kStages]
-  B_KVEMPTY = 6, // [kStages]
-  B_SFULL = 8,   // [2] per tile
-  B_PFULL = 10,  // [2]
-  B_OFULL = 12,  // [2]
-  B_OFREE = 14,  // [2]
-  B_DONE = 16,
-  B_COUNT = 17
+  B_QFULL = 0,    // [2] q buffer filled
+  B_QEMPTY = 2,   // [2] q buffer consumed
+  B_KVFULL = 4,   // [kStages]
+  B_KVEMPTY = 8,  // [kStages]
+  B_SFULL = 12,   // [tile][buf] = 12 + 2 t + b
+  B_PFULL = 16,   // [tile][buf]
+  B_PVDONE = 20,  // [tile][buf]
+  B_OFREE = 24,   // [tile]
+  B_DONE = 26,
+  B_COUNT = 27
 };
 
 struct Params {
@@ -74,6 +84,7 @@ struct Params {
   int64_t units;               // (batch*heads) * units_per_bh
   int units_per_bh;
   int n_chunks;
+  int rope_in_smem;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -86,9 +97,9 @@ struct Abort {
   volatile int* flag;
   int32_t* status;
   __device__ bool wait(uint64_t* bar, uint32_t parity) {
-    if (tc::mbar_try_wait(bar, parity)) return true;
+    if (tc::mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!tc::mbar_try_wait(bar, parity)) {
+    while (!tc::mbar_test_wait(bar, parity)) {
       if (*flag) return false;
       if (clock64() - t0 > 4000000000LL) {
         *flag = 1;
@@ -109,21 +120,26 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
   using namespace gtc;
   using S = Smem<D>;
   constexpr int KC = D / 8;  // 16-byte chunks per row
+  constexpr int CB = kChunk * 16;  // byte stride between 16-byte columns of a summary chunk
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
+  volatile int* prod_ok = abort_flag + 1;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) P3D_TRACE(999);
   Abort ab{abort_flag, P.ix.status};
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bars[B_QFULL + i], 64);
+      tc::mbar_init(&bars[B_QFULL + i], kProd);
       tc::mbar_init(&bars[B_QEMPTY + i], 1);
+      tc::mbar_init(&bars[B_OFREE + i], 128);
+    }
+    for (int i = 0; i < 4; ++i) {
       tc::mbar_init(&bars[B_SFULL + i], 1);
       tc::mbar_init(&bars[B_PFULL + i], 128);
-      tc::mbar_init(&bars[B_OFULL + i], 1);
-      tc::mbar_init(&bars[B_OFREE + i], 128);
+      tc::mbar_init(&bars[B_PVDONE + i], 1);
     }
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bars[B_KVFULL + i], 1);
@@ -133,7 +149,13 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 10) tc::tmem_alloc(tmem_slot, kTmemCols);
+  // the rotation table in shared memory when it fits (read by the query producer)
+  if (P.rope_in_smem) {
+    const int n = P.ix.rope_rows * P.ix.rope_pairs * 2;
+    float* dst = reinterpret_cast<float*>(smem + S::kRope);
+    for (int i = tid; i < n; i += blockDim.x) dst[i] = P.ix.rope[i];
+  }
+  if (warp == 12) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -147,7 +169,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     const int t = warp >> 2;
     const int rin = (warp & 3) * 32 + lane;
     const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t s_col = t * 128, o_col = 256 + t * 128;
+    const int nby = P.ix.geom.gy / P.ix.geom.by, nbx = P.ix.geom.gx / P.ix.geom.bx;
     int pc = 0;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int64_t bh = u / P.units_per_bh;
@@ -156,7 +178,6 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       // summaries excluded for this row: blocks meeting the cube [c-1, c+1]^3, kept as block
       // coordinate ranges [z0,z1] x [y0,y1] x [x0,x1] (empty when exclusion is off)
       int z0 = 0, z1 = -1, y0 = 0, y1 = -1, x0 = 0, x1 = -1;
-      const int nby = P.ix.geom.gy / P.ix.geom.by, nbx = P.ix.geom.gx / P.ix.geom.bx;
       if (P.exclude_near && valid) {
         const Coord c = decode(P.ix.coord[row]);
         const pack3d_geom& g = P.ix.geom;
@@ -165,14 +186,19 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         x0 = max(c.x - 1, 0) / g.bx; x1 = min(c.x + 1, g.gx - 1) / g.bx;
       }
       float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
       for (int j = 0; j < NC; ++j) {
-        const uint32_t it = (uint32_t)(pc * NC + j);
-        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + t], it & 1))) break;
+        const uint32_t gi = (uint32_t)(pc * NC + j);  // chunk counter of this tile
+        const int b = gi & 1;
+        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + 2 * t + b], (gi >> 1) & 1))) {
+          ok = false;
+          break;
+        }
+        if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2);
         tc::tc_fence_after();
         const int m0 = j * kChunk;
         const int ncol = min(kChunk, M - m0);
-        // exclusion bitmask of this chunk
-        uint32_t xm[4] = {0u, 0u, 0u, 0u};
+        uint32_t xm[2] = {0u, 0u};
         bool any_x = false;
         for (int mz = z0; mz <= z1; ++mz)
           for (int my = y0; my <= y1; ++my)
@@ -180,43 +206,49 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
               const int cidx = (mz * nby + my) * nbx + mx - m0;
               if (cidx >= 0 && cidx < kChunk) {
                 const uint32_t bit = 1u << (cidx & 31);
-                const int w = cidx >> 5;
-                xm[0] |= w == 0 ? bit : 0u;
-                xm[1] |= w == 1 ? bit : 0u;
-                xm[2] |= w == 2 ? bit : 0u;
-                xm[3] |= w == 3 ? bit : 0u;
+                xm[0] |= (cidx >> 5) == 0 ? bit : 0u;
+                xm[1] |= (cidx >> 5) == 1 ? bit : 0u;
                 any_x = true;
               }
             }
         const bool masked = any_x || ncol < kChunk;
-        // the whole 128-column chunk in registers: row max (log2 domain) ...
+        // the 64-column chunk in registers; masked entries become -inf in place
         uint32_t r[kChunk];
-        tc::tmem_ld64(tl + s_col, *reinterpret_cast<uint32_t(*)[64]>(&r[0]));
-        tc::tmem_ld64(tl + s_col + 64, *reinterpret_cast<uint32_t(*)[64]>(&r[64]));
+        tc::tmem_ld64(tl + s_col(t, b), r);
         tc::tmem_wait_ld();
-        float cmax = -INFINITY;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (!masked) {
 #pragma unroll
-        for (int k = 0; k < kChunk; ++k) {
-          float s = __uint_as_float(r[k]) * P.scale_log2;
-          if (masked && (((xm[k >> 5] >> (k & 31)) & 1u) || k >= ncol)) s = -INFINITY;
-          r[k] = __float_as_uint(s);
-          cmax = fmaxf(cmax, s);
+          for (int k = 0; k < kChunk; ++k) mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
+        } else {
+#pragma unroll
+          for (int k = 0; k < kChunk; ++k) {
+            if (((xm[k >> 5] >> (k & 31)) & 1u) || k >= ncol) r[k] = 0xff800000u;  // -inf
+            mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
+          }
         }
+        // row max in the log2 domain (the scale is positive)
+        const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
         const float m_new = fmaxf(m_run, cmax);
         const bool need = m_new > m_run + kRescaleLog2;  // false while everything is masked
         if (__any_sync(0xffffffffu, need) && j > 0) {
           // O_t holds sum_{<j} P V with the old max: wait for the previous PV, then rescale
-          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_OFULL + t], (it - 1) & 1))) break;
+          const uint32_t gp = gi - 1;
+          if (!__all_sync(0xffffffffu,
+                          ab.wait(&bars[B_PVDONE + 2 * t + (gp & 1)], (gp >> 1) & 1))) {
+            ok = false;
+            break;
+          }
           tc::tc_fence_after();
           const float f = need ? ex2(m_run - m_new) : 1.f;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t o[16];
-            tc::tmem_ld16(tl + o_col + c0, o);
+            tc::tmem_ld16(tl + o_col(t) + c0, o);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-            tc::tmem_st16(tl + o_col + c0, o);
+            tc::tmem_st16(tl + o_col(t) + c0, o);
           }
           tc::tmem_wait_st();
         }
@@ -224,46 +256,49 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           l_run *= ex2(m_run - m_new);
           m_run = m_new;
         }
-        const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        // ... then P = exp2(s - m) as bf16 over the first half of S_t
-        float lsum = 0.f;
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        // P = exp2(s * scale - m) as bf16 over the first half of this S buffer
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c0 = 0; c0 < kChunk; c0 += 32) {
           uint32_t p[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2(__uint_as_float(r[c0 + k]) - m_use);
-            const float p1 = ex2(__uint_as_float(r[c0 + k + 1]) - m_use);
-            lsum += p0 + p1;
+            const float p0 = ex2(fmaf(__uint_as_float(r[c0 + k]), P.scale_log2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(r[c0 + k + 1]), P.scale_log2, neg_m));
+            ls[(k >> 1) & 3] += p0 + p1;
             p[k >> 1] = tc::pack_bf16(p0, p1);
           }
-          tc::tmem_st16(tl + s_col + (c0 >> 1), p);
+          tc::tmem_st16(tl + s_col(t, b) + (c0 >> 1), p);
         }
-        l_run += lsum;
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tc::tmem_wait_st();
         tc::tc_fence_before();
-        tc::mbar_arrive(&bars[B_PFULL + t]);
+        tc::mbar_arrive(&bars[B_PFULL + 2 * t + b]);
+        if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2 + 1);
       }
-      if (*abort_flag) break;
+      if (!ok) break;
       // epilogue: o_glob = O / l, lse, mixer
-      const uint32_t last = (uint32_t)(pc * NC + NC - 1);
-      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_OFULL + t], last & 1))) break;
+      const uint32_t gl = (uint32_t)(pc * NC + NC - 1);
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVDONE + 2 * t + (gl & 1)], (gl >> 1) & 1)))
+        break;
       tc::tc_fence_after();
       // O row -> o_glob = O / l, kept packed as bf16 pairs; TMEM is released right after
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       uint32_t gp[(D + 31) / 32 * 16];
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tc::tmem_ld32(tl + o_col + c0, r);
+        uint32_t o[32];
+        tc::tmem_ld32(tl + o_col(t) + c0, o);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          gp[c0 / 2 + k] = tc::pack_bf16(__uint_as_float(r[2 * k]) * inv_l,
-                                         __uint_as_float(r[2 * k + 1]) * inv_l);
+          gp[c0 / 2 + k] = tc::pack_bf16(__uint_as_float(o[2 * k]) * inv_l,
+                                         __uint_as_float(o[2 * k + 1]) * inv_l);
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&bars[B_OFREE + t]);
+      if (rin == 0 && pc < 3) P3D_TRACE(1500 + pc * 4 + t * 2);
       if (valid) {
         const int64_t grow = bh * N + row;
         if (P.lse_glob)
@@ -291,116 +326,148 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         }
       }
     }
-  } else if (warp < 10) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------------ query producer
     // cp.async the unit's 256 q rows straight into the operand layout (every copy in flight at
     // once), then rotate each 16-byte piece in place with the row's coordinate.
-    const int ptid = tid - 256;  // 64 producer threads
+    const int ptid = tid - 256;
     constexpr int DA = D / 3;
     int32_t* coord_s = reinterpret_cast<int32_t*>(smem + S::kCoord);
-    volatile int* prod_ok = abort_flag + 1;
+    const float* rope = P.rope_in_smem ? reinterpret_cast<const float*>(smem + S::kRope) : P.ix.rope;
     int pc = 0;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int b = pc & 1;
       if (pc >= 2) {
-        // one thread waits; the named barrier hands its verdict to both producer warps
+        // one thread waits; the named barrier hands its verdict to all producer warps
         if (ptid == 0) *prod_ok = ab.wait(&bars[B_QEMPTY + b], ((pc >> 1) - 1) & 1) ? 1 : 0;
-        asm volatile("bar.sync 1, 64;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         if (!*prod_ok) break;
       }
+      if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4);
       const int64_t bh = u / P.units_per_bh;
       const int64_t row0 = (u % P.units_per_bh) * (kRows * kTiles);
-      uint8_t* qb = smem + S::kQ + b * kTiles * S::kTileBytes;
+      uint8_t* qb = smem + S::kQ + b * kTiles * S::kQTile;
       const __nv_bfloat16* qsrc = P.q + bh * N * D;
-      for (int c = ptid; c < kRows * kTiles * KC; c += 64) {
-        const int r = c / KC, kc = c % KC;
+      for (int c = ptid; c < kRows * kTiles * KC; c += kProd) {
+        int r, kc;
+        tc::PieceOrder<KC>::at(c, r, kc);
         const int64_t row = row0 + r;
         const bool ok = row < N;
-        tc::cp_async16(qb + (r >> 7) * S::kTileBytes + kc * 2048 + ((r & 127) >> 3) * 128 +
+        tc::cp_async16(qb + (r >> 7) * S::kQTile + kc * 2048 + ((r & 127) >> 3) * 128 +
                            (r & 7) * 16,
                        qsrc + (ok ? row : 0) * D + kc * 8, ok);
       }
       tc::cp_async_commit();
-      for (int r = ptid; r < kRows * kTiles; r += 64)
+      for (int r = ptid; r < kRows * kTiles; r += kProd)
         coord_s[r] = row0 + r < N ? P.ix.coord[row0 + r] : 0;
-      asm volatile("bar.sync 1, 64;" ::: "memory");
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       tc::cp_async_wait_all();
+      if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4 + 1);
 #pragma unroll 4
-      for (int c = ptid; c < kRows * kTiles * KC; c += 64) {
-        const int r = c / KC, kc = c % KC;
-        uint4* ptr = reinterpret_cast<uint4*>(qb + (r >> 7) * S::kTileBytes + kc * 2048 +
+      for (int c = ptid; c < kRows * kTiles * KC; c += kProd) {
+        int r, kc;
+        tc::PieceOrder<KC>::at(c, r, kc);
+        uint4* ptr = reinterpret_cast<uint4*>(qb + (r >> 7) * S::kQTile + kc * 2048 +
                                               ((r & 127) >> 3) * 128 + (r & 7) * 16);
         const uint4 x = *ptr;
         const Coord cc = decode(coord_s[r]);
         const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
         const int cv = coord_axis(cc, axis);
+        // (cos, sin) of the 4 pairs of this piece: 32 contiguous bytes of the table
+        const float4* cs4 = reinterpret_cast<const float4*>(rope + 2 * (cv * P.ix.rope_pairs + p0));
+        const float4 ca = cs4[0], cb = cs4[1];
+        const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
         const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
         uint32_t xo[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float2 cs = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, p0 + k);
           const float e0 = __uint_as_float(xin[k] << 16);
           const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
-          xo[k] = tc::pack_bf16(e0 * cs.x - e1 * cs.y, e0 * cs.y + e1 * cs.x);
+          xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
+                                e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
         }
         *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
       }
       tc::fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 64;" ::: "memory");  // coord_s is rewritten next unit
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // coord_s is rewritten next unit
       tc::mbar_arrive(&bars[B_QFULL + b]);
+      if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4 + 2);
     }
-  } else if (warp == 10) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
       int pc = 0;
       uint32_t kv_it = 0;
-      bool issued = false;
-      for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x, ++pc) {
-        const int b = pc & 1;
-        if (!ab.wait(&bars[B_QFULL + b], (pc >> 1) & 1)) break;
+      bool issued = false, ok = true;
+      for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++pc) {
+        const int qb = pc & 1;
+        if (!ab.wait(&bars[B_QFULL + qb], (pc >> 1) & 1)) break;
+        if (pc < 3) P3D_TRACE(2600 + pc);
         tc::tc_fence_after();
-        const uint32_t qaddr = tc::smem_u32(smem + S::kQ + b * kTiles * S::kTileBytes);
-        bool ok = true;
-        for (int j = 0; j < P.n_chunks && ok; ++j, ++kv_it) {
-          const int st = kv_it % kStages;
-          if (!ab.wait(&bars[B_KVFULL + st], (kv_it / kStages) & 1)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint32_t kaddr = tc::smem_u32(smem + S::kK + st * S::kTileBytes);
-          const uint32_t vaddr = tc::smem_u32(smem + S::kV + st * S::kTileBytes);
-          const uint32_t it = (uint32_t)(pc * P.n_chunks + j);
-          for (int t = 0; t < kTiles; ++t) {
-            // S_t / P_t is free once the previous PV on this tile has completed
-            if (it > 0 && !ab.wait(&bars[B_OFULL + t], (it - 1) & 1)) { ok = false; break; }
+        const uint32_t qaddr = tc::smem_u32(smem + S::kQ + qb * kTiles * S::kQTile);
+        // QK of chunk j is issued one step ahead of the PV of chunk j - 1
+        for (int j = 0; j <= NC && ok; ++j) {
+          if (j < NC) {
+            const uint32_t kv = kv_it + j;
+            const int st = kv % kStages;
+            if (!ab.wait(&bars[B_KVFULL + st], (kv / kStages) & 1)) { ok = false; break; }
+            if (pc < 3) P3D_TRACE(2500 + pc * 32 + j);
             tc::tc_fence_after();
+            const uint32_t kaddr = tc::smem_u32(smem + S::kK + st * S::kCTile);
+            const uint32_t gi = (uint32_t)(pc * NC + j);
+            const int b = gi & 1;
+            for (int t = 0; t < kTiles; ++t) {
+              // this S buffer held P of chunk gi - 2: free once that PV has completed
+              if (gi >= 2 && !ab.wait(&bars[B_PVDONE + 2 * t + b], ((gi >> 1) - 1) & 1)) {
+                ok = false;
+                break;
+              }
+              tc::tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint64_t a = tc::smem_desc(qaddr + t * S::kTileBytes + ks * 4096, 2048, 128);
-              const uint64_t bd = tc::smem_desc(kaddr + ks * 4096, 2048, 128);
-              tc::mma_ss(tbase + t * 128, a, bd, id_qk, ks > 0);
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint64_t a =
+                    tc::smem_desc(qaddr + t * S::kQTile + ks * 4096, 2048, 128);
+                const uint64_t bd = tc::smem_desc(kaddr + ks * 2 * CB, CB, 128);
+                tc::mma_ss(tbase + s_col(t, b), a, bd, id_qk, ks > 0);
+              }
+              tc::tc_commit(&bars[B_SFULL + 2 * t + b]);
+              if (pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2);
+              issued = true;
             }
-            tc::tc_commit(&bars[B_SFULL + t]);
-            issued = true;
+            if (!ok) break;
           }
-          if (!ok) break;
-          for (int t = 0; t < kTiles; ++t) {
-            if (!ab.wait(&bars[B_PFULL + t], it & 1)) { ok = false; break; }
-            if (j == 0 && pc > 0 && !ab.wait(&bars[B_OFREE + t], (pc - 1) & 1)) { ok = false; break; }
-            tc::tc_fence_after();
+          if (j >= 1) {
+            const int jj = j - 1;
+            const uint32_t kv = kv_it + jj;
+            const int st = kv % kStages;
+            const uint32_t vaddr = tc::smem_u32(smem + S::kV + st * S::kCTile);
+            const uint32_t gi = (uint32_t)(pc * NC + jj);
+            const int b = gi & 1;
+            for (int t = 0; t < kTiles; ++t) {
+              if (!ab.wait(&bars[B_PFULL + 2 * t + b], (gi >> 1) & 1)) { ok = false; break; }
+              if (jj == 0 && pc > 0 && !ab.wait(&bars[B_OFREE + t], (pc - 1) & 1)) {
+                ok = false;
+                break;
+              }
+              tc::tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < kChunk / 16; ++ks) {
-              const uint64_t bd = tc::smem_desc(vaddr + ks * 256, 128, 2048);
-              tc::mma_ts(tbase + 256 + t * 128, tbase + t * 128 + ks * 8, bd, id_pv,
-                         (j > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < kChunk / 16; ++ks) {
+                const uint64_t bd = tc::smem_desc(vaddr + ks * 256, 128, CB);
+                tc::mma_ts(tbase + o_col(t), tbase + s_col(t, b) + ks * 8, bd, id_pv,
+                           (jj > 0 || ks > 0) ? 1u : 0u);
+              }
+              tc::tc_commit(&bars[B_PVDONE + 2 * t + b]);
+              if (pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + jj * 2 + 1);
             }
-            tc::tc_commit(&bars[B_OFULL + t]);
+            if (!ok) break;
+            tc::tc_commit(&bars[B_KVEMPTY + st]);
           }
-          if (!ok) break;
-          tc::tc_commit(&bars[B_KVEMPTY + st]);
         }
+        kv_it += NC;
         if (!ok) break;
-        tc::tc_commit(&bars[B_QEMPTY + b]);
+        tc::tc_commit(&bars[B_QEMPTY + qb]);
       }
       // every MMA issued by this thread has completed before TMEM is released
       if (issued) {
@@ -417,18 +484,18 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x) {
         const int64_t bh = u / P.units_per_bh;
         bool ok = true;
-        for (int j = 0; j < P.n_chunks; ++j, ++kv_it) {
+        for (int j = 0; j < NC; ++j, ++kv_it) {
           const int st = kv_it % kStages;
           if (kv_it >= (uint32_t)kStages &&
               !ab.wait(&bars[B_KVEMPTY + st], ((kv_it / kStages) - 1) & 1)) { ok = false; break; }
-          tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kTileBytes);
+          tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kCTile);
           const int y = (int)(bh * M + j * kChunk);
-          uint8_t* kd = smem + S::kK + st * S::kTileBytes;
-          uint8_t* vd = smem + S::kV + st * S::kTileBytes;
+          uint8_t* kd = smem + S::kK + st * S::kCTile;
+          uint8_t* vd = smem + S::kV + st * S::kCTile;
 #pragma unroll
           for (int kc = 0; kc < KC; ++kc) {
-            tc::tma_load_2d(kd + kc * 2048, &map_k, 8 * kc, y, &bars[B_KVFULL + st]);
-            tc::tma_load_2d(vd + kc * 2048, &map_v, 8 * kc, y, &bars[B_KVFULL + st]);
+            tc::tma_load_2d(kd + kc * CB, &map_k, 8 * kc, y, &bars[B_KVFULL + st]);
+            tc::tma_load_2d(vd + kc * CB, &map_v, 8 * kc, y, &bars[B_KVFULL + st]);
           }
         }
         if (!ok) break;
@@ -441,7 +508,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 10) {
+  if (warp == 12) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, kTmemCols);
   }
@@ -469,14 +536,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, D] bf16 row-major viewed as 2D; box = 8 columns x 128 rows (one 16-byte column of
-// core matrices), no swizzle.
+// [rows, D] bf16 row-major viewed as 2D; box = 8 columns x 64 rows (one 16-byte column of
+// core matrices of a summary chunk), no swizzle.
 bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int D) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {8, 128};
+  cuuint32_t box[2] = {8, (cuuint32_t)gtc::kChunk};
   cuuint32_t es[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -525,6 +592,7 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   p.units_per_bh = (int)((ix.n + kRows * kTiles - 1) / (kRows * kTiles));
   p.units = bh * p.units_per_bh;
   p.n_chunks = (int)((ix.m + kChunk - 1) / kChunk);
+  p.rope_in_smem = (int64_t)ix.rope_rows * ix.rope_pairs * 8 <= kRopeSmemBytes ? 1 : 0;
   const int grid = (int)(p.units < sm_count() ? p.units : sm_count());
   k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mk, mv, p);
   count_launch();
@@ -543,3 +611,14 @@ cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void
 }
 
 }  // namespace p3d
+
+#ifdef P3D_TRACE_ENABLED
+extern "C" int p3d_trace_read_g(unsigned long long* host) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(host, p3d::g_trace, sizeof(unsigned long long) * 4096);
+}
+extern "C" int p3d_trace_clear_g() {
+  static unsigned long long z[4096];
+  return (int)cudaMemcpyToSymbol(p3d::g_trace, z, sizeof(z));
+}
+#endif

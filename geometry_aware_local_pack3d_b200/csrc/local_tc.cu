@@ -5,7 +5,7 @@
 // the border), found by coordinate, never by adjacency in memory; paper summary §3.5: streamed
 // online softmax, no gathered neighbour tensor in memory.
 //
-// A CTA owns one 8x4x4 (z, y, x) coordinate brick of 128 queries of one (batch, head). Its
+// A CTA (4 softmax warps, 3 gather warps, 1 MMA warp) owns one 8x4x4 (z, y, x) coordinate brick of 128 queries of one (batch, head). Its
 // 10x6x6 halo of keys is streamed through shared memory in 5 chunks of two halo z-slices
 // (72 keys, padded to 80). Rows are brick positions: row = 32 w + 16 dz + 4 y + x, so warp w
 // holds brick z-slices 2w, 2w+1 and needs exactly halo chunks w and w + 1. Per chunk c:
@@ -33,7 +33,8 @@ constexpr int kSliceKeys = HY * HX;     // 36
 constexpr int kChunkKeys = 2 * kSliceKeys;  // 72
 constexpr int kChunkPad = 80;           // MMA N (multiple of 16)
 constexpr int kChunks = HZ / 2;         // 5
-constexpr int kThreads = 288;           // 4 softmax + 4 producer + 1 MMA warps
+constexpr int kThreads = 256;           // 4 softmax + 3 producer + 1 MMA warps
+constexpr int kProd = 96;               // producer threads
 constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -80,9 +81,9 @@ struct Abort {
   volatile int* flag;
   int32_t* status;
   __device__ bool wait(uint64_t* bar, uint32_t parity) {
-    if (tc::mbar_try_wait(bar, parity)) return true;
+    if (tc::mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!tc::mbar_try_wait(bar, parity)) {
+    while (!tc::mbar_test_wait(bar, parity)) {
       if (*flag) return false;
       if (clock64() - t0 > 4000000000LL) {
         *flag = 1;
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) P3D_TRACE(3000);
   Abort ab{abort_flag, P.ix.status};
   const pack3d_geom& g = P.ix.geom;
   const int64_t N = P.ix.n;
@@ -137,9 +139,9 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
   const __nv_bfloat16* vb = P.v + bh * N * D;
 
   if (tid == 0) {
-    tc::mbar_init(&bars[B_QFULL], 128);
+    tc::mbar_init(&bars[B_QFULL], kProd);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bars[B_KVFULL + i], 128);
+      tc::mbar_init(&bars[B_KVFULL + i], kProd);
       tc::mbar_init(&bars[B_KVEMPTY + i], 1);
     }
     tc::mbar_init(&bars[B_SFULL], 1);
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 8) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 7) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -180,6 +182,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     bool ok = true;
     for (int c = 0; c < kChunks && ok; ++c) {
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL], c & 1))) { ok = false; break; }
+      if (lane == 0) P3D_TRACE(3100 + warp * 16 + c * 2);
       tc::tc_fence_after();
       const int part = c - warp;  // 0 or 1 when this warp owns chunk c
       if (part == 0 || part == 1) {
@@ -192,21 +195,20 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
           win[1] = (nb[3] >> 16) | (nb[4] << 16);
           win[2] = nb[4] >> 16;
         }
-        // pass 1: masked row max (log2 domain)
-        float cmax = -INFINITY;
+        // the chunk's 80 columns in registers; entries off the 3x3x3 cube become -inf, so the
+        // row max and P = exp2(s * scale - m) need no further masking (raw scores; scale > 0)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t r[kChunkPad];
 #pragma unroll
-        for (int c0 = 0; c0 < kChunkPad; c0 += 16) {
-          uint32_t r[16];
-          tc::tmem_ld16(tl + s_col + c0, r);
-          tc::tmem_wait_ld();
+        for (int c0 = 0; c0 < kChunkPad; c0 += 16)
+          tc::tmem_ld16(tl + s_col + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[c0]));
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int bit = c0 + k;
-            const bool on = (win[bit >> 5] >> (bit & 31)) & 1u;
-            const float s = __uint_as_float(r[k]) * P.scale_log2;
-            cmax = on ? fmaxf(cmax, s) : cmax;
-          }
+        for (int k = 0; k < kChunkPad; ++k) {
+          if (!((win[k >> 5] >> (k & 31)) & 1u)) r[k] = 0xff800000u;  // -inf off the cube
+          mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
         }
+        const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
         const float m_new = fmaxf(m_run, cmax);
         const bool need = m_new > m_run + kRescaleLog2;
         if (part == 1 && __any_sync(0xffffffffu, need)) {
@@ -230,26 +232,22 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
           m_run = m_new;
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        // pass 2: P over the first 40 columns of S
-        float lsum = 0.f;
+        // P over the first 40 columns of S
+        const float neg_m = -m_use;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c0 = 0; c0 < kChunkPad; c0 += 16) {
-          uint32_t r[16];
-          tc::tmem_ld16(tl + s_col + c0, r);
-          tc::tmem_wait_ld();
           uint32_t p[8];
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
-            const int bit = c0 + k;
-            const bool on0 = (win[bit >> 5] >> (bit & 31)) & 1u;
-            const bool on1 = (win[(bit + 1) >> 5] >> ((bit + 1) & 31)) & 1u;
-            const float p0 = on0 ? ex2(__uint_as_float(r[k]) * P.scale_log2 - m_use) : 0.f;
-            const float p1 = on1 ? ex2(__uint_as_float(r[k + 1]) * P.scale_log2 - m_use) : 0.f;
-            lsum += p0 + p1;
+            const float p0 = ex2(fmaf(__uint_as_float(r[c0 + k]), P.scale_log2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(r[c0 + k + 1]), P.scale_log2, neg_m));
+            ls[(k >> 1) & 3] += p0 + p1;
             p[k >> 1] = tc::pack_bf16(p0, p1);
           }
           ltc::tmem_st8(tl + s_col + (c0 >> 1), p);
         }
+        const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
         l_run += lsum;
       } else {
         const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -259,6 +257,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
       tc::tmem_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars[B_PFULL]);
+      if (lane == 0) P3D_TRACE(3100 + warp * 16 + c * 2 + 1);
     }
     if (ok) {
       // epilogue after the last PV: o_loc = O / l, lse_loc
@@ -284,11 +283,12 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
             dst[c0 / 8 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
           }
         }
+        if (lane == 0) P3D_TRACE(3400 + warp);
         if (slot >= 0 && P.lse_loc)
           P.lse_loc[bh * N + slot] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 7) {
     // --------------------------------------------------------- producer: q tile, then k/v chunks
     // Slots of the 128 queries and 360 halo keys and the rotation rows of the 22 coordinate
     // values the brick touches are staged in shared memory first; every row piece is then a
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     int32_t* slot_h = slot_q + 128;
     float2* rope_s = reinterpret_cast<float2*>(smem + S::kRope);  // [22][PR]
     volatile int* prod_ok = abort_flag + 1;
-    for (int i = ptid; i < 128 + HZ * kSliceKeys; i += 128) {
+    for (int i = ptid; i < 128 + HZ * kSliceKeys; i += kProd) {
       int z, y, x;
       if (i < 128) {
         const int w = i >> 5, l = i & 31;
@@ -311,32 +311,36 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
       const bool in = z >= 0 && z < g.gz && y >= 0 && y < g.gy && x >= 0 && x < g.gx;
       slot_q[i] = in ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : -1;
     }
-    for (int i = ptid; i < (HZ + HY + HX) * PR; i += 128) {
+    for (int i = ptid; i < (HZ + HY + HX) * PR; i += kProd) {
       const int idx = i / PR, pp = i % PR;
       const int cv = idx < HZ ? z0 - 1 + idx : (idx < HZ + HY ? y0 - 1 + idx - HZ : x0 - 1 + idx - HZ - HY);
       rope_s[i] = (cv >= 0 && cv < P.ix.rope_rows) ? rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp)
                                                    : make_float2(0.f, 0.f);
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 96;" ::: "memory");
+    if (ptid == 0) P3D_TRACE(3001);
     // rotation of one 16-byte piece (8 dims, 4 pairs) in place, for halo position (hz, hy, hx)
     auto rotate_at = [&](uint8_t* ptr, int hz, int hy, int hx, int kc) {
       const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
       const int idx = axis == 0 ? hz : (axis == 1 ? HZ + hy : HZ + HY + hx);
       const uint4 x = *reinterpret_cast<uint4*>(ptr);
+      const float4* cs4 = reinterpret_cast<const float4*>(rope_s + idx * PR + p0);
+      const float4 ca = cs4[0], cb = cs4[1];
+      const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
       const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
       uint32_t xo[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 cs = rope_s[idx * PR + p0 + k];
         const float e0 = __uint_as_float(xin[k] << 16);
         const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
-        xo[k] = tc::pack_bf16(e0 * cs.x - e1 * cs.y, e0 * cs.y + e1 * cs.x);
+        xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1], e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
       }
       *reinterpret_cast<uint4*>(ptr) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
     };
     // q tile: row r <-> brick (2w + dz, y, x) <-> halo (2w + dz + 1, y + 1, x + 1)
-    for (int i = ptid; i < 128 * KC; i += 128) {
-      const int r = i / KC, kc = i % KC;
+    for (int i = ptid; i < 128 * KC; i += kProd) {
+      int r, kc;
+      tc::PieceOrder<KC>::at(i, r, kc);
       const int slot = slot_q[r];
       tc::cp_async16(smem + S::kQ + kc * 2048 + (r >> 3) * 128 + (r & 7) * 16,
                      qb + (int64_t)(slot >= 0 ? slot : 0) * D + kc * 8, slot >= 0);
@@ -344,27 +348,29 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     tc::cp_async_commit();
     tc::cp_async_wait_all();
 #pragma unroll 4
-    for (int i = ptid; i < 128 * KC; i += 128) {
-      const int r = i / KC, kc = i % KC;
-      if (slot_q[r] < 0) continue;
-      const int w = r >> 5, l = r & 31;
+    for (int i = ptid; i < 128 * KC; i += kProd) {
+      int r, kc;
+      tc::PieceOrder<KC>::at(i, r, kc);
+      const int w = r >> 5, l = r & 31;  // pieces of absent rows are zero and stay zero
       rotate_at(smem + S::kQ + kc * 2048 + (r >> 3) * 128 + (r & 7) * 16, 2 * w + (l >> 4) + 1,
                 ((l >> 2) & 3) + 1, (l & 3) + 1, kc);
     }
     tc::fence_proxy_async_smem();
     tc::mbar_arrive(&bars[B_QFULL]);
+    if (ptid == 0) P3D_TRACE(3002);
     // halo chunks: key kk of chunk c is halo key 72 c + kk = (2c + kk / 36, (kk / 6) % 6, kk % 6)
     for (int c = 0; c < kChunks; ++c) {
       const int st = c & 1;
       if (c >= 2) {
         if (ptid == 0) *prod_ok = ab.wait(&bars[B_KVEMPTY + st], ((c - 2) >> 1) & 1) ? 1 : 0;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 96;" ::: "memory");
         if (!*prod_ok) break;
       }
       uint8_t* ks = smem + S::kK + st * S::kCBytes;
       uint8_t* vs = smem + S::kV + st * S::kCBytes;
-      for (int i = ptid; i < kChunkPad * KC; i += 128) {
-        const int kk = i / KC, kc = i % KC;
+      for (int i = ptid; i < kChunkPad * KC; i += kProd) {
+        int kk, kc;
+        tc::PieceOrder<KC>::at(i, kk, kc);
         const int slot = kk < kChunkKeys ? slot_h[c * kChunkKeys + kk] : -1;
         const int off = kc * (kChunkPad * 16) + (kk >> 3) * 128 + (kk & 7) * 16;
         const int64_t src = (int64_t)(slot >= 0 ? slot : 0) * D + kc * 8;
@@ -372,18 +378,23 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
         tc::cp_async16(vs + off, vb + src, slot >= 0);
       }
       tc::cp_async_commit();
+      if (ptid == 0) P3D_TRACE(3010 + c * 4);
       tc::cp_async_wait_all();
+      if (ptid == 0) P3D_TRACE(3010 + c * 4 + 1);
 #pragma unroll 4
-      for (int i = ptid; i < kChunkPad * KC; i += 128) {
-        const int kk = i / KC, kc = i % KC;
-        if (kk >= kChunkKeys || slot_h[c * kChunkKeys + kk] < 0) continue;
+      for (int i = ptid; i < kChunkPad * KC; i += kProd) {
+        int kk, kc;
+        tc::PieceOrder<KC>::at(i, kk, kc);
+        // zero-filled pieces (absent or padding keys) rotate to zero; padding keys index a
+        // table row inside the 22-row table, so no guard is needed
         rotate_at(ks + kc * (kChunkPad * 16) + (kk >> 3) * 128 + (kk & 7) * 16,
                   2 * c + kk / kSliceKeys, (kk / HX) % HY, kk % HX, kc);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars[B_KVFULL + st]);
+      if (ptid == 0) P3D_TRACE(3010 + c * 4 + 2);
     }
-  } else if (warp == 8 && lane == 0) {
+  } else if (warp == 7 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunkPad, false, false);
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
@@ -392,6 +403,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     for (int c = 0; c < kChunks && ok; ++c) {
       const int st = c & 1;
       if (!ab.wait(&bars[B_KVFULL + st], (c >> 1) & 1)) break;
+      P3D_TRACE(3300 + c * 2);
       // S holds P_{c-1} until PV_{c-1} has completed
       if (c >= 1 && !ab.wait(&bars[B_PVDONE], (c - 1) & 1)) break;
       tc::tc_fence_after();
@@ -403,7 +415,9 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
         tc::mma_ss(tbase, a, b, id_qk, ks > 0);
       }
       tc::tc_commit(&bars[B_SFULL]);
+      P3D_TRACE(3200 + c * 4);
       if (!ab.wait(&bars[B_PFULL], c & 1)) break;
+      P3D_TRACE(3200 + c * 4 + 1);
       tc::tc_fence_after();
       const uint32_t vaddr = tc::smem_u32(smem + S::kV + st * S::kCBytes);
 #pragma unroll
@@ -413,6 +427,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
       }
       tc::tc_commit(&bars[B_PVDONE]);
       tc::tc_commit(&bars[B_KVEMPTY + st]);
+      P3D_TRACE(3200 + c * 4 + 2);
     }
   }
 
@@ -420,7 +435,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
   // softmax warps before their epilogue; on an abort, drain any MMA still in flight.
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 7) {
     if (*abort_flag && lane == 0) {
       // a bounded extra wait for the final PV; it arrives once every issued MMA has finished
       tc::mbar_wait(&bars[B_PVDONE], (kChunks - 1) & 1, 100000000LL);
@@ -469,3 +484,14 @@ cudaError_t local_tc_dispatch(const pack3d_index& ix, const void* q, const void*
 }
 
 }  // namespace p3d
+
+#ifdef P3D_TRACE_ENABLED
+extern "C" int p3d_trace_read_l(unsigned long long* host) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(host, p3d::g_trace, sizeof(unsigned long long) * 4096);
+}
+extern "C" int p3d_trace_clear_l() {
+  static unsigned long long z[4096];
+  return (int)cudaMemcpyToSymbol(p3d::g_trace, z, sizeof(z));
+}
+#endif

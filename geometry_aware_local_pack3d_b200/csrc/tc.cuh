@@ -46,6 +46,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe of a phase (no suspension: the caller spins and sees completion at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait: gives up after `budget` SM clock cycles (returns false); never traps.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           long long budget = 4000000000LL) {
@@ -75,6 +87,20 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
+
+// Conflict-free ordering of (row, 16-byte column) pieces for a warp-wide pass over rows of a
+// no-swizzle operand: each group of 32 consecutive items covers RG rows x KG columns, so the 8
+// rows of a core matrix land on 8 distinct 16-byte bank groups and each row is read as KG
+// contiguous pieces from global memory. `rows` must be a multiple of RG.
+template <int KC> struct PieceOrder {
+  static constexpr int KG = (KC % 4 == 0) ? 4 : 2;
+  static constexpr int RG = 32 / KG;
+  __device__ __forceinline__ static void at(int i, int& row, int& kc) {
+    const int g = i >> 5, l = i & 31;
+    row = (g / (KC / KG)) * RG + (l % RG);
+    kc = (g % (KC / KG)) * KG + l / RG;
+  }
+};
 
 // ------------------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
