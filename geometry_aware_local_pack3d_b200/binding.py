@@ -79,6 +79,9 @@ def lib():
         L.pack3d_attn_bwd.restype = st
         L.pack3d_attn_bwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, st, st, st,
                                       f32, u32, _P, _P, _P, _P, _P, sz, _P]
+        L.pack3d_attn_bwd_noalloc.restype = st
+        L.pack3d_attn_bwd_noalloc.argtypes = [ip, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, st,
+                                              st, st, f32, u32, _P, _P, _P, _P, _P]
         L.pack3d_device_status.restype = st
         L.pack3d_device_status.argtypes = [ip, _P]
         L.pack3d_last_launch_count.restype = ctypes.c_int
@@ -232,6 +235,27 @@ def pack3d_attn_bwd(index, q, k, v, gate, ksum, vsum, saved, dO, *, scale=None,
                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(workspace),
                                  workspace.numel(), _stream(stream)), "pack3d_attn_bwd")
     return dict(dq=dq, dk=dk, dv=dv, dgate=dgate)
+
+
+def pack3d_attn_bwd_noalloc(index, q, k, v, gate, ksum, vsum, saved, dO, *, scale=None,
+                            exclude_near=False, stream=None):
+    """pack3d_attn_bwd with the library's built-in scratch buffer (no workspace argument)."""
+    _need_cuda(q, k, v, gate, ksum, vsum, dO)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dgate = torch.empty_like(gate)
+    flags = PACK3D_EXCLUDE_NEAR if exclude_near else 0
+    _check(lib().pack3d_attn_bwd_noalloc(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(gate), _ptr(ksum), _ptr(vsum), _ptr(saved["o_loc"]),
+                                         _ptr(saved["o_glob"]), _ptr(saved["lse_loc"]),
+                                         _ptr(saved["lse_glob"]), _ptr(dO), _dtype_code(q), B, H,
+                                         scale, flags, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate),
+                                         _stream(stream)), "pack3d_attn_bwd_noalloc")
+    return dict(dq=dq, dk=dk, dv=dv, dgate=dgate)
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def pack3d_device_status(index, stream=None):

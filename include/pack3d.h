@@ -160,6 +160,29 @@ pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void
                               void* dq, void* dk, void* dv, void* dgate, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Largest backward workspace pack3d_attn_bwd_noalloc can serve from its built-in buffer. */
+#define PACK3D_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* pack3d_attn_bwd without a caller workspace. (The paper has no counterpart: this is a service
+ * for callers that cannot allocate device memory, e.g. a host framework that owns every device
+ * allocation through its own pool and forbids libraries to allocate, or a latency-critical loop
+ * that cannot take cudaMalloc's implicit synchronisation.)
+ * Same arguments and results as pack3d_attn_bwd, minus workspace/workspace_bytes. The scratch
+ * comes from one device array of PACK3D_NOALLOC_SCRATCH_BYTES bytes inside the library, which
+ * every device that loads the library keeps until the process exits; nothing is allocated.
+ * Returns PACK3D_ERR_WORKSPACE when pack3d_bwd_workspace_bytes(...) exceeds that size.
+ * The first call on a device (with that device current) looks the array's address up once
+ * (cudaGetSymbolAddress); make that first call before any stream capture on the device.
+ * All calls share the array and it keeps the last call's contents (the kernels overwrite all
+ * they read); calls that overlap on the GPU race on it, so order them on one stream. */
+pack3d_status pack3d_attn_bwd_noalloc(const pack3d_index* idx, const void* q, const void* k,
+                                      const void* v, const void* gate, const void* ksum,
+                                      const void* vsum, const void* o_loc, const void* o_glob,
+                                      const float* lse_loc, const float* lse_glob,
+                                      const void* dO, int dtype, int batch, int heads,
+                                      float scale, uint32_t flags, void* dq, void* dk, void* dv,
+                                      void* dgate, void* stream);
+
 /* Reads (after synchronising `stream`) and clears the index's device status word: OK, or
  * the first device-detected error (DUP_COORD, COORD_RANGE, TIMEOUT). */
 pack3d_status pack3d_device_status(const pack3d_index* idx, void* stream);
