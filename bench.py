@@ -246,7 +246,7 @@ def main():
     geom = p3d.make_geom(w["grid"], w["block"], d)
     ix = p3d.pack3d_build_index(geom, coords=torch.from_numpy(w["coords"]).to(dev))
     q, k, v, a = (w[n].to(dt).to(dev).contiguous() for n in "qkva")
-    ksum = torch.empty((B, H, ix.m, d), dtype=dt, device=dev)
+    ksum = torch.empty(p3d.summary_tiles_shape(ix, B, H, d), dtype=dt, device=dev)
     vsum = torch.empty_like(ksum)
     o = torch.empty_like(q)
     excl = w["exclude_near"]

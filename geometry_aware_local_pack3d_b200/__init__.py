@@ -7,5 +7,5 @@ from .binding import (  # noqa: F401
     Index, Pack3DError, PACK3D_BF16, PACK3D_EXCLUDE_NEAR, PACK3D_F32, make_geom, lib,
     pack3d_attn_bwd, pack3d_attn_bwd_noalloc, pack3d_attn_fwd, pack3d_build_index, pack3d_bwd_workspace_bytes,
     pack3d_device_status, pack3d_index_bytes, pack3d_last_launch_count, pack3d_strerror,
-    pack3d_summarize,
+    pack3d_summarize, pack3d_summary_bytes, summary_rows, summary_tiles_shape,
 )

@@ -74,6 +74,8 @@ def lib():
         L.pack3d_attn_fwd.restype = st
         L.pack3d_attn_fwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, st, st, st, f32, u32, _P, _P,
                                       _P, _P, _P, _P]
+        L.pack3d_summary_bytes.restype = sz
+        L.pack3d_summary_bytes.argtypes = [ip, st, st, st]
         L.pack3d_bwd_workspace_bytes.restype = sz
         L.pack3d_bwd_workspace_bytes.argtypes = [ip, st, st, st]
         L.pack3d_attn_bwd.restype = st
@@ -174,13 +176,36 @@ def pack3d_build_index(geom, coords=None, perm=None, stream=None):
     return Index(buf, st)
 
 
+def summary_tiles_shape(index, batch, heads, d):
+    """Shape of a summary buffer: [B, H, T, d/8, 64, 8] with T = ceil(M / 64) (summary tiles)."""
+    return (batch, heads, (index.m + 63) // 64, d // 8, 64, 8)
+
+
+def summary_rows(tiles, m):
+    """Plain [B, H, M, d] view (a copy) of a summary-tile buffer, for inspection and tests."""
+    B, H, T, dc, _, _ = tiles.shape
+    return tiles.permute(0, 1, 2, 4, 3, 5).reshape(B, H, T * 64, dc * 8)[:, :, :m]
+
+
+def pack3d_summary_bytes(index, dtype_code, batch, heads):
+    st = index.struct if isinstance(index, Index) else index
+    return int(lib().pack3d_summary_bytes(ctypes.byref(st), dtype_code, batch, heads))
+
+
 def pack3d_summarize(index, k, v, ksum=None, vsum=None, stream=None):
+    """Block summaries of k, v into summary-tile buffers (allocated here when not given)."""
     _need_cuda(k, v)
     B, H, N, d = k.shape
+    shape = summary_tiles_shape(index, B, H, d)
     if ksum is None:
-        ksum = torch.empty((B, H, index.m, d), dtype=k.dtype, device=k.device)
+        ksum = torch.empty(shape, dtype=k.dtype, device=k.device)
     if vsum is None:
-        vsum = torch.empty((B, H, index.m, d), dtype=k.dtype, device=k.device)
+        vsum = torch.empty(shape, dtype=k.dtype, device=k.device)
+    need = pack3d_summary_bytes(index, _dtype_code(k), B, H)
+    for t in (ksum, vsum):
+        if t.numel() * t.element_size() < need:
+            raise ValueError(f"summary buffer holds {t.numel() * t.element_size()} bytes, "
+                             f"needs {need}")
     _check(lib().pack3d_summarize(ctypes.byref(index.struct), _ptr(k), _ptr(v), _dtype_code(k),
                                   B, H, _ptr(ksum), _ptr(vsum), _stream(stream)),
            "pack3d_summarize")

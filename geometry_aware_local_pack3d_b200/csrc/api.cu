@@ -130,6 +130,13 @@ extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q,
                                        static_cast<cudaStream_t>(stream)));
 }
 
+extern "C" size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int batch,
+                                       int heads) {
+  if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;
+  const size_t elem = dtype == PACK3D_BF16 ? 2 : 4;
+  return (size_t)batch * heads * (size_t)sum_tiles(idx->m) * 64 * idx->geom.head_dim * elem;
+}
+
 extern "C" size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch,
                                              int heads) {
   if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;

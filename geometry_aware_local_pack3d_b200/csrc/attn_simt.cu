@@ -146,14 +146,14 @@ __global__ void __launch_bounds__(128) k_global_fwd(
 #pragma unroll
   for (int e = 0; e < D; ++e) acc[e] = 0.f;
 
-  const T* kb = ksum + bh * (int64_t)M * D;
-  const T* vb = vsum + bh * (int64_t)M * D;
+  const int64_t MT = sum_tiles(M);
   for (int m0 = 0; m0 < M; m0 += CH) {
     const int cnt = min(CH, M - m0);
     __syncthreads();
     for (int t = threadIdx.x; t < cnt * D; t += blockDim.x) {
-      sk[t / D][t % D] = to_f(kb[(int64_t)m0 * D + t]);
-      sv[t / D][t % D] = to_f(vb[(int64_t)m0 * D + t]);
+      const int64_t off = sum_index(bh, m0 + t / D, t % D, D, MT);
+      sk[t / D][t % D] = to_f(ksum[off]);
+      sv[t / D][t % D] = to_f(vsum[off]);
     }
     __syncthreads();
     if (!live) continue;
@@ -211,6 +211,15 @@ __device__ __forceinline__ void wr_load(const T* __restrict__ p, WarpRow<D>& r, 
   for (int t = 0; t < WarpRow<D>::KT; ++t) {
     const int e = lane + 32 * t;
     r.x[t] = e < D ? to_f(p[e]) : 0.f;
+  }
+}
+template <typename T, int D>
+__device__ __forceinline__ void wr_load_sum(const T* __restrict__ base, int64_t bh, int64_t m,
+                                            int64_t mt, WarpRow<D>& r, int lane) {
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) {
+    const int e = lane + 32 * t;
+    r.x[t] = e < D ? to_f(base[sum_index(bh, m, e, D, mt)]) : 0.f;
   }
 }
 template <int D>
@@ -317,8 +326,8 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
   const int64_t bh = task / M;
   const int m = (int)(task % M);
   WarpRow<D> km, vm, ak, av, x, d;
-  wr_load<T, D>(ksum + task * D, km, lane);
-  wr_load<T, D>(vsum + task * D, vm, lane);
+  wr_load_sum<T, D>(ksum, bh, m, sum_tiles(M), km, lane);
+  wr_load_sum<T, D>(vsum, bh, m, sum_tiles(M), vm, lane);
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
   for (int64_t i = 0; i < ix.n; ++i) {
@@ -389,8 +398,8 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
     const int M = (int)ix.m;
     for (int m = 0; m < M; ++m) {
       if (exclude_near && block_is_near(ix, m, c)) continue;
-      wr_load<T, D>(ksum + (bh * M + m) * D, x, lane);
-      wr_load<T, D>(vsum + (bh * M + m) * D, y, lane);
+      wr_load_sum<T, D>(ksum, bh, m, sum_tiles(M), x, lane);
+      wr_load_sum<T, D>(vsum, bh, m, sum_tiles(M), y, lane);
       const float p = expf(wr_dot<D>(qr, x) * scale - lg);
       const float ds = p * ((1.f - g) * wr_dot<D>(d, y) - Dg) * scale;
 #pragma unroll

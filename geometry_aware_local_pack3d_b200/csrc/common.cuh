@@ -55,19 +55,54 @@ __device__ __forceinline__ bool block_is_near(const pack3d_index& ix, int m, con
 
 __device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + __expf(-a)); }
 
+// Summary tiles: the M summaries of each (batch, head) are stored in tiles of 64 (zero padded
+// to a whole tile); a tile holds d/8 columns, each 64 summaries x 8 consecutive elements. This
+// is the no-swizzle tensor-core operand layout of a 64-summary chunk, so one contiguous copy
+// moves a chunk into shared memory. Element (bh, m, e) lives at this element offset:
+__host__ __device__ __forceinline__ int64_t sum_index(int64_t bh, int64_t m, int e, int d,
+                                                      int64_t m_tiles) {
+  return ((bh * m_tiles + (m >> 6)) * (d >> 3) + (e >> 3)) * 512 + (m & 63) * 8 + (e & 7);
+}
+__host__ __device__ __forceinline__ int64_t sum_tiles(int64_t m) { return (m + 63) >> 6; }
+
 // Phase timestamps for one CTA, compiled in only by a tracing build (P3D_TRACE_ENABLED):
 // the kernels mark their handoffs with P3D_TRACE(slot); normal builds emit nothing.
 #ifdef P3D_TRACE_ENABLED
+#ifndef P3D_TRACE_CTA
+#define P3D_TRACE_CTA 0
+#endif
 static __device__ unsigned long long g_trace[4096];
 #define P3D_TRACE(slot)                                                            \
   do {                                                                             \
-    if (blockIdx.x == 0) {                                                         \
+    if (blockIdx.x == (P3D_TRACE_CTA)) {                                           \
       unsigned long long t_;                                                       \
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
       g_trace[(slot) & 4095] = t_;                                                 \
     }                                                                              \
   } while (0)
+// SM clock next to the global timer, for measuring the clock a kernel actually runs at
+#define P3D_TRACE_CLK(slot)                                                        \
+  do {                                                                             \
+    if (blockIdx.x == (P3D_TRACE_CTA)) {                                           \
+      unsigned long long t_;                                                       \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
+      g_trace[(slot) & 4095] = t_;                                                 \
+      g_trace[((slot) + 1) & 4095] = (unsigned long long)clock64();                \
+    }                                                                              \
+  } while (0)
+// SM clock only (fine-grained intervals inside one role)
+#define P3D_TRACE_C(slot)                                                          \
+  do {                                                                             \
+    if (blockIdx.x == (P3D_TRACE_CTA))                                             \
+      g_trace[(slot) & 4095] = (unsigned long long)clock64();                      \
+  } while (0)
 #else
+#define P3D_TRACE_C(slot) \
+  do {                    \
+  } while (0)
+#define P3D_TRACE_CLK(slot) \
+  do {                      \
+  } while (0)
 #define P3D_TRACE(slot) \
   do {                  \
   } while (0)

@@ -8,17 +8,21 @@
 // Work unit: 256 consecutive memory rows of one (batch, head) = two 128-row query tiles that
 // share every summary chunk (halves the L2 reads of the summaries). Persistent CTAs walk the
 // units round-robin. Warp roles (448 threads):
-//   warps 0-3   softmax + epilogue of tile 0 (thread = row, TMEM lanes 0..127)
+//   warps 0-3   softmax + epilogue of tile 0 (thread = row, TMEM lanes 0..127); the epilogue
+//               parks o_glob in the tile's (by then consumed) q area and applies the mixer
+//               with coalesced loads and stores, then releases the q buffer to the producer
 //   warps 4-7   softmax + epilogue of tile 1
 //   warps 8-11  query producer: cp.async of q rows into the K-major shared-memory A operand
 //               (double-buffered across units), then axial RoPE applied in place
 //   warp 12     MMA issuer (one thread) and TMEM owner
-//   warp 13     TMA producer: 64-summary chunks of ksum / vsum into a 4-stage ring
+//   warp 13     summary loader: each 64-summary chunk of ksum / vsum is one summary tile, i.e.
+//               already in the operand layout, fetched by one contiguous bulk copy per tensor
+//               into a 4-stage ring
 // Per 64-summary chunk j and tile t:  S_t[j%2] = q~_t K_j^T (SS MMA, fp32 in TMEM) -> the
 // softmax threads turn it into P = exp2(s - m) in bf16, written over S in TMEM ->
-// O_t += P V_j (TS MMA). S is double-buffered, and the issuer runs one chunk ahead (QK of
-// chunk j+1 is issued before the PV of chunk j), so the softmax of consecutive chunks runs
-// back to back while the tensor core works in its shadow. The running max uses a lazy
+// O_t += P V_j (TS MMA). S is double-buffered per tile; the issuer runs QK two chunks ahead
+// (PV_0(j), PV_1(j), QK_0(j+2), QK_1(j+2)), so the next S of a tile is ready when its softmax
+// finishes a chunk, and the two tiles' softmaxes overlap each other. The running max uses a lazy
 // rescale: O_t is corrected in TMEM only when a row's max grows by more than 2^8.
 // The summary order is the same for every query (block ids ascending) and rows never interact,
 // so a coordinate-carrying repack permutes the output bit for bit.
@@ -74,6 +78,8 @@ enum {
 struct Params {
   pack3d_index ix;
   const __nv_bfloat16* q;
+  const __nv_bfloat16* ksum;   // summary tiles
+  const __nv_bfloat16* vsum;
   const __nv_bfloat16* gate;
   const __nv_bfloat16* o_loc;  // may alias o
   __nv_bfloat16* o;
@@ -96,10 +102,14 @@ __device__ __forceinline__ float ex2(float x) {
 struct Abort {
   volatile int* flag;
   int32_t* status;
-  __device__ bool wait(uint64_t* bar, uint32_t parity) {
+  // Probing wait (a suspended try_wait wakes up measurably later). With `nap`, a short
+  // nanosleep between probes leaves the issue slots of the SM sub-partition to the warps that
+  // are working, above all the single MMA-issuing thread; the issuer itself waits without it.
+  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
     if (tc::mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!tc::mbar_test_wait(bar, parity)) {
+      if (nap) __nanosleep(32);
       if (*flag) return false;
       if (clock64() - t0 > 4000000000LL) {
         *flag = 1;
@@ -115,8 +125,7 @@ struct Abort {
 
 template <int D>
 __global__ void __launch_bounds__(gtc::kThreads, 1)
-    k_global_tc(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                const gtc::Params P) {
+    k_global_tc(const gtc::Params P) {
   using namespace gtc;
   using S = Smem<D>;
   constexpr int KC = D / 8;  // 16-byte chunks per row
@@ -133,7 +142,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bars[B_QFULL + i], kProd);
-      tc::mbar_init(&bars[B_QEMPTY + i], 1);
+      tc::mbar_init(&bars[B_QEMPTY + i], kRows * kTiles);
       tc::mbar_init(&bars[B_OFREE + i], 128);
     }
     for (int i = 0; i < 4; ++i) {
@@ -195,6 +204,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           break;
         }
         if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2);
+        if (rin == 0 && pc == 1 && j < 10) P3D_TRACE_C(3400 + j * 4 + t * 2);
         tc::tc_fence_after();
         const int m0 = j * kChunk;
         const int ncol = min(kChunk, M - m0);
@@ -214,8 +224,11 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         const bool masked = any_x || ncol < kChunk;
         // the 64-column chunk in registers; masked entries become -inf in place
         uint32_t r[kChunk];
+        const bool fine = rin == 0 && t == 0 && pc == 1 && j >= 2 && j < 6;  // fine trace points
+        if (fine) P3D_TRACE(1800 + j * 8);
         tc::tmem_ld64(tl + s_col(t, b), r);
         tc::tmem_wait_ld();
+        if (fine) P3D_TRACE(1800 + j * 8 + 1);
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (!masked) {
 #pragma unroll
@@ -230,6 +243,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         // row max in the log2 domain (the scale is positive)
         const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
         const float m_new = fmaxf(m_run, cmax);
+        if (fine) P3D_TRACE(1800 + j * 8 + 2);
         const bool need = m_new > m_run + kRescaleLog2;  // false while everything is masked
         if (__any_sync(0xffffffffu, need) && j > 0) {
           // O_t holds sum_{<j} P V with the old max: wait for the previous PV, then rescale
@@ -272,10 +286,13 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           tc::tmem_st16(tl + s_col(t, b) + (c0 >> 1), p);
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        if (fine) P3D_TRACE(1800 + j * 8 + 3);
         tc::tmem_wait_st();
+        if (fine) P3D_TRACE(1800 + j * 8 + 4);
         tc::tc_fence_before();
         tc::mbar_arrive(&bars[B_PFULL + 2 * t + b]);
         if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2 + 1);
+        if (rin == 0 && pc == 1 && j < 10) P3D_TRACE_C(3400 + j * 4 + t * 2 + 1);
       }
       if (!ok) break;
       // epilogue: o_glob = O / l, lse, mixer
@@ -299,32 +316,59 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(&bars[B_OFREE + t]);
       if (rin == 0 && pc < 3) P3D_TRACE(1500 + pc * 4 + t * 2);
+      // Mixer, coalesced: the unit's last QK has completed (its PV is done), so this tile's q
+      // area in shared memory is free and holds exactly 128 rows of D bf16. Each thread parks
+      // its o_glob row there (16-byte chunk c of row r at chunk slot (c + r) mod KC, which
+      // spreads a warp's stores over the banks); each warp then walks its 32 rows piece by
+      // piece, so consecutive lanes touch consecutive 16 bytes of o_loc, o and o_glob.
+      uint8_t* stage = smem + S::kQ + (pc & 1) * kTiles * S::kQTile + t * S::kQTile;
+      tc::fence_proxy_async_smem();  // the tensor core's reads of this area came first
+#pragma unroll
+      for (int c = 0; c < KC; ++c)
+        *reinterpret_cast<uint4*>(stage + rin * (D * 2) + ((c + rin) % KC) * 16) =
+            make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
+      float gsig = 0.f;
       if (valid) {
         const int64_t grow = bh * N + row;
         if (P.lse_glob)
           P.lse_glob[grow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-        const float a = __bfloat162float(P.gate[grow]);
-        const float g = 1.f / (1.f + __expf(-a));
-        const uint4* ol = reinterpret_cast<const uint4*>(P.o_loc + grow * D);
-        uint4* oo = reinterpret_cast<uint4*>(P.o + grow * D);
-        uint4* og = P.o_glob ? reinterpret_cast<uint4*>(P.o_glob + grow * D) : nullptr;
-#pragma unroll
-        for (int c = 0; c < KC; ++c) {
-          const uint4 lv = ol[c];
-          const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-          uint32_t outw[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t gw = gp[4 * c + k];
-            const float g0 = __uint_as_float(gw << 16), g1 = __uint_as_float(gw & 0xffff0000u);
-            const float l0 = __uint_as_float(lw[k] << 16);
-            const float l1 = __uint_as_float(lw[k] & 0xffff0000u);
-            outw[k] = tc::pack_bf16(g * l0 + (1.f - g) * g0, g * l1 + (1.f - g) * g1);
-          }
-          oo[c] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          if (og) og[c] = make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
-        }
+        gsig = 1.f / (1.f + __expf(-__bfloat162float(P.gate[grow])));
       }
+      __syncwarp();
+      const int wr0 = (warp & 3) * 32;  // the warp's first row within the tile
+      const int64_t row_w = row - lane;  // memory row of the warp's first row
+      // o_loc may alias o (in-place mixing): every piece a lane stores is one it loaded itself,
+      // and all of its loads come first
+      uint4 lrow[KC];
+#pragma unroll
+      for (int i = 0; i < KC; ++i) {
+        const int pidx = i * 32 + lane, r = pidx / KC, c = pidx % KC;
+        lrow[i] = row_w + r < N
+                      ? reinterpret_cast<const uint4*>(P.o_loc + (bh * N + row_w + r) * D)[c]
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < KC; ++i) {
+        const int pidx = i * 32 + lane, r = pidx / KC, c = pidx % KC;
+        const float g = __shfl_sync(0xffffffffu, gsig, r);
+        const uint4 gv = *reinterpret_cast<const uint4*>(stage + (wr0 + r) * (D * 2) +
+                                                         ((c + wr0 + r) % KC) * 16);
+        if (row_w + r >= N) continue;
+        const uint32_t lw[4] = {lrow[i].x, lrow[i].y, lrow[i].z, lrow[i].w};
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint32_t outw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float g0 = __uint_as_float(gw[k] << 16), g1 = __uint_as_float(gw[k] & 0xffff0000u);
+          const float l0 = __uint_as_float(lw[k] << 16), l1 = __uint_as_float(lw[k] & 0xffff0000u);
+          outw[k] = tc::pack_bf16(g * l0 + (1.f - g) * g0, g * l1 + (1.f - g) * g1);
+        }
+        const int64_t off = (bh * N + row_w + r) * D;
+        reinterpret_cast<uint4*>(P.o + off)[c] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        if (P.o_glob) reinterpret_cast<uint4*>(P.o_glob + off)[c] = gv;
+      }
+      // this thread's reads of the q area are done: the producer may refill it
+      tc::mbar_arrive(&bars[B_QEMPTY + (pc & 1)]);
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------------ query producer
@@ -395,91 +439,112 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
-      const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
-      int pc = 0;
-      uint32_t kv_it = 0;
-      bool issued = false, ok = true;
-      for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++pc) {
-        const int qb = pc & 1;
-        if (!ab.wait(&bars[B_QFULL + qb], (pc >> 1) & 1)) break;
-        if (pc < 3) P3D_TRACE(2600 + pc);
+    // Fixed order per chunk j: PV_0(j), PV_1(j), then QK_0(j+2), QK_1(j+2). QK_t(j+2) reuses
+    // the S buffer of chunk j, so it only waits for PV_t(j) to complete; it is thus issued
+    // while the softmax of tile t works on chunk j+1, and S_t(j+2) is ready when that softmax
+    // finishes. The whole warp runs the schedule with warp-uniform values (descriptors are
+    // formed once and advanced by adding address offsets: the start address is the low 14
+    // bits and every offset keeps it in range); one elected lane issues the tcgen05 MMAs and
+    // commits. This keeps the issuing instruction stream short and uniform.
+    const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
+    const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
+    const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
+    const uint64_t kd0 = tc::smem_desc(tc::smem_u32(smem + S::kK), CB, 128);
+    const uint64_t vd0 = tc::smem_desc(tc::smem_u32(smem + S::kV), 128, CB);
+    // every lane probes; the verdict is the same on all lanes
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, ab.wait(bar, parity, false));
+    };
+    int pc = 0;
+    uint32_t kv_it = 0;
+    bool issued = false, ok = true;
+    for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++pc) {
+      const int qb = pc & 1;
+      if (!wwait(&bars[B_QFULL + qb], (pc >> 1) & 1)) break;
+      if (lane == 0 && pc < 3) P3D_TRACE(2600 + pc);
+      tc::tc_fence_after();
+      const uint64_t qd0 =
+          tc::smem_desc(tc::smem_u32(smem + S::kQ + qb * kTiles * S::kQTile), 2048, 128);
+      // QK_t(j): S_t[buffer of j] = q~_t K_j^T
+      auto issue_qk = [&](int t, int j) -> bool {
+        const uint32_t kv = kv_it + j;
+        const uint32_t gi = (uint32_t)(pc * NC + j);
+        const int b = gi & 1;
+        const bool fq = lane == 0 && pc == 1 && j >= 4 && j < 8;
+        const int fs = 3000 + j * 40 + t * 10;
+        if (fq) P3D_TRACE_C(fs);
+        if (t == 0 && !wwait(&bars[B_KVFULL + kv % kStages], (kv / kStages) & 1)) return false;
+        if (fq) P3D_TRACE_C(fs + 1);
+        // this S buffer held P of chunk gi - 2 until that PV completed
+        if (gi >= 2 && !wwait(&bars[B_PVDONE + 2 * t + b], ((gi >> 1) - 1) & 1)) return false;
+        if (fq) P3D_TRACE_C(fs + 2);
         tc::tc_fence_after();
-        const uint32_t qaddr = tc::smem_u32(smem + S::kQ + qb * kTiles * S::kQTile);
-        // QK of chunk j is issued one step ahead of the PV of chunk j - 1
-        for (int j = 0; j <= NC && ok; ++j) {
-          if (j < NC) {
-            const uint32_t kv = kv_it + j;
-            const int st = kv % kStages;
-            if (!ab.wait(&bars[B_KVFULL + st], (kv / kStages) & 1)) { ok = false; break; }
-            if (pc < 3) P3D_TRACE(2500 + pc * 32 + j);
-            tc::tc_fence_after();
-            const uint32_t kaddr = tc::smem_u32(smem + S::kK + st * S::kCTile);
-            const uint32_t gi = (uint32_t)(pc * NC + j);
-            const int b = gi & 1;
-            for (int t = 0; t < kTiles; ++t) {
-              // this S buffer held P of chunk gi - 2: free once that PV has completed
-              if (gi >= 2 && !ab.wait(&bars[B_PVDONE + 2 * t + b], ((gi >> 1) - 1) & 1)) {
-                ok = false;
-                break;
-              }
-              tc::tc_fence_after();
+        const uint64_t a0 = qd0 + (uint64_t)((t * S::kQTile) >> 4);
+        const uint64_t b0 = kd0 + (uint64_t)(((kv % kStages) * S::kCTile) >> 4);
+        const uint32_t dt = tb + s_col(t, b);
+        if (tc::elect_one()) {
 #pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t a =
-                    tc::smem_desc(qaddr + t * S::kQTile + ks * 4096, 2048, 128);
-                const uint64_t bd = tc::smem_desc(kaddr + ks * 2 * CB, CB, 128);
-                tc::mma_ss(tbase + s_col(t, b), a, bd, id_qk, ks > 0);
-              }
-              tc::tc_commit(&bars[B_SFULL + 2 * t + b]);
-              if (pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2);
-              issued = true;
-            }
-            if (!ok) break;
-          }
-          if (j >= 1) {
-            const int jj = j - 1;
-            const uint32_t kv = kv_it + jj;
-            const int st = kv % kStages;
-            const uint32_t vaddr = tc::smem_u32(smem + S::kV + st * S::kCTile);
-            const uint32_t gi = (uint32_t)(pc * NC + jj);
-            const int b = gi & 1;
-            for (int t = 0; t < kTiles; ++t) {
-              if (!ab.wait(&bars[B_PFULL + 2 * t + b], (gi >> 1) & 1)) { ok = false; break; }
-              if (jj == 0 && pc > 0 && !ab.wait(&bars[B_OFREE + t], (pc - 1) & 1)) {
-                ok = false;
-                break;
-              }
-              tc::tc_fence_after();
-#pragma unroll
-              for (int ks = 0; ks < kChunk / 16; ++ks) {
-                const uint64_t bd = tc::smem_desc(vaddr + ks * 256, 128, CB);
-                tc::mma_ts(tbase + o_col(t), tbase + s_col(t, b) + ks * 8, bd, id_pv,
-                           (jj > 0 || ks > 0) ? 1u : 0u);
-              }
-              tc::tc_commit(&bars[B_PVDONE + 2 * t + b]);
-              if (pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + jj * 2 + 1);
-            }
-            if (!ok) break;
-            tc::tc_commit(&bars[B_KVEMPTY + st]);
-          }
+          for (int ks = 0; ks < D / 16; ++ks)
+            tc::mma_ss(dt, a0 + (uint64_t)(ks * (4096 >> 4)),
+                       b0 + (uint64_t)(ks * (2 * CB >> 4)), id_qk, ks > 0);
+          tc::tc_commit(&bars[B_SFULL + 2 * t + b]);
         }
-        kv_it += NC;
+        __syncwarp();
+        if (fq) P3D_TRACE_C(fs + 4);
+        if (lane == 0 && pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2);
+        if (lane == 0 && pc < 3 && t == 0) P3D_TRACE(2500 + pc * 32 + j);
+        if (lane == 0 && pc == 1 && j == 0 && t == 0) P3D_TRACE_CLK(3900);
+        if (lane == 0 && pc == 8 && j == 0 && t == 0) P3D_TRACE_CLK(3902);
+        issued = true;
+        return true;
+      };
+      for (int j = 0; j < 2 && j < NC && ok; ++j)
+        for (int t = 0; t < kTiles && ok; ++t) ok = issue_qk(t, j);
+      for (int j = 0; j < NC && ok; ++j) {
+        const uint32_t kv = kv_it + j;
+        const uint32_t gi = (uint32_t)(pc * NC + j);
+        const int b = gi & 1;
+        const uint64_t v0 = vd0 + (uint64_t)(((kv % kStages) * S::kCTile) >> 4);
+        for (int t = 0; t < kTiles; ++t) {
+          const bool fp = lane == 0 && pc == 1 && j >= 2 && j < 6;
+          const int fs = 3000 + (j + 2) * 40 + 20 + t * 10;
+          if (fp) P3D_TRACE_C(fs);
+          if (!wwait(&bars[B_PFULL + 2 * t + b], (gi >> 1) & 1)) { ok = false; break; }
+          if (fp) P3D_TRACE_C(fs + 1);
+          // the first PV of a unit overwrites O_t: the previous epilogue must have read it
+          if (j == 0 && pc > 0 && !wwait(&bars[B_OFREE + t], (pc - 1) & 1)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t at = tb + s_col(t, b), dt = tb + o_col(t);
+          if (tc::elect_one()) {
+#pragma unroll
+            for (int ks = 0; ks < kChunk / 16; ++ks)
+              tc::mma_ts(dt, at + ks * 8, v0 + (uint64_t)(ks * (256 >> 4)), id_pv,
+                         (j > 0 || ks > 0) ? 1u : 0u);
+            tc::tc_commit(&bars[B_PVDONE + 2 * t + b]);
+          }
+          __syncwarp();
+          if (fp) P3D_TRACE_C(fs + 4);
+          if (lane == 0 && pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2 + 1);
+        }
         if (!ok) break;
-        tc::tc_commit(&bars[B_QEMPTY + qb]);
+        // both tiles' PVs of chunk j are issued: the stage is free once they complete
+        if (tc::elect_one()) tc::tc_commit(&bars[B_KVEMPTY + kv % kStages]);
+        __syncwarp();
+        if (j + 2 < NC)
+          for (int t = 0; t < kTiles && ok; ++t) ok = issue_qk(t, j + 2);
       }
-      // every MMA issued by this thread has completed before TMEM is released
-      if (issued) {
-        tc::tc_commit(&bars[B_DONE]);
-        tc::mbar_wait(&bars[B_DONE], 0, 4000000000LL);
-      }
+      kv_it += NC;
+    }
+    // every MMA issued by this warp has completed before TMEM is released
+    if (issued) {
+      if (tc::elect_one()) tc::tc_commit(&bars[B_DONE]);
+      __syncwarp();
+      tc::mbar_wait(&bars[B_DONE], 0, 4000000000LL);
     }
   } else {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ summary loader
     if (lane == 0) {
-      tc::tma_prefetch_desc(&map_k);
-      tc::tma_prefetch_desc(&map_v);
+      const int64_t MT = sum_tiles(M);
       uint32_t kv_it = 0;
       for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x) {
         const int64_t bh = u / P.units_per_bh;
@@ -489,18 +554,15 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           if (kv_it >= (uint32_t)kStages &&
               !ab.wait(&bars[B_KVEMPTY + st], ((kv_it / kStages) - 1) & 1)) { ok = false; break; }
           tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kCTile);
-          const int y = (int)(bh * M + j * kChunk);
-          uint8_t* kd = smem + S::kK + st * S::kCTile;
-          uint8_t* vd = smem + S::kV + st * S::kCTile;
-#pragma unroll
-          for (int kc = 0; kc < KC; ++kc) {
-            tc::tma_load_2d(kd + kc * CB, &map_k, 8 * kc, y, &bars[B_KVFULL + st]);
-            tc::tma_load_2d(vd + kc * CB, &map_v, 8 * kc, y, &bars[B_KVFULL + st]);
-          }
+          const int64_t tile = (bh * MT + j) * (int64_t)(kChunk * D);  // element offset
+          tc::bulk_g2s(smem + S::kK + st * S::kCTile, P.ksum + tile, S::kCTile,
+                       &bars[B_KVFULL + st]);
+          tc::bulk_g2s(smem + S::kV + st * S::kCTile, P.vsum + tile, S::kCTile,
+                       &bars[B_KVFULL + st]);
         }
         if (!ok) break;
       }
-      // the last loads issued to each stage have landed before the CTA may exit
+      // the last copies issued to each stage have landed before the CTA may exit
       for (uint32_t k = (kv_it > (uint32_t)kStages ? kv_it - kStages : 0); k < kv_it; ++k)
         tc::mbar_wait(&bars[B_KVFULL + (k % kStages)], (k / kStages) & 1, 4000000000LL);
     }
@@ -515,53 +577,6 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ host side
-namespace {
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, D] bf16 row-major viewed as 2D; box = 8 columns x 64 rows (one 16-byte column of
-// core matrices of a summary chunk), no swizzle.
-bool encode_rows(CUtensorMap* map, const void* base, int64_t rows, int D) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {8, (cuuint32_t)gtc::kChunk};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-}  // namespace
 
 template <int D>
 cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* gate,
@@ -569,9 +584,6 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
                              float scale, int excl, void* o, float* lse_glob, void* o_glob,
                              cudaStream_t s) {
   using namespace gtc;
-  CUtensorMap mk, mv;
-  if (!encode_rows(&mk, ksum, bh * ix.m, D) || !encode_rows(&mv, vsum, bh * ix.m, D))
-    return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(k_global_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -582,6 +594,8 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   Params p;
   p.ix = ix;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.ksum = static_cast<const __nv_bfloat16*>(ksum);
+  p.vsum = static_cast<const __nv_bfloat16*>(vsum);
   p.gate = static_cast<const __nv_bfloat16*>(gate);
   p.o_loc = static_cast<const __nv_bfloat16*>(o_loc);
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -594,7 +608,7 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   p.n_chunks = (int)((ix.m + kChunk - 1) / kChunk);
   p.rope_in_smem = (int64_t)ix.rope_rows * ix.rope_pairs * 8 <= kRopeSmemBytes ? 1 : 0;
   const int grid = (int)(p.units < sm_count() ? p.units : sm_count());
-  k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mk, mv, p);
+  k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(p);
   count_launch();
   return cudaGetLastError();
 }

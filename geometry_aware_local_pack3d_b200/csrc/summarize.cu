@@ -1,5 +1,6 @@
 // Rotate-then-pool block summaries (project page "Geometry Matters in Packed 3D Attention",
-// Chapter 3 "Rotate first, then pool"; paper summary §3.2 and §B.5).
+// Chapter 3 "Rotate first, then pool"; paper summary §3.2 and §B.5), written in summary tiles
+// (see sum_index in common.cuh; the tail of the last tile is written as zeros).
 //
 //   ksum[b,h,m] = (1/|S_m|) sum_{s} R(c_j) k[b,h,j],   vsum[b,h,m] = (1/|S_m|) sum_{s} v[b,h,j]
 //   with j = members[m][s], s the canonical slot.
@@ -7,7 +8,8 @@
 // HBM-bound: every k and v row is read exactly once with 16-byte vector loads. One warp per
 // summary: lane l handles 16-byte chunk (l % C) of member rows s = l / C, l / C + R, ...
 // (C chunks per row, R = 32 / C rows per pass); the R partial sums are then combined in fixed
-// order with warp shuffles. The summation order depends on canonical slots only, never on
+// order with warp shuffles. Absent members (and the zero padding of the last summary tile)
+// contribute with weight 0. The summation order depends on canonical slots only, never on
 // memory slots, so a coordinate-carrying repack gives bit-identical summaries.
 #include "common.cuh"
 #include "launch.h"
@@ -27,9 +29,10 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
   const int lane = threadIdx.x & 31;
   const int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t M = ix.m;
-  if (task >= bh_count * M) return;
-  const int64_t bh = task / M;
-  const int m = (int)(task % M);
+  const int64_t MT = sum_tiles(M);
+  if (task >= bh_count * MT * 64) return;
+  const int64_t bh = task / (MT * 64);
+  const int m = (int)(task % (MT * 64));  // m >= M: zero padding of the last tile
   const int vol = ix.block_volume;
   const int r = lane / C, c = lane % C;
   const bool active = r < R;
@@ -42,23 +45,35 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
 
   const T* kb = k + bh * ix.n * D;
   const T* vb = v + bh * ix.n * D;
-  if (active) {
-#pragma unroll 4
-    for (int s = r; s < vol; s += R) {
-      const int j = ix.members[(int64_t)m * vol + s];
-      if (j < 0) continue;
-      const Coord cj = decode(ix.coord[j]);
-      const int cv = coord_axis(cj, axis);
+  // Members are taken 32 at a time: lane l fetches the slot and coordinate of member b0 + l
+  // once, and every lane then reads them by shuffle, so the 16-byte k/v loads of many members
+  // are independent and in flight together (the loop body has no branch).
+  for (int b0 = 0; b0 < vol; b0 += 32) {
+    int jl = -1;
+    int32_t cl = 0;
+    if (m < M && b0 + lane < vol) {
+      jl = ix.members[(int64_t)m * vol + b0 + lane];
+      if (jl >= 0) cl = ix.coord[jl];
+    }
+#pragma unroll 8
+    for (int i = 0; i < (32 + R - 1) / R; ++i) {
+      const int sl = r + R * i;  // member b0 + sl, canonical-slot order within this lane
+      const int j = __shfl_sync(0xffffffffu, jl, sl & 31);
+      const int32_t cc = __shfl_sync(0xffffffffu, cl, sl & 31);
+      const bool use = active && sl < 32 && b0 + sl < vol && j >= 0;
+      const int64_t row = use ? j : 0;
+      const float wgt = use ? 1.f : 0.f;
+      const int cv = coord_axis(decode(cc), axis);
       float xk[E], xv[E];
-      Vec<T>::load(kb + (int64_t)j * D + c * E, xk);
-      Vec<T>::load(vb + (int64_t)j * D + c * E, xv);
+      Vec<T>::load(kb + row * D + c * E, xk);
+      Vec<T>::load(vb + row * D + c * E, xv);
 #pragma unroll
       for (int e = 0; e < E; e += 2) {
-        const float2 cs = rope_cs(ix.rope, ix.rope_pairs, cv, p0 + e / 2);
-        ak[e] += xk[e] * cs.x - xk[e + 1] * cs.y;
-        ak[e + 1] += xk[e] * cs.y + xk[e + 1] * cs.x;
-        av[e] += xv[e];
-        av[e + 1] += xv[e + 1];
+        const float2 cs = rope_cs(ix.rope, ix.rope_pairs, use ? cv : 0, p0 + e / 2);
+        ak[e] += wgt * (xk[e] * cs.x - xk[e + 1] * cs.y);
+        ak[e + 1] += wgt * (xk[e] * cs.y + xk[e + 1] * cs.x);
+        av[e] += wgt * xv[e];
+        av[e + 1] += wgt * xv[e + 1];
       }
     }
   }
@@ -79,22 +94,22 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
     }
   }
   if (r == 0) {
-    const int cnt = ix.count[m];
+    const int cnt = m < M ? ix.count[m] : 0;
     const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       ak[e] *= inv;
       av[e] *= inv;
     }
-    Vec<T>::store(ksum + (bh * M + m) * D + c * E, ak);
-    Vec<T>::store(vsum + (bh * M + m) * D + c * E, av);
+    Vec<T>::store(ksum + sum_index(bh, m, c * E, D, MT), ak);
+    Vec<T>::store(vsum + sum_index(bh, m, c * E, D, MT), av);
   }
 }
 
 template <typename T, int D>
 cudaError_t launch_summarize(const pack3d_index& ix, const void* k, const void* v, int64_t bh,
                              void* ksum, void* vsum, cudaStream_t s) {
-  const int64_t tasks = bh * ix.m;
+  const int64_t tasks = bh * sum_tiles(ix.m) * 64;
   const unsigned blocks = (unsigned)((tasks + 3) / 4);
   k_summarize<T, D><<<blocks, 128, 0, s>>>(ix, static_cast<const T*>(k), static_cast<const T*>(v),
                                             bh, static_cast<T*>(ksum), static_cast<T*>(vsum));

@@ -16,8 +16,14 @@
  *
  * Conventions shared by every call:
  *   - Tensors are dense, row-major [B, H, N, d] with N in MEMORY order (the packing);
- *     gate logits are [B, H, N]; lse outputs are float32 [B, H, N]. Summaries are
- *     [B, H, M, d] with M = number of blocks, block ids raster over the block grid.
+ *     gate logits are [B, H, N]; lse outputs are float32 [B, H, N].
+ *   - Summaries (ksum, vsum) hold M = number of blocks summaries per (b, h), block ids raster
+ *     over the block grid, in SUMMARY TILES: the summaries of each (b, h) are grouped in tiles
+ *     of 64 (the last tile zero-padded); a tile is d/8 columns of 64 summaries x 8 consecutive
+ *     elements. Element (b, h, m, e) sits at element offset
+ *         (((b*H + h)*T + m/64)*(d/8) + e/8)*512 + (m%64)*8 + e%8,   T = ceil(M/64),
+ *     and a buffer takes pack3d_summary_bytes(...) bytes. A tile is exactly the tensor-core
+ *     operand layout of a 64-summary chunk, so the forward moves it with one bulk copy.
  *   - dtype: PACK3D_F32 or PACK3D_BF16 for q, k, v, gate, summaries, outputs and gradients.
  *     All accumulation, softmax and logsumexp run in float32.
  *   - Pointers marked "device" must be device (or managed) memory of the current device;
@@ -118,7 +124,8 @@ pack3d_status pack3d_build_index(const pack3d_geom* g, const int32_t* coords,
 /* Rotate-then-pool block summaries: ksum[m] = mean over members j of R(c_j) k_j and
  * vsum[m] = mean of v_j, summed in canonical-slot order (project page Ch.3 "Rotate first,
  * then pool"; paper summary §3.2, §B.5).
- * k, v       device [B, H, N, d] dtype;  ksum, vsum device [B, H, M, d] dtype (outputs). */
+ * k, v       device [B, H, N, d] dtype;  ksum, vsum device summary tiles, dtype, each of
+ *            pack3d_summary_bytes(idx, dtype, B, H) bytes (outputs; the padding is zeroed). */
 pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const void* v,
                                int dtype, int batch, int heads, void* ksum, void* vsum,
                                void* stream);
@@ -126,7 +133,7 @@ pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const voi
 /* PACK3D forward: local branch + global branch over (ksum, vsum) + sigmoid mixer
  * (project page Ch.3 Contracts 1-3; paper summary §3.2, §3.3, §3.5).
  * q, k, v    device [B, H, N, d] dtype;  gate device [B, H, N] dtype (logits a).
- * ksum, vsum device [B, H, M, d] dtype from pack3d_summarize of the same k, v.
+ * ksum, vsum device summary tiles from pack3d_summarize of the same k, v.
  * scale      softmax scale tau (both branches); pass 1/sqrt(d) for the usual choice.
  * flags      0 or PACK3D_EXCLUDE_NEAR.
  * o          device [B, H, N, d] dtype (output).
@@ -140,6 +147,10 @@ pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void
                               const void* vsum, int dtype, int batch, int heads, float scale,
                               uint32_t flags, void* o, float* lse_loc, float* lse_glob,
                               void* o_loc, void* o_glob, void* stream);
+
+/* Bytes of one summary buffer (ksum or vsum) for B x H heads in summary tiles. Host-only;
+ * 0 if the arguments are invalid. */
+size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int batch, int heads);
 
 /* Bytes of device workspace pack3d_attn_bwd needs. Host-only. */
 size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch, int heads);
