@@ -1,7 +1,10 @@
 """Benchmark of the PACK3D attention forward on B200 (one process per GPU).
 
 A step is one pass of the operator's hot path over one batch of synthetic input: block
-summaries (pack3d_summarize) followed by the fused forward (pack3d_attn_fwd) -- the index of
+summaries with the rotated keys written in the same pass (pack3d_summarize_rotated), the local
+branch on those keys (pack3d_attn_local with PACK3D_K_ROTATED), then the global branch with the
+mixer (pack3d_attn_global) -- the two halves of pack3d_attn_fwd, called separately so that each
+kernel is timed with CUDA events on the stream it runs on -- the index of
 the packed field is built once per geometry before timing, as it is amortised over layers,
 heads and batches. Default workload: the 65,536-token field (32x32x64 grid, batch 2, 8 heads,
 head_dim 96, bf16, 4x4x4 blocks -> 1,024 summaries, raster-block packing).
@@ -143,16 +146,23 @@ def kernel_traffic(kernel_key):
     return d["bytes_per_launch_full"]
 
 
-def fwd_algorithmic(w):
+def algorithmic(w):
+    """Per-launch algorithmic work of the three kernels of a step (each row read or written
+    once; index tables read once)."""
     B, H, d = w["batch"], w["heads"], w["d"]
     N = int(np.prod(w["grid"]))
     M = int(np.prod([g // b for g, b in zip(w["grid"], w["block"])]))
-    flops_glob = 4.0 * N * M * d * B * H
     el = 2  # bf16
-    bytes_fwd = (4 * B * H * N * d * el + B * H * N * el + 2 * B * H * M * d * el
-                 + N * 4 * (1 + 27))
-    bytes_sum = 2 * B * H * N * d * el + 2 * B * H * M * d * el + N * 4 * 2
-    return flops_glob, bytes_fwd, bytes_sum
+    e = B * H * N * d * el  # bytes of one [B, H, N, d] tensor
+    return {
+        # k, v read; summary tiles and the rotated keys written; members + coords read
+        "summarize": {"bytes": 3 * e + 2 * B * H * M * d * el + N * 4 * 2},
+        # q, rotated k, v read; o_loc written; inverse map read
+        "local": {"bytes": 4 * e + N * 4},
+        # the global contraction: 2 N M d (QK) + 2 N M d (PV) per (batch, head)
+        "global": {"flops": 4.0 * N * M * d * B * H,
+                   "bytes": 3 * e + B * H * N * el + 2 * B * H * M * d * el},
+    }
 
 
 # -------------------------------------------------------------------------------- oracle
@@ -248,6 +258,7 @@ def main():
     q, k, v, a = (w[n].to(dt).to(dev).contiguous() for n in "qkva")
     ksum = torch.empty(p3d.summary_tiles_shape(ix, B, H, d), dtype=dt, device=dev)
     vsum = torch.empty_like(ksum)
+    k_rot = torch.empty_like(k)
     o = torch.empty_like(q)
     excl = w["exclude_near"]
     stream = torch.cuda.current_stream()
@@ -255,14 +266,18 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        p3d.pack3d_summarize(ix, k, v, ksum, vsum)
+        p3d.pack3d_summarize_rotated(ix, k, v, ksum, vsum, k_rot)
         n = p3d.pack3d_last_launch_count()
         if ev is not None:
             ev[1].record(stream)
-        p3d.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=excl, o=o)
+        p3d.pack3d_attn_local(ix, q, k_rot, v, k_rotated=True, o_loc=o)
         n += p3d.pack3d_last_launch_count()
         if ev is not None:
             ev[2].record(stream)
+        p3d.pack3d_attn_global(ix, q, a, ksum, vsum, o, exclude_near=excl, o=o)
+        n += p3d.pack3d_last_launch_count()
+        if ev is not None:
+            ev[3].record(stream)
         return n
 
     for _ in range(max(args.warmup, 0)):
@@ -275,7 +290,7 @@ def main():
     clocks = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     if clocks:
         clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
     t0.record(stream)
@@ -289,12 +304,13 @@ def main():
     clk = clocks.stop() if clocks else None
 
     ms = t0.elapsed_time(t1) / args.steps
-    ms_sum = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    ms_fwd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_k = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+            for i, name in enumerate(("summarize", "local", "global"))}
     if world > 1:
-        tt = torch.tensor([ms, ms_sum, ms_fwd], device=dev)
+        tt = torch.tensor([ms] + [ms_k[n] for n in ("summarize", "local", "global")], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, ms_sum, ms_fwd = (float(x) for x in tt.tolist())
+        vals = [float(x) for x in tt.tolist()]
+        ms, ms_k = vals[0], dict(zip(("summarize", "local", "global"), vals[1:]))
 
     # end to end through the public API with host buffers: H2D of the inputs and D2H of o
     e2e = None
@@ -334,24 +350,39 @@ def main():
 
     if rank == 0:
         peaks = measured_peaks()
-        flops, bytes_fwd, bytes_sum = fwd_algorithmic(w)
-        achieved = flops / (ms_fwd / 1e3) / 1e12
-        roof = {"kernel": "pack3d_attn_fwd", "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16"],
-                "peak_source": f"{peaks['source']} bf16 dense burst",
-                "traffic": kernel_traffic("attn_fwd_" + args.workload),
-                "algorithmic_flops_per_launch": flops, "ms_per_launch": ms_fwd}
-        summ_gbs = bytes_sum / (ms_sum / 1e3) / 1e9
+        alg = algorithmic(w)
+        kernel_names = {"summarize": "k_summarize (pack3d_summarize_rotated)",
+                        "local": "k_local_tma (pack3d_attn_local)",
+                        "global": "k_global_tc (pack3d_attn_global)"}
+        kernels = {}
+        for name in ("summarize", "local", "global"):
+            sec = ms_k[name] / 1e3
+            if "flops" in alg[name]:
+                ach = alg[name]["flops"] / sec / 1e12
+                ent = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16"],
+                       "unit": "TFLOP/s", "frac": ach / peaks["bf16"],
+                       "algorithmic_flops_per_launch": alg[name]["flops"],
+                       "peak_source": f"{peaks['source']} bf16 dense burst"}
+            else:
+                ach = alg[name]["bytes"] / sec / 1e9
+                ent = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                       "frac": ach / peaks["hbm"],
+                       "peak_source": f"{peaks['source']} HBM copy"}
+            ent.update({"kernel": kernel_names[name], "ms_per_launch": ms_k[name],
+                        "algorithmic_bytes_per_launch": alg[name]["bytes"],
+                        "traffic": kernel_traffic(f"{name}_{args.workload}")})
+            kernels[name] = ent
+        dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
+        roof = dict(kernels[dominant])
         line = {
             "metric": METRIC, "value": world * B * N / (ms / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(args.workload, w),
             "roofline": roof,
-            "kernels": {"pack3d_summarize": {"ms": ms_sum, "GB/s": summ_gbs,
-                                             "frac_hbm": summ_gbs / peaks["hbm"],
-                                             "algorithmic_bytes": bytes_sum},
-                        "pack3d_attn_fwd": {"ms": ms_fwd}},
+            "kernels": kernels,
+            # the global contraction's flops over the whole forward (local + global kernels)
+            "fwd_tflops": alg["global"]["flops"] / ((ms_k["local"] + ms_k["global"]) / 1e3) / 1e12,
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,

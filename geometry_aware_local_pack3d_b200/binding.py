@@ -19,6 +19,7 @@ PACK3D_OK = 0
 PACK3D_F32 = 0
 PACK3D_BF16 = 1
 PACK3D_EXCLUDE_NEAR = 1
+PACK3D_K_ROTATED = 2
 
 STATUS_NAMES = {0: "PACK3D_OK", 1: "PACK3D_ERR_INVALID_ARG", 2: "PACK3D_ERR_UNSUPPORTED",
                 3: "PACK3D_ERR_DUP_COORD", 4: "PACK3D_ERR_COORD_RANGE", 5: "PACK3D_ERR_ALIGN",
@@ -72,6 +73,13 @@ def lib():
         L.pack3d_summarize.restype = st
         L.pack3d_summarize.argtypes = [ip, _P, _P, st, st, st, _P, _P, _P]
         L.pack3d_attn_fwd.restype = st
+        L.pack3d_attn_local.restype = st
+        L.pack3d_attn_local.argtypes = [ip, _P, _P, _P, st, st, st, f32, u32, _P, _P, _P]
+        L.pack3d_attn_global.restype = st
+        L.pack3d_attn_global.argtypes = [ip, _P, _P, _P, _P, _P, st, st, st, f32, u32, _P, _P,
+                                         _P, _P]
+        L.pack3d_summarize_rotated.restype = st
+        L.pack3d_summarize_rotated.argtypes = [ip, _P, _P, st, st, st, _P, _P, _P, _P]
         L.pack3d_attn_fwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, st, st, st, f32, u32, _P, _P,
                                       _P, _P, _P, _P]
         L.pack3d_summary_bytes.restype = sz
@@ -212,10 +220,34 @@ def pack3d_summarize(index, k, v, ksum=None, vsum=None, stream=None):
     return ksum, vsum
 
 
+def pack3d_summarize_rotated(index, k, v, ksum=None, vsum=None, k_rot=None, stream=None):
+    """Block summaries plus the rotated keys R(c) k in one pass; returns (ksum, vsum, k_rot)."""
+    _need_cuda(k, v)
+    B, H, N, d = k.shape
+    shape = summary_tiles_shape(index, B, H, d)
+    if ksum is None:
+        ksum = torch.empty(shape, dtype=k.dtype, device=k.device)
+    if vsum is None:
+        vsum = torch.empty(shape, dtype=k.dtype, device=k.device)
+    if k_rot is None:
+        k_rot = torch.empty_like(k)
+    need = pack3d_summary_bytes(index, _dtype_code(k), B, H)
+    for t in (ksum, vsum):
+        if t.numel() * t.element_size() < need:
+            raise ValueError(f"summary buffer holds {t.numel() * t.element_size()} bytes, "
+                             f"needs {need}")
+    _check(lib().pack3d_summarize_rotated(ctypes.byref(index.struct), _ptr(k), _ptr(v),
+                                          _dtype_code(k), B, H, _ptr(ksum), _ptr(vsum),
+                                          _ptr(k_rot), _stream(stream)),
+           "pack3d_summarize_rotated")
+    return ksum, vsum, k_rot
+
+
 def pack3d_attn_fwd(index, q, k, v, gate, ksum, vsum, *, scale=None, exclude_near=False,
-                    o=None, lse_loc=None, lse_glob=None, o_loc=None, o_glob=None,
-                    save_for_backward=False, stream=None):
-    """Returns a dict with o and, when requested, lse_loc, lse_glob, o_loc, o_glob."""
+                    k_rotated=False, o=None, lse_loc=None, lse_glob=None, o_loc=None,
+                    o_glob=None, save_for_backward=False, stream=None):
+    """Returns a dict with o and, when requested, lse_loc, lse_glob, o_loc, o_glob.
+    k_rotated: k is the k_rot of pack3d_summarize_rotated (bf16, tensor-core path)."""
     _need_cuda(q, k, v, gate, ksum, vsum)
     B, H, N, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -227,12 +259,43 @@ def pack3d_attn_fwd(index, q, k, v, gate, ksum, vsum, *, scale=None, exclude_nea
         lse_glob = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse_glob is None else lse_glob
         o_loc = torch.empty_like(q) if o_loc is None else o_loc
         o_glob = torch.empty_like(q) if o_glob is None else o_glob
-    flags = PACK3D_EXCLUDE_NEAR if exclude_near else 0
+    flags = (PACK3D_EXCLUDE_NEAR if exclude_near else 0) | (PACK3D_K_ROTATED if k_rotated else 0)
     _check(lib().pack3d_attn_fwd(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(gate), _ptr(ksum), _ptr(vsum), _dtype_code(q), B, H, scale,
                                  flags, _ptr(o), _ptr(lse_loc), _ptr(lse_glob), _ptr(o_loc),
                                  _ptr(o_glob), _stream(stream)), "pack3d_attn_fwd")
     return dict(o=o, lse_loc=lse_loc, lse_glob=lse_glob, o_loc=o_loc, o_glob=o_glob)
+
+
+def pack3d_attn_local(index, q, k, v, *, scale=None, k_rotated=False, o_loc=None,
+                      lse_loc=None, stream=None):
+    """Local branch alone: returns (o_loc, lse_loc); lse_loc only when a buffer is passed."""
+    _need_cuda(q, k, v)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o_loc is None:
+        o_loc = torch.empty_like(q)
+    flags = PACK3D_K_ROTATED if k_rotated else 0
+    _check(lib().pack3d_attn_local(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
+                                   _dtype_code(q), B, H, scale, flags, _ptr(o_loc),
+                                   _ptr(lse_loc), _stream(stream)), "pack3d_attn_local")
+    return o_loc, lse_loc
+
+
+def pack3d_attn_global(index, q, gate, ksum, vsum, o_loc, *, scale=None, exclude_near=False,
+                       o=None, lse_glob=None, o_glob=None, stream=None):
+    """Global branch + mixer over a given o_loc (o may be o_loc itself): returns o."""
+    _need_cuda(q, gate, ksum, vsum, o_loc)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q)
+    flags = PACK3D_EXCLUDE_NEAR if exclude_near else 0
+    _check(lib().pack3d_attn_global(ctypes.byref(index.struct), _ptr(q), _ptr(gate), _ptr(ksum),
+                                    _ptr(vsum), _ptr(o_loc), _dtype_code(q), B, H, scale, flags,
+                                    _ptr(o), _ptr(lse_glob), _ptr(o_glob), _stream(stream)),
+           "pack3d_attn_global")
+    return o
 
 
 def pack3d_bwd_workspace_bytes(index, dtype_code, batch, heads):

@@ -10,12 +10,7 @@ namespace p3d {
 thread_local int g_launches = 0;
 
 cudaError_t summarize_dispatch(const pack3d_index& ix, const void* k, const void* v, int dtype,
-                               int64_t bh, void* ksum, void* vsum, cudaStream_t s);
-cudaError_t fwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
-                              const void* v, const void* gate, const void* ksum,
-                              const void* vsum, int dtype, int64_t bh, float scale, int excl,
-                              void* o, float* lse_loc, float* lse_glob, void* o_loc,
-                              void* o_glob, cudaStream_t s);
+                               int64_t bh, void* ksum, void* vsum, void* krot, cudaStream_t s);
 cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
                               const void* v, const void* gate, const void* ksum,
                               const void* vsum, const void* o_loc, const void* o_glob,
@@ -23,12 +18,19 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
                               void* dv, void* dgate, void* ws, cudaStream_t s);
 size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh);
+cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const void* gate,
+                                 const void* ksum, const void* vsum, const void* o_loc,
+                                 int dtype, int64_t bh, float scale, int excl, void* o,
+                                 float* lse_glob, void* o_glob, cudaStream_t s);
 cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
                                 const void* v, int dtype, int64_t bh, float scale, void* o_loc,
                                 float* lse_loc, cudaStream_t s);
 cudaError_t local_tc_dispatch(const pack3d_index& ix, const void* q, const void* k,
                               const void* v, int64_t bh, float scale, void* o_loc,
                               float* lse_loc, cudaStream_t s);
+cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void* k_rot,
+                               const void* v, int64_t bh, float scale, void* o_loc,
+                               float* lse_loc, cudaStream_t s);
 cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
                                float scale, int excl, void* o, float* lse_glob, void* o_glob,
@@ -97,8 +99,52 @@ extern "C" pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k
   if (st != PACK3D_OK) return st;
   if ((st = check_rows({k, v, ksum, vsum})) != PACK3D_OK) return st;
   return cuda_status(summarize_dispatch(*idx, k, v, dtype, (int64_t)batch * heads, ksum, vsum,
-                                        static_cast<cudaStream_t>(stream)));
+                                        nullptr, static_cast<cudaStream_t>(stream)));
 }
+
+extern "C" pack3d_status pack3d_summarize_rotated(const pack3d_index* idx, const void* k,
+                                                  const void* v, int dtype, int batch, int heads,
+                                                  void* ksum, void* vsum, void* k_rot,
+                                                  void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({k, v, ksum, vsum, k_rot})) != PACK3D_OK) return st;
+  if (k_rot == k) return PACK3D_ERR_INVALID_ARG;  // other members of a block still read k
+  return cuda_status(summarize_dispatch(*idx, k, v, dtype, (int64_t)batch * heads, ksum, vsum,
+                                        k_rot, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+// local branch: o_loc (normalised) and lse_loc
+pack3d_status run_local(const pack3d_index* idx, const void* q, const void* k, const void* v,
+                        int dtype, int64_t bh, float scale, bool k_rotated, void* o_loc,
+                        float* lse_loc, cudaStream_t s) {
+  if (dtype == PACK3D_BF16 && bf16_tensor_path())
+    return cuda_status(k_rotated ? local_tma_dispatch(*idx, q, k, v, bh, scale, o_loc, lse_loc, s)
+                                 : local_tc_dispatch(*idx, q, k, v, bh, scale, o_loc, lse_loc, s));
+  return cuda_status(local_simt_dispatch(*idx, q, k, v, dtype, bh, scale, o_loc, lse_loc, s));
+}
+
+// global branch over the summaries + the sigmoid mixer with a given o_loc (o may alias it)
+pack3d_status run_global(const pack3d_index* idx, const void* q, const void* gate,
+                         const void* ksum, const void* vsum, const void* o_loc, int dtype,
+                         int64_t bh, float scale, int excl, void* o, float* lse_glob,
+                         void* o_glob, cudaStream_t s) {
+  if (dtype == PACK3D_BF16 && bf16_tensor_path())
+    return cuda_status(global_tc_dispatch(*idx, q, gate, ksum, vsum, o_loc, bh, scale, excl, o,
+                                          lse_glob, o_glob, s));
+  return cuda_status(global_simt_dispatch(*idx, q, gate, ksum, vsum, o_loc, dtype, bh, scale,
+                                          excl, o, lse_glob, o_glob, s));
+}
+
+pack3d_status check_flags(int dtype, uint32_t flags, uint32_t allowed) {
+  if (flags & ~allowed) return PACK3D_ERR_INVALID_ARG;
+  if ((flags & PACK3D_K_ROTATED) && !(dtype == PACK3D_BF16 && bf16_tensor_path()))
+    return PACK3D_ERR_UNSUPPORTED;
+  return PACK3D_OK;
+}
+}  // namespace
 
 extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void* k,
                                          const void* v, const void* gate, const void* ksum,
@@ -112,22 +158,52 @@ extern "C" pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q,
   if ((st = check_rows({q, k, v, ksum, vsum, o})) != PACK3D_OK) return st;
   if (!gate) return PACK3D_ERR_INVALID_ARG;
   if ((o_loc && !aligned16(o_loc)) || (o_glob && !aligned16(o_glob))) return PACK3D_ERR_ALIGN;
-  if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
-  const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
+  if (!(scale > 0.f)) return PACK3D_ERR_INVALID_ARG;
+  if ((st = check_flags(dtype, flags, PACK3D_EXCLUDE_NEAR | PACK3D_K_ROTATED)) != PACK3D_OK)
+    return st;
   const int64_t bh = (int64_t)batch * heads;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == PACK3D_BF16 && bf16_tensor_path()) {
-    // local branch first (its normalised output goes to o_loc, or to o until it is mixed),
-    // then the tensor-core global branch with the mixer in its epilogue
-    void* ol = o_loc ? o_loc : o;
-    cudaError_t e = local_tc_dispatch(*idx, q, k, v, bh, scale, ol, lse_loc, s);
-    if (e != cudaSuccess) return PACK3D_ERR_CUDA;
-    return cuda_status(global_tc_dispatch(*idx, q, gate, ksum, vsum, ol, bh, scale, excl, o,
-                                          lse_glob, o_glob, s));
-  }
-  return cuda_status(fwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, dtype, bh, scale, excl,
-                                       o, lse_loc, lse_glob, o_loc, o_glob,
-                                       static_cast<cudaStream_t>(stream)));
+  // local branch first (its normalised output goes to o_loc, or to o until it is mixed), then
+  // the global branch with the mixer in its epilogue
+  void* ol = o_loc ? o_loc : o;
+  st = run_local(idx, q, k, v, dtype, bh, scale, (flags & PACK3D_K_ROTATED) != 0, ol, lse_loc, s);
+  if (st != PACK3D_OK) return st;
+  return run_global(idx, q, gate, ksum, vsum, ol, dtype, bh, scale,
+                    (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0, o, lse_glob, o_glob, s);
+}
+
+extern "C" pack3d_status pack3d_attn_local(const pack3d_index* idx, const void* q, const void* k,
+                                           const void* v, int dtype, int batch, int heads,
+                                           float scale, uint32_t flags, void* o_loc,
+                                           float* lse_loc, void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({q, k, v, o_loc})) != PACK3D_OK) return st;
+  if (!(scale > 0.f)) return PACK3D_ERR_INVALID_ARG;
+  if ((st = check_flags(dtype, flags, PACK3D_K_ROTATED)) != PACK3D_OK) return st;
+  return run_local(idx, q, k, v, dtype, (int64_t)batch * heads, scale,
+                   (flags & PACK3D_K_ROTATED) != 0, o_loc, lse_loc,
+                   static_cast<cudaStream_t>(stream));
+}
+
+extern "C" pack3d_status pack3d_attn_global(const pack3d_index* idx, const void* q,
+                                            const void* gate, const void* ksum,
+                                            const void* vsum, const void* o_loc, int dtype,
+                                            int batch, int heads, float scale, uint32_t flags,
+                                            void* o, float* lse_glob, void* o_glob,
+                                            void* stream) {
+  reset_launches();
+  pack3d_status st = check_common(idx, dtype, batch, heads);
+  if (st != PACK3D_OK) return st;
+  if ((st = check_rows({q, ksum, vsum, o_loc, o})) != PACK3D_OK) return st;
+  if (!gate) return PACK3D_ERR_INVALID_ARG;
+  if (o_glob && !aligned16(o_glob)) return PACK3D_ERR_ALIGN;
+  if (!(scale > 0.f)) return PACK3D_ERR_INVALID_ARG;
+  if ((st = check_flags(dtype, flags, PACK3D_EXCLUDE_NEAR)) != PACK3D_OK) return st;
+  return run_global(idx, q, gate, ksum, vsum, o_loc, dtype, (int64_t)batch * heads, scale,
+                    (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0, o, lse_glob, o_glob,
+                    static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int batch,

@@ -482,23 +482,6 @@ static BwdWork carve(const pack3d_index& ix, int64_t bh, void* ws) {
 }
 
 template <typename T, int D>
-cudaError_t fwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
-                     const void* gate, const void* ksum, const void* vsum, int64_t bh,
-                     float scale, int excl, void* o, float* lse_loc, float* lse_glob,
-                     void* o_loc, void* o_glob, cudaStream_t s) {
-  const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
-  T* ol = static_cast<T*>(o_loc ? o_loc : o);  // the local output may live in `o` until mixed
-  k_local_fwd<T, D><<<grid, 128, 0, s>>>(ix, static_cast<const T*>(q), static_cast<const T*>(k),
-                                          static_cast<const T*>(v), scale, ol, lse_loc);
-  k_global_fwd<T, D, 32><<<grid, 128, 0, s>>>(
-      ix, static_cast<const T*>(q), static_cast<const T*>(ksum), static_cast<const T*>(vsum),
-      static_cast<const T*>(gate), ol, scale, excl, static_cast<T*>(o), lse_glob,
-      static_cast<T*>(o_glob));
-  count_launch(2);
-  return cudaGetLastError();
-}
-
-template <typename T, int D>
 cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
                      const void* gate, const void* ksum, const void* vsum, const void* o_loc,
                      const void* o_glob, const float* lse_loc, const float* lse_glob,
@@ -528,17 +511,26 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
   return cudaGetLastError();
 }
 
-cudaError_t fwd_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
-                              const void* v, const void* gate, const void* ksum,
-                              const void* vsum, int dtype, int64_t bh, float scale, int excl,
-                              void* o, float* lse_loc, float* lse_glob, void* o_loc,
-                              void* o_glob, cudaStream_t s) {
+// Global branch + mixer only, over a given local output (which `o` may alias).
+cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const void* gate,
+                                 const void* ksum, const void* vsum, const void* o_loc,
+                                 int dtype, int64_t bh, float scale, int excl, void* o,
+                                 float* lse_glob, void* o_glob, cudaStream_t s) {
+  const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
   const int d = ix.geom.head_dim;
-#define P3D_FWD(T, D) \
-  fwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, bh, scale, excl, o, lse_loc, lse_glob, o_loc, o_glob, s)
-  if (dtype == PACK3D_BF16) return d == 96 ? P3D_FWD(__nv_bfloat16, 96) : P3D_FWD(__nv_bfloat16, 48);
-  return d == 96 ? P3D_FWD(float, 96) : P3D_FWD(float, 48);
-#undef P3D_FWD
+#define P3D_GLB(T, D)                                                                          \
+  k_global_fwd<T, D, 32><<<grid, 128, 0, s>>>(                                                 \
+      ix, static_cast<const T*>(q), static_cast<const T*>(ksum), static_cast<const T*>(vsum), \
+      static_cast<const T*>(gate), static_cast<const T*>(o_loc), scale, excl, static_cast<T*>(o), \
+      lse_glob, static_cast<T*>(o_glob))
+  if (dtype == PACK3D_BF16) {
+    if (d == 96) P3D_GLB(__nv_bfloat16, 96); else P3D_GLB(__nv_bfloat16, 48);
+  } else {
+    if (d == 96) P3D_GLB(float, 96); else P3D_GLB(float, 48);
+  }
+#undef P3D_GLB
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,

@@ -1,0 +1,692 @@
+// Local branch of PACK3D attention, row-gather form (bf16 I/O, head_dim 48 or 96), for keys
+// that were rotated once up front (pack3d_summarize_rotated).
+//
+// Project page "Geometry Matters in Packed 3D Attention", Chapter 3 Contract 1: each query
+// attends exactly to every token of its 3x3x3 coordinate neighbourhood, found by coordinate,
+// never by adjacency in memory; paper summary §3.5: streamed online softmax, no gathered
+// neighbour tensor in memory.
+//
+// Work unit: one 8x4x4 (z, y, x) brick of 128 queries of one (batch, head); persistent CTAs
+// walk bricks with a grid stride, two CTAs per SM. Per brick:
+//   * one 3D TMA box load brings the memory slots of the brick's 10x6x6 halo from the inverse
+//     map (x start rounded down to a 16-byte boundary: box 12x6x10 int32);
+//   * TMA row gathers (tile::gather4, 4 rows of 64 columns each, 128-byte swizzle) bring the
+//     128 q rows (rows outside the grid are requested past the end of the tensor and arrive as
+//     zeros), and two warps rotate the q tile in shared memory (axial RoPE by the brick
+//     coordinates);
+//   * the same two warps fetch, per halo z-slice, the 36 rotated key rows and value rows
+//     (padded to 48 with zero rows) with one cp.async per 16-byte piece, straight into the
+//     128-byte-swizzle layout (measured on B200: scattered 192-byte rows arrive about 1.7x
+//     faster this way than through gather4, whose per-operation cost caps it);
+// Chunk s = halo z-slice s (s = 0..9). Row r = 32 w + 16 dz + 4 y + x holds brick position
+// (2w + dz, y, x), so warp w needs exactly slices 2w .. 2w+3 and chunk s is owned by warps
+// max(0, (s-2)/2) .. min(3, s/2). Per chunk:
+//   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2 at column 0 or 64)
+//   owners: 3x3x3 mask, online softmax, P = exp2(s - m) as bf16 over the buffer's first 24
+//   columns;  O += P_s v_s  (TS MMA, N = d, TMEM columns 128..) with the rows of the other
+//   warps disabled through the MMA's output-lane mask, so non-owners never touch chunk s.
+// QK runs two chunks ahead of PV, so S_{s+2} is ready when the owners finish chunk s + 1. Each
+// warp zeroes its O rows when it starts a brick; its epilogue runs after the PV of its last
+// chunk. Every query sits at the same row and every neighbour at the same column whatever the
+// packing, so a coordinate-carrying repack permutes the output bit for bit.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace p3d {
+
+namespace lg {
+constexpr int BZ = 8, BY = 4, BX = 4;  // brick
+constexpr int HY = BY + 2, HX = BX + 2;
+constexpr int kChunks = BZ + 2;        // halo z-slices
+constexpr int kSliceKeys = HY * HX;    // 36
+constexpr int kNK = 48;                // chunk rows (MMA N of QK, K of PV)
+constexpr int kStages = 3;
+constexpr int kThreads = 256;          // softmax 0-3, TMA 4, k/v fetch + q rotation 5-6, MMA 7
+constexpr int kRot = 64;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kOCol = 128;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kBoxX = 12, kBoxY = 6, kBoxZ = 10;  // slot box: x from x0 - 4
+constexpr int kBoxBytes = kBoxX * kBoxY * kBoxZ * 4;
+constexpr int kBoxPitch = 3072;
+
+__device__ __forceinline__ uint32_t s_col(int b) { return b ? 64u : 0u; }
+
+template <int D> struct Smem {
+  static constexpr int CBN = (D + 63) / 64;  // 64-column blocks of a row (2 for 96, 1 for 48)
+  static constexpr int kQBlk = 128 * 128;    // one column block of the q tile
+  static constexpr int kCBlk = kNK * 128;    // one column block of a k or v chunk
+  static constexpr int kStage = CBN * kCBlk;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + CBN * kQBlk;
+  static constexpr int kV = kK + kStages * kStage;
+  static constexpr int kBox = kV + kStages * kStage;  // [2] slot boxes
+  static constexpr int kRope = kBox + 2 * kBoxPitch;  // [16][d/6] (cos, sin) of the q tile
+  static constexpr int kBar = kRope + 16 * (D / 6) * 8;
+  static constexpr int kBytes = kBar + 512;
+};
+
+enum {
+  B_QLOAD = 0, B_QFULL = 1, B_QEMPTY = 2, B_KVFULL = 3, B_KVEMPTY = 6, B_BOX = 9, B_BOXFREE = 11,
+  B_SFULL = 13,  // [warp][buffer]
+  B_PFULL = 21,  // [warp][buffer]
+  B_PVALL = 29, B_EPI = 30,  // B_EPI: [warp]
+  B_DRAIN = 34, B_COUNT = 35
+};
+static_assert(8 * B_COUNT + 16 <= 512, "barrier area");
+
+struct Params {
+  pack3d_index ix;
+  const __nv_bfloat16* k_rot;  // rotated keys [B, H, N, d]
+  const __nv_bfloat16* v;
+  __nv_bfloat16* o_loc;
+  float* lse_loc;  // optional
+  float scale_log2;
+  int nbz, nby, nbx;
+  int box_tma;        // slot boxes by TMA (else plain loads)
+  int64_t tiles;      // batch * heads * bricks
+  int64_t rows;       // batch * heads * N: first row index past the gathered tensors
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
+struct Abort {
+  volatile int* flag;
+  int32_t* status;
+  // probing wait; with `nap` a short sleep between probes leaves issue slots to working warps
+  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
+    if (tc::mbar_test_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!tc::mbar_test_wait(bar, parity)) {
+      if (nap) __nanosleep(32);
+      if (*flag) return false;
+      if (clock64() - t0 > 4000000000LL) {
+        *flag = 1;
+        set_status(status, PACK3D_ERR_TIMEOUT);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+// clock64 trace slots of the first four bricks a CTA processes (tracing builds only)
+#define GTR(ti, off)                                       \
+  do {                                                     \
+    if ((ti) < 4) P3D_TRACE_C((ti) * 400 + (off));         \
+  } while (0)
+
+// first and last softmax warp owning halo slice s
+__device__ __forceinline__ int owner_lo(int s) { return max(0, (s - 2) >> 1); }
+__device__ __forceinline__ int owner_hi(int s) { return min(3, s >> 1); }
+
+}  // namespace lg
+
+template <int D>
+__global__ void __launch_bounds__(lg::kThreads, 2)
+    k_local_tma(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mg,
+                const lg::Params P) {
+  using namespace lg;
+  using S = Smem<D>;
+  constexpr int CBN = S::CBN;
+  constexpr int KC = D / 8;  // 16-byte pieces of a q row
+  constexpr int DA = D / 3;
+  constexpr int PR = D / 6;  // rotation pairs per axis
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  Abort ab{abort_flag, P.ix.status};
+  const pack3d_geom& g = P.ix.geom;
+  const int64_t N = P.ix.n;
+  const int64_t bricks = (int64_t)P.nbz * P.nby * P.nbx;
+  auto origin = [&](int64_t t, int64_t& bh, int& z0, int& y0, int& x0) {
+    bh = t / bricks;
+    const int64_t br = t % bricks;
+    z0 = (int)(br / (P.nby * P.nbx)) * BZ;
+    y0 = (int)((br / P.nbx) % P.nby) * BY;
+    x0 = (int)(br % P.nbx) * BX;
+  };
+  auto in_grid = [&](int z, int y, int x) {
+    return z >= 0 && z < g.gz && y >= 0 && y < g.gy && x >= 0 && x < g.gx;
+  };
+
+  if (tid == 0) {
+    tc::mbar_init(&bars[B_QLOAD], 1);
+    tc::mbar_init(&bars[B_QFULL], kRot);
+    tc::mbar_init(&bars[B_QEMPTY], 1);
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&bars[B_KVFULL + i], kRot);
+      tc::mbar_init(&bars[B_KVEMPTY + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars[B_BOX + i], 1);
+      tc::mbar_init(&bars[B_BOXFREE + i], 4 + 2);  // softmax warps + producer warps
+    }
+    for (int i = 0; i < 8; ++i) {
+      tc::mbar_init(&bars[B_SFULL + i], 1);
+      tc::mbar_init(&bars[B_PFULL + i], 32);
+    }
+    tc::mbar_init(&bars[B_PVALL], 1);
+    for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[B_EPI + i], 1);
+    tc::mbar_init(&bars[B_DRAIN], 1);
+    abort_flag[0] = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tc::tma_prefetch_desc(&mq);
+    if (P.box_tma) tc::tma_prefetch_desc(&mg);
+  }
+  // the padding rows 36..47 of every k/v stage are never written by the producers: zero them
+  // once (the MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
+  for (int i = tid; i < kStages * 2 * CBN * (kNK - kSliceKeys) * 8; i += kThreads) {
+    const int piece = i & 7, row = kSliceKeys + (i >> 3) % (kNK - kSliceKeys);
+    const int blk = (i >> 3) / (kNK - kSliceKeys);  // stage * 2 * CBN + tensor * CBN + cb
+    const int st = blk / (2 * CBN), ten = (blk / CBN) & 1, cb = blk % CBN;
+    *reinterpret_cast<uint4*>(smem + (ten ? S::kV : S::kK) + st * S::kStage + cb * S::kCBlk +
+                              (row >> 3) * 1024 + (row & 7) * 128 + piece * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+  tc::fence_proxy_async_smem();
+  if (warp == 7) tc::tmem_alloc(tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp < 4) {
+    // --------------------------------------------------------- softmax + epilogue (row = tid)
+    const int w = warp;
+    int ti = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
+      // lane-derived values from opaque copies each brick (keeps the score row in registers)
+      int ln = lane;
+      uint32_t tl = tbase;
+      asm volatile("" : "+r"(ln), "+r"(tl));
+      tl += (uint32_t)(w * 32) << 16;
+      const int dz = ln >> 4, qy = (ln >> 2) & 3, qx = ln & 3;
+      int64_t bh;
+      int z0, y0, x0;
+      origin(t, bh, z0, y0, x0);
+      const int bb = ti & 1;
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + bb], (ti >> 1) & 1))) break;
+      const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
+      const int cz = z0 + 2 * w + dz, cy = y0 + qy, cx = x0 + qx;
+      const bool valid = cz < g.gz && cy < g.gy && cx < g.gx;
+      // neighbour bits of the warp's four slices: bit hy * 6 + hx of slice 2w + i
+      uint64_t nb[4] = {0ull, 0ull, 0ull, 0ull};
+      if (valid) {
+#pragma unroll
+        for (int o = 0; o < 27; ++o) {
+          const int ddz = o / 9 - 1, ddy = (o / 3) % 3 - 1, ddx = o % 3 - 1;
+          const int hy = qy + 1 + ddy, hx = qx + 1 + ddx;
+          const int hz = 2 * w + dz + 1 + ddz;  // halo slice
+          if (!in_grid(cz + ddz, cy + ddy, cx + ddx)) continue;
+          if (box[(hz * kBoxY + hy) * kBoxX + hx + 3] < 0) continue;
+          const uint64_t bit = 1ull << (hy * HX + hx);
+          nb[1 + ddz] |= dz == 0 ? bit : 0ull;  // slice index i = dz + 1 + ddz
+          nb[2 + ddz] |= dz == 1 ? bit : 0ull;
+        }
+      }
+      // this warp's O rows start at zero (the previous brick's epilogue has read them)
+      {
+        const uint32_t zr[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 16) tc::tmem_st16(tl + kOCol + c0, zr);
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s = 2 * w + i, b = i & 1;
+        const uint32_t gs = (uint32_t)ti * kChunks + s;
+        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + 2 * w + b], (i >> 1) & 1))) {
+          ok = false;
+          break;
+        }
+        if (ln == 0) GTR(ti, 110 + w * 20 + i * 4);
+        tc::tc_fence_after();
+        // the chunk's 48 scores; entries off the 3x3x3 cube become -inf
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t r[kNK];
+#pragma unroll
+        for (int c0 = 0; c0 < kNK; c0 += 16)
+          tc::tmem_ld16(tl + s_col(b) + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[c0]));
+        tc::tmem_wait_ld();
+        const uint64_t win = nb[i];
+#pragma unroll
+        for (int k = 0; k < kNK; ++k) {
+          if (!((win >> k) & 1ull)) r[k] = 0xff800000u;
+          mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
+        }
+        const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
+        const float m_new = fmaxf(m_run, cmax);
+        const bool need = m_new > m_run + kRescaleLog2;
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          // O rows hold earlier chunks at the old max: rescale once the previous PV is done
+          // (PVALL phase gs - 1 is the only incomplete or just-completed phase here)
+          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVALL], (gs - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const float f = need ? ex2(m_run - m_new) : 1.f;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tc::tmem_ld16(tl + kOCol + c0, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+            tc::tmem_st16(tl + kOCol + c0, o);
+          }
+        }
+        if (need) {
+          l_run *= ex2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t p[kNK / 2];
+#pragma unroll
+        for (int k = 0; k < kNK; k += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(r[k]), P.scale_log2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(r[k + 1]), P.scale_log2, neg_m));
+          ls[(k >> 1) & 3] += p0 + p1;
+          p[k >> 1] = tc::pack_bf16(p0, p1);
+        }
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tc::tmem_st16(tl + s_col(b), *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
+        lg::tmem_st8(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[8]>(&p[16]));
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bars[B_PFULL + 2 * w + b]);
+        if (ln == 0) GTR(ti, 111 + w * 20 + i * 4);
+      }
+      if (!ok) break;
+      // epilogue after the PV of the warp's last slice: o_loc = O / l, lse_loc
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_EPI + w], ti & 1))) break;
+      tc::tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint32_t ow[D / 2];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        uint32_t o[16];
+        tc::tmem_ld16(tl + kOCol + c0, o);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ow[c0 / 2 + k] =
+              tc::pack_bf16(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+      }
+      const int slot =
+          valid ? box[((2 * w + dz + 1) * kBoxY + qy + 1) * kBoxX + qx + 4] : -1;
+      __syncwarp();
+      if (ln == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
+      if (ln == 0) GTR(ti, 190 + w);
+      if (slot >= 0) {
+        uint4* dst = reinterpret_cast<uint4*>(P.o_loc + (bh * N + slot) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+          dst[c] = make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
+        if (P.lse_loc)
+          P.lse_loc[bh * N + slot] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      }
+    }
+  } else if (warp == 4) {
+    // --------------------------------------------------------- TMA: slot boxes and q rows
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, ab.wait(bar, parity));
+    };
+    int ti = 0;
+    uint32_t q_loads = 0, box_loads[2] = {0u, 0u};  // copies issued, for the exit
+    for (int64_t t = blockIdx.x; t < P.tiles; t += gridDim.x, ++ti) {
+      int64_t bh;
+      int z0, y0, x0;
+      origin(t, bh, z0, y0, x0);
+      const int bb = ti & 1;
+      int32_t* box = reinterpret_cast<int32_t*>(smem + S::kBox + bb * kBoxPitch);
+      if (lane == 0) GTR(ti, 0);
+      if (ti >= 2 && !wwait(&bars[B_BOXFREE + bb], ((ti >> 1) - 1) & 1)) break;
+      if (lane == 0) GTR(ti, 1);
+      ++box_loads[bb];
+      if (P.box_tma) {
+        if (lane == 0) {
+          tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
+          tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
+        }
+      } else {
+        for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
+          const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
+          const int z = z0 - 1 + bz, y = y0 - 1 + by, x = x0 - 4 + bx;
+          box[i] = in_grid(z, y, x) ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : 0;
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars[B_BOX + bb]);
+      }
+      if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
+      if (lane == 0) GTR(ti, 2);
+      // q rows: lane l gathers rows 4l .. 4l+3 of the tile (rows off the grid: past the end)
+      if (ti >= 1 && !wwait(&bars[B_QEMPTY], (ti - 1) & 1)) break;
+      int qr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = 4 * lane + j, rw = r >> 5, rl = r & 31;
+        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = rl & 3;
+        const int slot = in_grid(z0 + z, y0 + y, x0 + x)
+                             ? box[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
+                             : -1;
+        qr[j] = slot >= 0 ? (int)(bh * N + slot) : (int)P.rows;
+      }
+      if (lane == 0) tc::mbar_expect_tx(&bars[B_QLOAD], 128 * 128 * CBN);
+      ++q_loads;
+      __syncwarp();
+#pragma unroll
+      for (int cb = 0; cb < CBN; ++cb)
+        tc::tma_gather4(smem + S::kQ + cb * S::kQBlk + lane * 512, &mq, cb * 64, qr[0], qr[1],
+                        qr[2], qr[3], &bars[B_QLOAD]);
+      if (lane == 0) GTR(ti, 3);
+    }
+    // nothing may still be landing in shared memory when the CTA exits (bounded waits)
+    if (lane == 0) {
+      if (q_loads) tc::mbar_wait(&bars[B_QLOAD], (q_loads - 1) & 1, 100000000LL);
+      for (int b2 = 0; b2 < 2; ++b2)
+        if (box_loads[b2])
+          tc::mbar_wait(&bars[B_BOX + b2], (box_loads[b2] - 1) & 1, 100000000LL);
+    }
+  } else if (warp < 7) {
+    // --------------------------------------------------------- k/v rows and q rotation (64 thr)
+    // Halo slice s of rotated keys and values: 36 rows x d, one cp.async per 16-byte piece
+    // (rows off the grid are zero-filled), written at its 128-byte-swizzle position; each
+    // thread publishes a slice once its own copies have landed. Between slices 1 and 2 the same
+    // threads rotate the brick's q tile, which the TMA warp has gathered meanwhile.
+    const int pt = tid - 160;
+    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope);  // [16][PR]
+    volatile int* pflag = abort_flag + 1;                          // [2], used alternately
+    int nwait = 0;
+    // one bounded wait by one thread, its verdict shared with all 64 (named barrier 2)
+    auto pwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      volatile int* f = pflag + (nwait++ & 1);
+      if (pt == 0) *f = ab.wait(bar, parity) ? 1 : 0;
+      asm volatile("bar.sync 2, 64;" ::: "memory");
+      return *f != 0;
+    };
+    // this thread's pieces, the same in every slice: (row, 16-byte column) and the swizzled
+    // shared-memory offset, packed as off16 | row << 16 | col << 24
+    constexpr int KPIECES = kSliceKeys * KC;
+    constexpr int NP = (KPIECES + kRot - 1) / kRot;
+    uint32_t pc[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      const int p = pt + j * kRot;
+      const int row = p / KC, c = p % KC;
+      const int off = (c >> 3) * S::kCBlk + (row >> 3) * 1024 + (row & 7) * 128 +
+                      (((c & 7) ^ (row & 7)) << 4);
+      pc[j] = p < KPIECES ? ((uint32_t)(off >> 4) | ((uint32_t)row << 16) | ((uint32_t)c << 24))
+                          : 0xffffffffu;
+    }
+    const __nv_bfloat16* kg = P.k_rot;
+    const __nv_bfloat16* vg = P.v;
+    int ti = 0;
+    uint32_t gs = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
+      int64_t bh;
+      int z0, y0, x0;
+      origin(t, bh, z0, y0, x0);
+      const int bb = ti & 1;
+      const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
+      if (!pwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
+      const int64_t rbase = bh * N;
+      for (int s = 0; s < kChunks; ++s, ++gs) {
+        const int st = gs % kStages;
+        if (gs >= (uint32_t)kStages && !pwait(&bars[B_KVEMPTY + st], ((gs / kStages) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if (pt == 0) GTR(ti, 10 + s * 2);
+        uint8_t* kd = smem + S::kK + st * S::kStage;
+        uint8_t* vd = smem + S::kV + st * S::kStage;
+        const bool zin = z0 - 1 + s >= 0 && z0 - 1 + s < g.gz;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+          if (pc[j] == 0xffffffffu) continue;
+          const int row = (pc[j] >> 16) & 0xff, c = pc[j] >> 24;
+          const int hy = row / HX, hx = row % HX;
+          const int y = y0 - 1 + hy, x = x0 - 1 + hx;
+          int slot = -1;
+          if (zin && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
+            slot = box[(s * kBoxY + hy) * kBoxX + hx + 3];
+          const int64_t src = (rbase + (slot >= 0 ? slot : 0)) * D + c * 8;
+          const uint32_t off = (pc[j] & 0xffffu) << 4;
+          tc::cp_async16(kd + off, kg + src, slot >= 0);
+          tc::cp_async16(vd + off, vg + src, slot >= 0);
+        }
+        tc::cp_async_commit();
+        if (pt == 0) GTR(ti, 11 + s * 2);
+        if (s > 0) {
+          // the previous slice has landed: publish it to the MMA warp
+          tc::cp_async_wait_group<1>();
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars[B_KVFULL + (gs - 1) % kStages]);
+        }
+        if (s == 1) {
+          // q tile of this brick: rotation rows z0..z0+7, y0..y0+3, x0..x0+3 (rows off the
+          // grid are zero and any finite rotation keeps them zero)
+          for (int i = pt; i < 16 * PR; i += kRot) {
+            const int idx = i / PR, pp = i % PR;
+            int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : x0 + idx - 12);
+            cv = min(cv, P.ix.rope_rows - 1);
+            rope_q[i] = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp);
+          }
+          if (!pwait(&bars[B_QLOAD], ti & 1)) { ok = false; break; }
+          if (pt == 0) GTR(ti, 40);
+#pragma unroll 4
+          for (int i = pt; i < 128 * KC; i += kRot) {
+            const int c = i >> 7, r = i & 127;
+            const int cb = c >> 3, cc = c & 7;
+            uint4* ptr = reinterpret_cast<uint4*>(smem + S::kQ + cb * S::kQBlk + (r >> 3) * 1024 +
+                                                  (r & 7) * 128 + ((cc ^ (r & 7)) << 4));
+            const int rw = r >> 5, rl = r & 31;
+            const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
+            const int idx =
+                axis == 0 ? 2 * rw + (rl >> 4) : (axis == 1 ? 8 + ((rl >> 2) & 3) : 12 + (rl & 3));
+            const float4* cs4 = reinterpret_cast<const float4*>(rope_q + idx * PR + p0);
+            const float4 ca = cs4[0], cbv = cs4[1];
+            const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
+            const uint4 x = *ptr;
+            const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
+            uint32_t xo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float e0 = __uint_as_float(xin[k] << 16);
+              const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+              xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
+                                    e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
+            }
+            *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars[B_QFULL]);
+          if (pt == 0) GTR(ti, 41);
+        }
+      }
+      if (!ok) break;
+      // the brick's last slice, and this warp's reads of the slot box, are done
+      tc::cp_async_wait_group<0>();
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[B_KVFULL + (gs - 1) % kStages]);
+      __syncwarp();
+      if ((pt & 31) == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
+      asm volatile("bar.sync 2, 64;" ::: "memory");  // rope_q is rewritten for the next brick
+    }
+    tc::cp_async_wait_all();  // nothing may still be landing in shared memory at exit
+  } else {
+    // --------------------------------------------------------- MMA issuer (warp 7)
+    // Per slice s: PV(s) for its owners (other rows disabled), then -- once PV(s) has
+    // completed, which frees S buffer s % 2 -- QK(s + 2). The whole warp runs the schedule with
+    // warp-uniform values; one elected lane issues the MMAs and commits.
+    const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
+    const uint32_t id_qk = tc::idesc_bf16_f32(128, kNK, false, false);
+    const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
+    const uint64_t qd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kQ), 16, 1024);
+    const uint64_t kd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kK), 16, 1024);
+    const uint64_t vd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kV), S::kCBlk, 1024);
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, ab.wait(bar, parity, false));
+    };
+    int ti = 0;
+    uint32_t gs = 0;
+    bool ok = true;
+    // QK(s) of chunk counter gc into S buffer s % 2; the buffer was freed by the PVALL wait
+    // of chunk gc - 2
+    auto issue_qk = [&](int s, uint32_t gc) -> bool {
+      const int st = gc % kStages;
+      if (!wwait(&bars[B_KVFULL + st], (gc / kStages) & 1)) return false;
+      tc::tc_fence_after();
+      const uint64_t b0 = kd0 + (uint64_t)((st * S::kStage) >> 4);
+      const uint32_t dt = tb + s_col(s & 1);
+      if (tc::elect_one()) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;  // 16 columns = 32 bytes into the swizzled row
+          tc::mma_ss(dt, qd0 + (uint64_t)(((ks >> 2) * S::kQBlk + off) >> 4),
+                     b0 + (uint64_t)(((ks >> 2) * S::kCBlk + off) >> 4), id_qk, ks > 0);
+        }
+        for (int w = owner_lo(s); w <= owner_hi(s); ++w)
+          tc::tc_commit(&bars[B_SFULL + 2 * w + (s & 1)]);
+        if (s == kChunks - 1) tc::tc_commit(&bars[B_QEMPTY]);  // q tile free for the next brick
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
+      if (!wwait(&bars[B_QFULL], ti & 1)) break;
+      if (lane == 0) GTR(ti, 50);
+      tc::tc_fence_after();
+      ok = issue_qk(0, gs) && issue_qk(1, gs + 1);
+      if (lane == 0) GTR(ti, 51);
+      for (int s = 0; s < kChunks && ok; ++s, ++gs) {
+        const int st = gs % kStages, b = s & 1;
+        const int wlo = owner_lo(s), whi = owner_hi(s);
+        for (int w = wlo; w <= whi && ok; ++w)
+          ok = wwait(&bars[B_PFULL + 2 * w + b], ((s - 2 * w) >> 1) & 1);
+        if (!ok) break;
+        if (lane == 0) GTR(ti, 60 + s * 4);
+        tc::tc_fence_after();
+        const uint32_t m0 = (0 < wlo || 0 > whi) ? 0xffffffffu : 0u;
+        const uint32_t m1 = (1 < wlo || 1 > whi) ? 0xffffffffu : 0u;
+        const uint32_t m2 = (2 < wlo || 2 > whi) ? 0xffffffffu : 0u;
+        const uint32_t m3 = (3 < wlo || 3 > whi) ? 0xffffffffu : 0u;
+        const uint64_t v0 = vd0 + (uint64_t)((st * S::kStage) >> 4);
+        if (tc::elect_one()) {
+#pragma unroll
+          for (int ks = 0; ks < kNK / 16; ++ks)
+            tc::mma_ts_masked(tb + kOCol, tb + s_col(b) + ks * 8, v0 + (uint64_t)(ks * (2048 >> 4)),
+                              id_pv, 1u, m0, m1, m2, m3);
+          tc::tc_commit(&bars[B_KVEMPTY + st]);
+          tc::tc_commit(&bars[B_PVALL]);
+          if ((s & 1) && s >= 3) tc::tc_commit(&bars[B_EPI + ((s - 3) >> 1)]);
+        }
+        __syncwarp();
+        if (lane == 0) GTR(ti, 61 + s * 4);
+        // PV(s) complete: S buffer s % 2 may take QK(s + 2); observed for every chunk, in order
+        if (!wwait(&bars[B_PVALL], gs & 1)) { ok = false; break; }
+        if (lane == 0) GTR(ti, 62 + s * 4);
+        if (s + 2 < kChunks) ok = issue_qk(s + 2, gs + 2);
+        if (lane == 0) GTR(ti, 63 + s * 4);
+      }
+    }
+    // every MMA this warp issued has completed once this commit arrives (bounded wait)
+    if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
+    __syncwarp();
+    tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL);
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 7) {
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* k_rot,
+                             const void* v, int64_t bh, float scale, void* o_loc, float* lse_loc,
+                             cudaStream_t s) {
+  using namespace lg;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_local_tma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<D>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(k_local_tma<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             100) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  Params p;
+  p.ix = ix;
+  p.o_loc = static_cast<__nv_bfloat16*>(o_loc);
+  p.lse_loc = lse_loc;
+  p.scale_log2 = scale * kLog2e;
+  p.nbz = (ix.geom.gz + BZ - 1) / BZ;
+  p.nby = (ix.geom.gy + BY - 1) / BY;
+  p.nbx = (ix.geom.gx + BX - 1) / BX;
+  p.tiles = bh * p.nbz * p.nby * p.nbx;
+  p.rows = bh * ix.n;
+  if (p.tiles <= 0) return cudaSuccess;
+  if (p.rows >= 0x7fffffffLL) return cudaErrorInvalidValue;  // gather row indices are int32
+  p.k_rot = static_cast<const __nv_bfloat16*>(k_rot);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  CUtensorMap mq, mg;
+  memset(&mg, 0, sizeof(mg));
+  if (!encode_gather_rows_bf16(&mq, q, p.rows, D)) return cudaErrorInvalidValue;
+  p.box_tma = encode_grid_i32(&mg, ix.inv, ix.geom.gz, ix.geom.gy, ix.geom.gx, kBoxX, kBoxY, kBoxZ)
+                  ? 1
+                  : 0;
+  const int64_t cap = 2 * (int64_t)sm_count();
+  const unsigned grid = (unsigned)(p.tiles < cap ? p.tiles : cap);
+  k_local_tma<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mq, mg, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void* k_rot,
+                               const void* v, int64_t bh, float scale, void* o_loc,
+                               float* lse_loc, cudaStream_t s) {
+  if (ix.geom.head_dim == 96)
+    return launch_local_tma<96>(ix, q, k_rot, v, bh, scale, o_loc, lse_loc, s);
+  return launch_local_tma<48>(ix, q, k_rot, v, bh, scale, o_loc, lse_loc, s);
+}
+
+}  // namespace p3d
+
+#ifdef P3D_TRACE_ENABLED
+extern "C" int p3d_trace_read_t(unsigned long long* host) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(host, p3d::g_trace, sizeof(unsigned long long) * 4096);
+}
+extern "C" int p3d_trace_clear_t() {
+  static unsigned long long z[4096];
+  return (int)cudaMemcpyToSymbol(p3d::g_trace, z, sizeof(z));
+}
+#endif

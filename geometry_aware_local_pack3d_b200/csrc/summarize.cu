@@ -5,6 +5,10 @@
 //   ksum[b,h,m] = (1/|S_m|) sum_{s} R(c_j) k[b,h,j],   vsum[b,h,m] = (1/|S_m|) sum_{s} v[b,h,j]
 //   with j = members[m][s], s the canonical slot.
 //
+// With a k_rot buffer the rotated key rows R(c_j) k[b,h,j] are written out as well (every
+// token is the member of exactly one block, so each row is written once), for the local branch
+// to gather without rotating.
+//
 // HBM-bound: every k and v row is read exactly once with 16-byte vector loads. One warp per
 // summary: lane l handles 16-byte chunk (l % C) of member rows s = l / C, l / C + R, ...
 // (C chunks per row, R = 32 / C rows per pass); the R partial sums are then combined in fixed
@@ -20,7 +24,8 @@ namespace p3d {
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __restrict__ k,
                                                    const T* __restrict__ v, int64_t bh_count,
-                                                   T* __restrict__ ksum, T* __restrict__ vsum) {
+                                                   T* __restrict__ ksum, T* __restrict__ vsum,
+                                                   T* __restrict__ krot) {
   constexpr int E = Vec<T>::E;
   constexpr int C = D / E;       // chunks per row
   constexpr int R = 32 / C;      // member rows per pass
@@ -64,17 +69,20 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
       const int64_t row = use ? j : 0;
       const float wgt = use ? 1.f : 0.f;
       const int cv = coord_axis(decode(cc), axis);
-      float xk[E], xv[E];
+      float xk[E], xv[E], rk[E];
       Vec<T>::load(kb + row * D + c * E, xk);
       Vec<T>::load(vb + row * D + c * E, xv);
 #pragma unroll
       for (int e = 0; e < E; e += 2) {
         const float2 cs = rope_cs(ix.rope, ix.rope_pairs, use ? cv : 0, p0 + e / 2);
-        ak[e] += wgt * (xk[e] * cs.x - xk[e + 1] * cs.y);
-        ak[e + 1] += wgt * (xk[e] * cs.y + xk[e + 1] * cs.x);
+        rk[e] = xk[e] * cs.x - xk[e + 1] * cs.y;
+        rk[e + 1] = xk[e] * cs.y + xk[e + 1] * cs.x;
+        ak[e] += wgt * rk[e];
+        ak[e + 1] += wgt * rk[e + 1];
         av[e] += wgt * xv[e];
         av[e + 1] += wgt * xv[e + 1];
       }
+      if (krot && use) Vec<T>::store(krot + bh * ix.n * D + row * D + c * E, rk);
     }
   }
   // combine the R partial sums in the fixed order r = 0, 1, ..., R-1 (each lane's own
@@ -108,24 +116,26 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
 
 template <typename T, int D>
 cudaError_t launch_summarize(const pack3d_index& ix, const void* k, const void* v, int64_t bh,
-                             void* ksum, void* vsum, cudaStream_t s) {
+                             void* ksum, void* vsum, void* krot, cudaStream_t s) {
   const int64_t tasks = bh * sum_tiles(ix.m) * 64;
   const unsigned blocks = (unsigned)((tasks + 3) / 4);
   k_summarize<T, D><<<blocks, 128, 0, s>>>(ix, static_cast<const T*>(k), static_cast<const T*>(v),
-                                            bh, static_cast<T*>(ksum), static_cast<T*>(vsum));
+                                            bh, static_cast<T*>(ksum), static_cast<T*>(vsum),
+                                            static_cast<T*>(krot));
   count_launch();
   return cudaGetLastError();
 }
 
+// krot may be null (summaries only)
 cudaError_t summarize_dispatch(const pack3d_index& ix, const void* k, const void* v, int dtype,
-                               int64_t bh, void* ksum, void* vsum, cudaStream_t s) {
+                               int64_t bh, void* ksum, void* vsum, void* krot, cudaStream_t s) {
   const int d = ix.geom.head_dim;
   if (dtype == PACK3D_BF16) {
-    if (d == 96) return launch_summarize<__nv_bfloat16, 96>(ix, k, v, bh, ksum, vsum, s);
-    return launch_summarize<__nv_bfloat16, 48>(ix, k, v, bh, ksum, vsum, s);
+    if (d == 96) return launch_summarize<__nv_bfloat16, 96>(ix, k, v, bh, ksum, vsum, krot, s);
+    return launch_summarize<__nv_bfloat16, 48>(ix, k, v, bh, ksum, vsum, krot, s);
   }
-  if (d == 96) return launch_summarize<float, 96>(ix, k, v, bh, ksum, vsum, s);
-  return launch_summarize<float, 48>(ix, k, v, bh, ksum, vsum, s);
+  if (d == 96) return launch_summarize<float, 96>(ix, k, v, bh, ksum, vsum, krot, s);
+  return launch_summarize<float, 48>(ix, k, v, bh, ksum, vsum, krot, s);
 }
 
 }  // namespace p3d

@@ -63,6 +63,10 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
 /* attn_fwd / attn_bwd flag: drop, for each query, the summaries whose block box meets the
  * cube [c-1, c+1]^3 around the query's coordinate. */
 #define PACK3D_EXCLUDE_NEAR 1u
+/* attn_fwd flag: `k` holds the rotated keys R(c_j) k_j written by pack3d_summarize_rotated
+ * (the local branch then gathers them without rotating). bf16 on the tensor-core path only;
+ * otherwise the call returns UNSUPPORTED. */
+#define PACK3D_K_ROTATED 2u
 
 /* Geometry of a packed field: grid extents, block (summary) extents, RoPE plan. */
 typedef struct {
@@ -130,12 +134,22 @@ pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const voi
                                int dtype, int batch, int heads, void* ksum, void* vsum,
                                void* stream);
 
+/* As pack3d_summarize, and in the same pass writes the rotated keys
+ * k_rot[b,h,j] = R(c_j) k[b,h,j] (axial RoPE of each token's coordinate, rounded to dtype).
+ * The pages rotate q and k inside attention; doing it for k once here, where every key row is
+ * already read, lets the local branch fetch key rows with plain row gathers.
+ * k_rot      device [B, H, N, d] dtype (output); must not alias k. */
+pack3d_status pack3d_summarize_rotated(const pack3d_index* idx, const void* k, const void* v,
+                                       int dtype, int batch, int heads, void* ksum, void* vsum,
+                                       void* k_rot, void* stream);
+
 /* PACK3D forward: local branch + global branch over (ksum, vsum) + sigmoid mixer
  * (project page Ch.3 Contracts 1-3; paper summary §3.2, §3.3, §3.5).
  * q, k, v    device [B, H, N, d] dtype;  gate device [B, H, N] dtype (logits a).
  * ksum, vsum device summary tiles from pack3d_summarize of the same k, v.
  * scale      softmax scale tau (both branches); pass 1/sqrt(d) for the usual choice.
- * flags      0 or PACK3D_EXCLUDE_NEAR.
+ * flags      0, or PACK3D_EXCLUDE_NEAR and/or PACK3D_K_ROTATED (k is then the k_rot of
+ *            pack3d_summarize_rotated).
  * o          device [B, H, N, d] dtype (output).
  * lse_loc, lse_glob  device float32 [B, H, N] or NULL: natural-log logsumexp of each
  *            branch's logits (-inf where every summary is excluded).
@@ -147,6 +161,23 @@ pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void
                               const void* vsum, int dtype, int batch, int heads, float scale,
                               uint32_t flags, void* o, float* lse_loc, float* lse_glob,
                               void* o_loc, void* o_glob, void* stream);
+
+/* The two halves of pack3d_attn_fwd as separate calls (same kernels, same results).
+ * pack3d_attn_local: the local branch alone (project page Ch.3 Contract 1; paper summary
+ *   §3.5): o_loc [B, H, N, d] dtype (output, normalised) and lse_loc float32 [B, H, N] or
+ *   NULL. flags: 0 or PACK3D_K_ROTATED.
+ * pack3d_attn_global: the global branch over (ksum, vsum) and the sigmoid mixer
+ *   o = g o_loc + (1 - g) o_glob (Ch.3 Contract 2; paper summary §3.3), given the o_loc of
+ *   pack3d_attn_local; `o` may be the same buffer as o_loc (mixed in place). lse_glob and
+ *   o_glob as in pack3d_attn_fwd. flags: 0 or PACK3D_EXCLUDE_NEAR.
+ * Errors as pack3d_attn_fwd. */
+pack3d_status pack3d_attn_local(const pack3d_index* idx, const void* q, const void* k,
+                                const void* v, int dtype, int batch, int heads, float scale,
+                                uint32_t flags, void* o_loc, float* lse_loc, void* stream);
+pack3d_status pack3d_attn_global(const pack3d_index* idx, const void* q, const void* gate,
+                                 const void* ksum, const void* vsum, const void* o_loc,
+                                 int dtype, int batch, int heads, float scale, uint32_t flags,
+                                 void* o, float* lse_glob, void* o_glob, void* stream);
 
 /* Bytes of one summary buffer (ksum or vsum) for B x H heads in summary tiles. Host-only;
  * 0 if the arguments are invalid. */

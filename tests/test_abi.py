@@ -90,6 +90,25 @@ def test_attn_calls_reject_bad_arguments_before_launch():
     assert L.pack3d_attn_fwd(ctypes.byref(ix), fake, fake, fake, fake, fake, fake, 1, 1, 1,
                              0.1, 8, fake, None, None, None, None, None) == 1
     assert L.pack3d_summarize(ctypes.byref(ix), fake, None, 1, 1, 1, fake, fake, None) == 1
+    # rotated keys: no output buffer, output aliasing the input keys, misaligned output
+    assert L.pack3d_summarize_rotated(ctypes.byref(ix), fake, fake, 1, 1, 1, fake, fake, None,
+                                      None) == 1
+    assert L.pack3d_summarize_rotated(ctypes.byref(ix), fake, fake, 1, 1, 1, fake, fake, fake,
+                                      None) == 1
+    assert L.pack3d_summarize_rotated(ctypes.byref(ix), fake, fake, 1, 1, 1, fake, fake,
+                                      ctypes.c_void_p(0x100008), None) == 5
+    # split calls: missing output, wrong flags for each half
+    assert L.pack3d_attn_local(ctypes.byref(ix), fake, fake, fake, 1, 1, 1, 0.1, 0, None, None,
+                               None) == 1
+    assert L.pack3d_attn_local(ctypes.byref(ix), fake, fake, fake, 1, 1, 1, 0.1,
+                               b.PACK3D_EXCLUDE_NEAR, fake, None, None) == 1
+    assert L.pack3d_attn_global(ctypes.byref(ix), fake, None, fake, fake, fake, 1, 1, 1, 0.1, 0,
+                                fake, None, None, None) == 1
+    assert L.pack3d_attn_global(ctypes.byref(ix), fake, fake, fake, fake, fake, 1, 1, 1, 0.1,
+                                b.PACK3D_K_ROTATED, fake, None, None, None) == 1
+    # PACK3D_K_ROTATED is a bf16 tensor-core feature: fp32 is refused before any launch
+    assert L.pack3d_attn_fwd(ctypes.byref(ix), fake, fake, fake, fake, fake, fake, 0, 1, 1,
+                             0.1, b.PACK3D_K_ROTATED, fake, None, None, None, None, None) == 2
     assert L.pack3d_attn_bwd(ctypes.byref(ix), *([fake] * 8), None, None, fake, 1, 1, 1, 0.1,
                              0, fake, fake, fake, fake, fake, 1 << 30, None) == 1
     assert b.pack3d_bwd_workspace_bytes(ix, 1, 1, 1) > 0

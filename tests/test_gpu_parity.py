@@ -51,14 +51,21 @@ def gpu_index(w, d, via="coords"):
     return m.pack3d_build_index(geom, perm=torch.from_numpy(np.asarray(w["perm"])).cuda())
 
 
-def gpu_forward(w, exclude_near, save=False, ix=None):
+def gpu_forward(w, exclude_near, save=False, ix=None, rotated=False):
+    """rotated: summaries and rotated keys in one pass, then the forward on the rotated keys
+    (the row-gather local branch)."""
     m = p3d()
     dt = tdtype(w["dtype"])
     ix = ix or gpu_index(w, w["d"])
     q, k, v, a = (w[n].to(dt).cuda().contiguous() for n in "qkva")
-    ksum, vsum = m.pack3d_summarize(ix, k, v)
-    out = m.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=exclude_near,
-                            save_for_backward=True if save else False)
+    if rotated:
+        ksum, vsum, k_rot = m.pack3d_summarize_rotated(ix, k, v)
+        out = m.pack3d_attn_fwd(ix, q, k_rot, v, a, ksum, vsum, exclude_near=exclude_near,
+                                k_rotated=True, save_for_backward=True if save else False)
+    else:
+        ksum, vsum = m.pack3d_summarize(ix, k, v)
+        out = m.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=exclude_near,
+                                save_for_backward=True if save else False)
     torch.cuda.synchronize()
     out.update(ksum=ksum, vsum=vsum, ix=ix, q=q, k=k, v=v, a=a)
     return out
@@ -157,8 +164,8 @@ def test_summaries(dtype, d):
     assert torch.count_nonzero(tail) == 0
 
 
-def full_compare(w, exclude_near, what=""):
-    g = gpu_forward(w, exclude_near, save=True)
+def full_compare(w, exclude_near, what="", rotated=False):
+    g = gpu_forward(w, exclude_near, save=True, rotated=rotated)
     ref = orc.forward(w["q"].numpy(), w["k"].numpy(), w["v"].numpy(), w["a"].numpy(),
                       w["coords"], w["grid"], w["block"], exclude_near=exclude_near)
     for key in ("o", "o_loc", "o_glob", "lse_loc", "lse_glob"):
@@ -205,8 +212,8 @@ def sampled_rows(n, count, seed=0):
     return np.unique(np.concatenate([rng.choice(n, count, replace=False), edge]))
 
 
-def sampled_compare(w, exclude_near, heads=((0, 0), (-1, -1)), count=96):
-    g = gpu_forward(w, exclude_near, save=True)
+def sampled_compare(w, exclude_near, heads=((0, 0), (-1, -1)), count=96, rotated=False):
+    g = gpu_forward(w, exclude_near, save=True, rotated=rotated)
     idx = orc.build_index(w["coords"], w["grid"], w["block"])
     rows = sampled_rows(len(w["coords"]), count)
     for (b, h) in heads:
@@ -307,3 +314,90 @@ def test_bf16_thin_grid_unit_blocks():
     w = small((3, 5, 7), (1, 1, 1), 1, 2, 48, "bf16", "random", qkv_std=48 ** -0.5)
     full_compare(w, True)
     full_compare(w, False)
+
+
+# --------------------------------------------- rotated keys + row-gather local branch (bf16)
+@pytest.mark.parametrize("d", [48, 96])
+def test_summarize_rotated_keys_and_summaries(d):
+    m = p3d()
+    w = small((4, 8, 8), (2, 4, 4), 2, 2, d, "bf16", "random", qkv_std=d ** -0.5)
+    ix = gpu_index(w, d)
+    k, v = (w[n].to(torch.bfloat16).cuda().contiguous() for n in "kv")
+    ks, vs, k_rot = m.pack3d_summarize_rotated(ix, k, v)
+    ks0, vs0 = m.pack3d_summarize(ix, k, v)
+    torch.cuda.synchronize()
+    # the same summaries as the summaries-only pass, bit for bit
+    assert torch.equal(ks, ks0) and torch.equal(vs, vs0)
+    # rotated keys: the oracle's R(c) k rounded to bf16
+    ref = orc.rope(w["k"].numpy(), w["coords"])
+    assert_close(np64(k_rot), ref, "bf16", "k_rot")
+    # the input keys are untouched
+    assert torch.equal(k.cpu(), w["k"].to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("kind", inputs.PACKINGS)
+@pytest.mark.parametrize("exclude_near", [False, True])
+def test_forward_rotated_keys_packings(kind, exclude_near):
+    w = small((8, 8, 16), (4, 4, 4), 1, 2, 96, "bf16", kind, qkv_std=96 ** -0.5)
+    full_compare(w, exclude_near, f"rot/{kind}/{exclude_near}/", rotated=True)
+
+
+@pytest.mark.parametrize("grid,block,d", [((6, 10, 12), (3, 2, 4), 48),   # partial bricks
+                                          ((5, 6, 10), (5, 3, 2), 96),    # gx*4 % 16 != 0
+                                          ((3, 5, 7), (1, 1, 1), 48),     # thin, unit blocks
+                                          ((9, 4, 4), (3, 2, 2), 96)])    # one brick column
+def test_forward_rotated_keys_ragged_grids(grid, block, d):
+    w = small(grid, block, 2, 1, d, "bf16", "random", qkv_std=d ** -0.5)
+    full_compare(w, False, "rot/", rotated=True)
+    full_compare(w, True, "rot/excl/", rotated=True)
+
+
+def test_forward_rotated_keys_65k_field_sampled():
+    sampled_compare(inputs.make_workload("field65k_bf16"), False, rotated=True)
+
+
+def test_forward_rotated_keys_match_unrotated_path_65k_field():
+    # both local-branch forms see the same rotated keys up to bf16 rounding of R(c) k: the
+    # outputs agree to bf16 resolution everywhere
+    w = inputs.make_workload("field65k_bf16")
+    a = gpu_forward(w, False, rotated=False)["o"].float()
+    b = gpu_forward(w, False, rotated=True)["o"].float()
+    assert float((a - b).abs().max()) <= 2e-2
+    assert float((a - b).norm() / a.norm()) <= 5e-3
+
+
+def test_repacking_equivariance_is_exact_rotated_keys():
+    outs = {}
+    for kind in inputs.PACKINGS:
+        w = inputs.make_workload("field65k_repack_bf16", packing_kind=kind)
+        g = gpu_forward(w, True, rotated=True)
+        outs[kind] = inputs.unpack(g["o"].cpu(), w["perm"])
+        del g
+    for kind in inputs.PACKINGS:
+        assert torch.equal(outs[kind], outs["raster"]), kind
+
+
+@pytest.mark.parametrize("dtype,d,rotated", [("bf16", 96, True), ("bf16", 96, False),
+                                             ("bf16", 48, True), ("fp32", 48, False)])
+def test_split_local_global_calls_equal_fused_forward(dtype, d, rotated):
+    # pack3d_attn_local + pack3d_attn_global run the same kernels as pack3d_attn_fwd
+    m = p3d()
+    w = small((8, 8, 16), (4, 4, 4), 2, 2, d, dtype, "morton", qkv_std=d ** -0.5)
+    g = gpu_forward(w, True, save=True, rotated=rotated)
+    kk = g["k"]
+    if rotated:
+        _, _, kk = m.pack3d_summarize_rotated(g["ix"], g["k"], g["v"])
+    lse_loc = torch.empty_like(g["lse_loc"])
+    o_loc, _ = m.pack3d_attn_local(g["ix"], g["q"], kk, g["v"], k_rotated=rotated,
+                                   lse_loc=lse_loc)
+    lse_glob = torch.empty_like(g["lse_glob"])
+    o = m.pack3d_attn_global(g["ix"], g["q"], g["a"], g["ksum"], g["vsum"], o_loc,
+                             exclude_near=True, lse_glob=lse_glob)
+    torch.cuda.synchronize()
+    assert torch.equal(o_loc, g["o_loc"]) and torch.equal(lse_loc, g["lse_loc"])
+    assert torch.equal(o, g["o"]) and torch.equal(lse_glob, g["lse_glob"])
+    # in place: the global call may mix into the o_loc buffer itself
+    o2 = m.pack3d_attn_global(g["ix"], g["q"], g["a"], g["ksum"], g["vsum"], o_loc,
+                              exclude_near=True, o=o_loc)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, g["o"])
