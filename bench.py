@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--skip-bwd", action="store_true",
+                    help="skip the (untimed-step) backward and index-build measurements")
     return ap.parse_args()
 
 
@@ -312,6 +314,52 @@ def main():
         vals = [float(x) for x in tt.tolist()]
         ms, ms_k = vals[0], dict(zip(("summarize", "local", "global"), vals[1:]))
 
+    # Outside the headline step: the index build (once per geometry) and the backward of the
+    # same field (dO ~ N(0, 1), seed 2), each timed with CUDA events on this stream.
+    extra = {}
+    if not args.skip_bwd and world == 1:
+        coords_d = torch.from_numpy(w["coords"]).to(dev)
+        ie0, ie1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p3d.pack3d_build_index(geom, coords=coords_d)
+        ie0.record(stream)
+        for _ in range(3):
+            p3d.pack3d_build_index(geom, coords=coords_d)
+        ie1.record(stream)
+        torch.cuda.synchronize()
+        extra["index_build"] = {"ms": ie0.elapsed_time(ie1) / 3,
+                                "note": "inverse map, neighbour and block tables, RoPE table; "
+                                        "includes the call's one host synchronisation"}
+        saved = p3d.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=excl,
+                                    save_for_backward=True)
+        dO = inputs.pack(inputs.upstream_grad(B, H, w["grid"], d), w["perm"]).to(dt).to(dev)
+        ws = torch.empty(p3d.pack3d_bwd_workspace_bytes(ix, 1 if dt == torch.bfloat16 else 0,
+                                                        B, H), dtype=torch.uint8, device=dev)
+        p3d.pack3d_attn_bwd(ix, q, k, v, a, ksum, vsum, saved, dO, exclude_near=excl, workspace=ws)
+        be0, be1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        be0.record(stream)
+        nb = 3
+        for _ in range(nb):
+            p3d.pack3d_attn_bwd(ix, q, k, v, a, ksum, vsum, saved, dO, exclude_near=excl,
+                                workspace=ws)
+        be1.record(stream)
+        torch.cuda.synchronize()
+        bms = be0.elapsed_time(be1) / nb
+        M = int(np.prod([g_ // b_ for g_, b_ in zip(w["grid"], w["block"])]))
+        # SURVEY-style count: the global branch's backward is 2.5x its forward contraction
+        # (dS, dq, dK_sum, dV_sum: 5 products of N x M x d per (batch, head))
+        bflops = 10.0 * N * M * d * B * H
+        peaks_b = measured_peaks()
+        extra["attn_bwd"] = {"ms": bms, "tokens_per_s": B * N / (bms / 1e3),
+                             "roofline": {"bound": "tensor", "algorithmic_flops": bflops,
+                                          "achieved": bflops / (bms / 1e3) / 1e12,
+                                          "peak": peaks_b["bf16"], "unit": "TFLOP/s",
+                                          "frac": bflops / (bms / 1e3) / 1e12 / peaks_b["bf16"]},
+                             "path": "global branch on tensor cores (k_bwd_dsum_tc, "
+                                     "k_bwd_dq_tc); row prologue, local branch, un-pooling and "
+                                     "inverse RoPE on CUDA cores (k_bwd_prep, k_bwd_dq, "
+                                     "k_bwd_dkv)"}
+        del saved, dO, ws
+
     # end to end through the public API with host buffers: H2D of the inputs and D2H of o
     e2e = None
     if not args.skip_e2e:
@@ -387,6 +435,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
         }
+        line.update(extra)
         if not args.skip_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

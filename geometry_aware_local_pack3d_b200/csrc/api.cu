@@ -16,8 +16,8 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               const void* vsum, const void* o_loc, const void* o_glob,
                               const float* lse_loc, const float* lse_glob, const void* dO,
                               int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
-                              void* dv, void* dgate, void* ws, cudaStream_t s);
-size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh);
+                              void* dv, void* dgate, void* ws, bool tc, cudaStream_t s);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, bool tc);
 cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                  const void* ksum, const void* vsum, const void* o_loc,
                                  int dtype, int64_t bh, float scale, int excl, void* o,
@@ -61,6 +61,11 @@ pack3d_status check_rows(std::initializer_list<const void*> ptrs) {
 }
 
 pack3d_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
+
+bool bf16_tensor_path();
+// the backward's global branch runs on tensor cores for bf16 (unless the CUDA-core path is
+// selected); float32 stays on CUDA cores for the 1e-4 bar
+bool bwd_tensor_path(int dtype) { return dtype == PACK3D_BF16 && bf16_tensor_path(); }
 
 // bf16 runs the global branch on tcgen05 tensor cores unless PACK3D_BF16_PATH=simt selects the
 // CUDA-core kernels (both compute the whole operator).
@@ -216,7 +221,7 @@ extern "C" size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int b
 extern "C" size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch,
                                              int heads) {
   if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;
-  return bwd_workspace_bytes(*idx, (int64_t)batch * heads);
+  return bwd_workspace_bytes(*idx, (int64_t)batch * heads, bwd_tensor_path(dtype));
 }
 
 extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
@@ -237,9 +242,10 @@ extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q,
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return PACK3D_ERR_ALIGN;
   if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
   const int64_t bh = (int64_t)batch * heads;
-  if (workspace_bytes < bwd_workspace_bytes(*idx, bh)) return PACK3D_ERR_WORKSPACE;
+  const bool tc = bwd_tensor_path(dtype);
+  if (workspace_bytes < bwd_workspace_bytes(*idx, bh, tc)) return PACK3D_ERR_WORKSPACE;
   const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
   return cuda_status(bwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc,
                                        lse_glob, dO, dtype, bh, scale, excl, dq, dk, dv, dgate,
-                                       workspace, static_cast<cudaStream_t>(stream)));
+                                       workspace, tc, static_cast<cudaStream_t>(stream)));
 }

@@ -18,6 +18,8 @@
 // never on memory slots, except the sums over all queries in k_bwd_dsum.
 #include <math.h>
 
+#include "bwd_work.h"
+
 #include "common.cuh"
 #include "launch.h"
 #include "vec.cuh"
@@ -264,15 +266,6 @@ __device__ __forceinline__ void wr_rotate(const pack3d_index& ix, const Coord& c
   }
 }
 
-struct BwdWork {
-  float* qr;    // [BH, N, D]
-  float* kr;    // [BH, N, D]
-  float* Dl;    // [BH, N]
-  float* Dg;    // [BH, N]
-  float* dks;   // [BH, M, D]
-  float* dvs;   // [BH, M, D]
-};
-
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __restrict__ q,
                                                   const T* __restrict__ k,
@@ -300,10 +293,21 @@ __global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __re
     }
   }
   wr_load<T, D>(dO + row * D, d, lane);
+  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
+  if (w.qtb) {
+    // tensor-core path: the rotated q and (1 - g) dO rows in bf16, the MMA operands
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) {
+      const int e = lane + 32 * t;
+      if (e < D) {
+        w.qtb[row * D + e] = __float2bfloat16_rn(w.qr[row * D + e]);
+        w.dogb[row * D + e] = __float2bfloat16_rn((1.f - g) * d.x[t]);
+      }
+    }
+  }
   wr_load<T, D>(o_loc + row * D, a, lane);
   wr_load<T, D>(o_glob + row * D, b, lane);
   const float dl = wr_dot<D>(d, a), dgl = wr_dot<D>(d, b);
-  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
   if (lane == 0) {
     dgate[row] = from_f<T>((dl - dgl) * g * (1.f - g));
     w.Dl[row] = g * dl;
@@ -392,9 +396,14 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
 #pragma unroll
     for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = fmaf(ds, x.x[t], acc.x[t]);
   }
-  // global branch
+  // global branch (computed by the tensor-core kernel into the workspace on that path)
   const float lg = lse_glob[row], Dg = w.Dg[row];
-  if (lg != -INFINITY) {
+  if (w.dqg) {
+    WarpRow<D> gq;
+    wr_load_f<D>(w.dqg + row * D, gq, lane);
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] += gq.x[t];
+  } else if (lg != -INFINITY) {
     const int M = (int)ix.m;
     for (int m = 0; m < M; ++m) {
       if (exclude_near && block_is_near(ix, m, c)) continue;
@@ -447,12 +456,24 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
   // un-pool: 1/|S| of the block summary's gradient
   const int b = ix.block_of[j];
   const float inv = 1.f / (float)ix.count[b];
-  wr_load_f<D>(w.dks + (bh * ix.m + b) * D, x, lane);
-  wr_load_f<D>(w.dvs + (bh * ix.m + b) * D, d, lane);
+  // the summary gradients may come in per-query-range partials: summed in range order
+  const int64_t part = (int64_t)(rows / ix.n) * ix.m * D;
+  WarpRow<D> sk, sv;
+#pragma unroll
+  for (int t = 0; t < WarpRow<D>::KT; ++t) sk.x[t] = sv.x[t] = 0.f;
+  for (int sp = 0; sp < w.nsplit; ++sp) {
+    wr_load_f<D>(w.dks + sp * part + (bh * ix.m + b) * D, x, lane);
+    wr_load_f<D>(w.dvs + sp * part + (bh * ix.m + b) * D, d, lane);
+#pragma unroll
+    for (int t = 0; t < WarpRow<D>::KT; ++t) {
+      sk.x[t] += x.x[t];
+      sv.x[t] += d.x[t];
+    }
+  }
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) {
-    ak.x[t] = fmaf(x.x[t], inv, ak.x[t]);
-    av.x[t] = fmaf(d.x[t], inv, av.x[t]);
+    ak.x[t] = fmaf(sk.x[t], inv, ak.x[t]);
+    av.x[t] = fmaf(sv.x[t], inv, av.x[t]);
   }
   wr_rotate<D>(ix, c, ak, lane, -1.f);
   wr_store<T, D>(dk + row * D, ak, lane);
@@ -460,34 +481,21 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
 }
 
 // ------------------------------------------------------------------------------ launchers
-size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh) {
-  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t D = ix.geom.head_dim;
-  return 2 * a(sizeof(float) * bh * ix.n * D) + 2 * a(sizeof(float) * bh * ix.n) +
-         2 * a(sizeof(float) * bh * ix.m * D);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, bool tc) {
+  return bwd_workspace_bytes_for(ix, bh, tc);
 }
 
-static BwdWork carve(const pack3d_index& ix, int64_t bh, void* ws) {
-  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t D = ix.geom.head_dim;
-  char* p = static_cast<char*>(ws);
-  BwdWork w;
-  w.qr = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n * D);
-  w.kr = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n * D);
-  w.Dl = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n);
-  w.Dg = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.n);
-  w.dks = reinterpret_cast<float*>(p); p += a(sizeof(float) * bh * ix.m * D);
-  w.dvs = reinterpret_cast<float*>(p);
-  return w;
-}
+cudaError_t bwd_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* ksum,
+                            const void* vsum, const float* lse_glob, int64_t bh, float scale,
+                            int excl, cudaStream_t s);
 
 template <typename T, int D>
 cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
                      const void* gate, const void* ksum, const void* vsum, const void* o_loc,
                      const void* o_glob, const float* lse_loc, const float* lse_glob,
                      const void* dO, int64_t bh, float scale, int excl, void* dq, void* dk,
-                     void* dv, void* dgate, void* ws, cudaStream_t s) {
-  const BwdWork w = carve(ix, bh, ws);
+                     void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
+  const BwdWork w = bwd_carve(ix, bh, ws, tc);
   const int64_t rows = bh * ix.n;
   const unsigned rb = (unsigned)((rows + 3) / 4);
   const unsigned mb = (unsigned)((bh * ix.m + 3) / 4);
@@ -499,15 +507,23 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
   k_bwd_prep<T, D><<<rb, 128, 0, s>>>(ix, tq, tk, tg, static_cast<const T*>(o_loc),
                                        static_cast<const T*>(o_glob), tdo, rows, w,
                                        static_cast<T*>(dgate));
-  k_bwd_dsum<T, D><<<mb, 128, 0, s>>>(ix, static_cast<const T*>(ksum),
-                                       static_cast<const T*>(vsum), tg, tdo, lse_glob, scale,
-                                       excl, bh, w);
+  count_launch();
+  if (tc) {
+    // the global branch's summary gradients and its part of dq on tensor cores
+    const cudaError_t e = bwd_tc_dispatch(ix, w, ksum, vsum, lse_glob, bh, scale, excl, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    k_bwd_dsum<T, D><<<mb, 128, 0, s>>>(ix, static_cast<const T*>(ksum),
+                                         static_cast<const T*>(vsum), tg, tdo, lse_glob, scale,
+                                         excl, bh, w);
+    count_launch();
+  }
   k_bwd_dq<T, D><<<rb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
                                      static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
                                      scale, excl, rows, w, static_cast<T*>(dq));
   k_bwd_dkv<T, D><<<rb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, w,
                                       static_cast<T*>(dk), static_cast<T*>(dv));
-  count_launch(4);
+  count_launch(2);
   return cudaGetLastError();
 }
 
@@ -557,11 +573,11 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               const void* vsum, const void* o_loc, const void* o_glob,
                               const float* lse_loc, const float* lse_glob, const void* dO,
                               int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
-                              void* dv, void* dgate, void* ws, cudaStream_t s) {
+                              void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
   const int d = ix.geom.head_dim;
 #define P3D_BWD(T, D)                                                                         \
   bwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc, lse_glob, dO, bh, scale, \
-                 excl, dq, dk, dv, dgate, ws, s)
+                 excl, dq, dk, dv, dgate, ws, tc, s)
   if (dtype == PACK3D_BF16) return d == 96 ? P3D_BWD(__nv_bfloat16, 96) : P3D_BWD(__nv_bfloat16, 48);
   return d == 96 ? P3D_BWD(float, 96) : P3D_BWD(float, 48);
 #undef P3D_BWD

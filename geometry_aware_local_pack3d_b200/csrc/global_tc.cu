@@ -7,22 +7,25 @@
 //
 // Work unit: 256 consecutive memory rows of one (batch, head) = two 128-row query tiles that
 // share every summary chunk (halves the L2 reads of the summaries). Persistent CTAs walk the
-// units round-robin. Warp roles (448 threads):
+// units round-robin. Warp roles (480 threads):
 //   warps 0-3   softmax + epilogue of tile 0 (thread = row, TMEM lanes 0..127); the epilogue
-//               parks o_glob in the tile's (by then consumed) q area and applies the mixer
-//               with coalesced loads and stores, then releases the q buffer to the producer
+//               normalises O, writes lse, and parks o_glob in the tile's (by then consumed)
+//               q area
 //   warps 4-7   softmax + epilogue of tile 1
-//   warps 8-11  query producer: cp.async of q rows into the K-major shared-memory A operand
-//               (double-buffered across units), then axial RoPE applied in place
-//   warp 12     MMA issuer (one thread) and TMEM owner
-//   warp 13     summary loader: each 64-summary chunk of ksum / vsum is one summary tile, i.e.
+//   warps 8-11  query producer and mixer: before refilling a q buffer, apply the sigmoid mixer
+//               to the unit staged there (coalesced o_loc / gate loads and o stores, overlapped
+//               with the next unit's compute); then cp.async of q rows into the K-major
+//               shared-memory A operand (double-buffered across units) and axial RoPE in place
+//   warp 12     MMA issuer of tile 0 (whole warp, one elected lane issues) and TMEM owner
+//   warp 13     MMA issuer of tile 1
+//   warp 14     summary loader: each 64-summary chunk of ksum / vsum is one summary tile, i.e.
 //               already in the operand layout, fetched by one contiguous bulk copy per tensor
 //               into a 4-stage ring
 // Per 64-summary chunk j and tile t:  S_t[j%2] = q~_t K_j^T (SS MMA, fp32 in TMEM) -> the
 // softmax threads turn it into P = exp2(s - m) in bf16, written over S in TMEM ->
-// O_t += P V_j (TS MMA). S is double-buffered per tile; the issuer runs QK two chunks ahead
-// (PV_0(j), PV_1(j), QK_0(j+2), QK_1(j+2)), so the next S of a tile is ready when its softmax
-// finishes a chunk, and the two tiles' softmaxes overlap each other. The running max uses a lazy
+// O_t += P V_j (TS MMA). S is double-buffered per tile; each tile's issuer runs QK two chunks
+// ahead of PV, so the next S of a tile is ready when its softmax finishes a chunk, and the two
+// tiles' chains run independently on the shared tensor core. The running max uses a lazy
 // rescale: O_t is corrected in TMEM only when a row's max grows by more than 2^8.
 // The summary order is the same for every query (block ids ascending) and rows never interact,
 // so a coordinate-carrying repack permutes the output bit for bit.
@@ -39,11 +42,18 @@ constexpr int kRows = 128;        // rows per tile
 constexpr int kTiles = 2;         // tiles per unit
 constexpr int kChunk = 64;        // summaries per chunk
 constexpr int kStages = 4;        // summary ring depth
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kProd = 128;        // query producer threads
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kRopeSmemBytes = 16384;
+#ifndef P3D_POLY_EVERY
+#define P3D_POLY_EVERY 0
+#endif
+// softmax exponentials: one column pair in kPolyEvery computed on the FMA pipe (0: none). On
+// B200 the kernel measured 0.600 / 0.605 / 0.610 / 0.624 ms with none / 1 in 8 / 1 in 4 /
+// 1 in 2 at the 65,536-token field, so the MUFU pipe is not what bounds it: off by default.
+constexpr int kPolyEvery = P3D_POLY_EVERY;
 
 // TMEM columns: tile t uses [256 t, 256 t + 256): S buffers at +0 and +64, O at +128.
 __host__ __device__ constexpr uint32_t s_col(int t, int b) { return 256u * t + 64u * b; }
@@ -71,8 +81,8 @@ enum {
   B_PFULL = 16,   // [tile][buf]
   B_PVDONE = 20,  // [tile][buf]
   B_OFREE = 24,   // [tile]
-  B_DONE = 26,
-  B_COUNT = 27
+  B_DONE = 26,    // [tile]
+  B_COUNT = 28
 };
 
 struct Params {
@@ -152,9 +162,9 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     }
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bars[B_KVFULL + i], 1);
-      tc::mbar_init(&bars[B_KVEMPTY + i], 1);
+      tc::mbar_init(&bars[B_KVEMPTY + i], kTiles);  // both tiles' PVs of the chunk
     }
-    tc::mbar_init(&bars[B_DONE], 1);
+    for (int i = 0; i < kTiles; ++i) tc::mbar_init(&bars[B_DONE + i], 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -232,7 +242,9 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (!masked) {
 #pragma unroll
-          for (int k = 0; k < kChunk; ++k) mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
+          for (int k = 0; k < kChunk; k += 2)
+            mx[(k >> 1) & 3] =
+                tc::max3f(mx[(k >> 1) & 3], __uint_as_float(r[k]), __uint_as_float(r[k + 1]));
         } else {
 #pragma unroll
           for (int k = 0; k < kChunk; ++k) {
@@ -271,21 +283,29 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           m_run = m_new;
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-        // P = exp2(s * scale - m) as bf16 over the first half of this S buffer
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = exp2(s * scale - m) as bf16 over the first half of this S buffer; the scaling
+        // and the row sum run two columns per instruction (packed fp32)
+        float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        const float2 sl2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
         for (int c0 = 0; c0 < kChunk; c0 += 32) {
           uint32_t p[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(r[c0 + k]), P.scale_log2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(r[c0 + k + 1]), P.scale_log2, neg_m));
-            ls[(k >> 1) & 3] += p0 + p1;
-            p[k >> 1] = tc::pack_bf16(p0, p1);
+            const float2 x = tc::fma2(
+                make_float2(__uint_as_float(r[c0 + k]), __uint_as_float(r[c0 + k + 1])), sl2, nm2);
+            // one pair in kPolyEvery on the FMA pipe: the MUFU pipe bounds this loop otherwise
+            const float2 e = (kPolyEvery > 0 && (k >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1) ==
+                                                    kPolyEvery - 1)
+                                 ? tc::exp2_poly2(x)
+                                 : make_float2(ex2(x.x), ex2(x.y));
+            ls[(k >> 1) & 3] = tc::add2(ls[(k >> 1) & 3], e);
+            p[k >> 1] = tc::pack_bf16(e.x, e.y);
           }
           tc::tmem_st16(tl + s_col(t, b) + (c0 >> 1), p);
         }
-        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l_run += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
         if (fine) P3D_TRACE(1800 + j * 8 + 3);
         tc::tmem_wait_st();
         if (fine) P3D_TRACE(1800 + j * 8 + 4);
@@ -295,7 +315,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         if (rin == 0 && pc == 1 && j < 10) P3D_TRACE_C(3400 + j * 4 + t * 2 + 1);
       }
       if (!ok) break;
-      // epilogue: o_glob = O / l, lse, mixer
+      // epilogue: o_glob = O / l and lse (the producer warps apply the mixer)
       const uint32_t gl = (uint32_t)(pc * NC + NC - 1);
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVDONE + 2 * t + (gl & 1)], (gl >> 1) & 1)))
         break;
@@ -316,59 +336,20 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(&bars[B_OFREE + t]);
       if (rin == 0 && pc < 3) P3D_TRACE(1500 + pc * 4 + t * 2);
-      // Mixer, coalesced: the unit's last QK has completed (its PV is done), so this tile's q
-      // area in shared memory is free and holds exactly 128 rows of D bf16. Each thread parks
-      // its o_glob row there (16-byte chunk c of row r at chunk slot (c + r) mod KC, which
-      // spreads a warp's stores over the banks); each warp then walks its 32 rows piece by
-      // piece, so consecutive lanes touch consecutive 16 bytes of o_loc, o and o_glob.
+      // The unit's last QK has completed (its PV is done), so this tile's q area in shared
+      // memory is free and holds exactly 128 rows of d bf16: each thread parks its o_glob row
+      // there (16-byte chunk c of row r at chunk slot (c + r) mod KC, which spreads a warp's
+      // stores over the banks). The producer warps apply the mixer from there, with coalesced
+      // accesses, while these warps go on with the next unit.
       uint8_t* stage = smem + S::kQ + (pc & 1) * kTiles * S::kQTile + t * S::kQTile;
       tc::fence_proxy_async_smem();  // the tensor core's reads of this area came first
 #pragma unroll
       for (int c = 0; c < KC; ++c)
         *reinterpret_cast<uint4*>(stage + rin * (D * 2) + ((c + rin) % KC) * 16) =
             make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
-      float gsig = 0.f;
-      if (valid) {
-        const int64_t grow = bh * N + row;
-        if (P.lse_glob)
-          P.lse_glob[grow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-        gsig = 1.f / (1.f + __expf(-__bfloat162float(P.gate[grow])));
-      }
-      __syncwarp();
-      const int wr0 = (warp & 3) * 32;  // the warp's first row within the tile
-      const int64_t row_w = row - lane;  // memory row of the warp's first row
-      // o_loc may alias o (in-place mixing): every piece a lane stores is one it loaded itself,
-      // and all of its loads come first
-      uint4 lrow[KC];
-#pragma unroll
-      for (int i = 0; i < KC; ++i) {
-        const int pidx = i * 32 + lane, r = pidx / KC, c = pidx % KC;
-        lrow[i] = row_w + r < N
-                      ? reinterpret_cast<const uint4*>(P.o_loc + (bh * N + row_w + r) * D)[c]
-                      : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int i = 0; i < KC; ++i) {
-        const int pidx = i * 32 + lane, r = pidx / KC, c = pidx % KC;
-        const float g = __shfl_sync(0xffffffffu, gsig, r);
-        const uint4 gv = *reinterpret_cast<const uint4*>(stage + (wr0 + r) * (D * 2) +
-                                                         ((c + wr0 + r) % KC) * 16);
-        if (row_w + r >= N) continue;
-        const uint32_t lw[4] = {lrow[i].x, lrow[i].y, lrow[i].z, lrow[i].w};
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        uint32_t outw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float g0 = __uint_as_float(gw[k] << 16), g1 = __uint_as_float(gw[k] & 0xffff0000u);
-          const float l0 = __uint_as_float(lw[k] << 16), l1 = __uint_as_float(lw[k] & 0xffff0000u);
-          outw[k] = tc::pack_bf16(g * l0 + (1.f - g) * g0, g * l1 + (1.f - g) * g1);
-        }
-        const int64_t off = (bh * N + row_w + r) * D;
-        reinterpret_cast<uint4*>(P.o + off)[c] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        if (P.o_glob) reinterpret_cast<uint4*>(P.o_glob + off)[c] = gv;
-      }
-      // this thread's reads of the q area are done: the producer may refill it
-      tc::mbar_arrive(&bars[B_QEMPTY + (pc & 1)]);
+      if (valid && P.lse_glob)
+        P.lse_glob[bh * N + row] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      tc::mbar_arrive(&bars[B_QEMPTY + (pc & 1)]);  // o_glob of this unit is staged
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------------ query producer
@@ -378,14 +359,71 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     constexpr int DA = D / 3;
     int32_t* coord_s = reinterpret_cast<int32_t*>(smem + S::kCoord);
     const float* rope = P.rope_in_smem ? reinterpret_cast<const float*>(smem + S::kRope) : P.ix.rope;
+    // Mixer of unit k (the k-th unit of this CTA), once the softmax warps have staged its
+    // o_glob in q buffer k % 2: o = g o_loc + (1 - g) o_glob, g = sigmoid(a), over the unit's
+    // 256 rows with consecutive threads on consecutive 16 bytes. o_loc may alias o (in-place
+    // mixing): every piece a thread stores is one it loaded itself, and loads come first.
+    auto mix = [&](int k) {
+      const int64_t uk = blockIdx.x + (int64_t)k * gridDim.x;
+      const int64_t bh = uk / P.units_per_bh;
+      const int64_t row0 = (uk % P.units_per_bh) * (kRows * kTiles);
+      const uint8_t* stage = smem + S::kQ + (k & 1) * kTiles * S::kQTile;
+      constexpr int G = D == 96 ? 12 : 6;  // pieces per thread in flight
+      static_assert((kRows * kTiles * KC / kProd) % G == 0, "mixer groups");
+#pragma unroll 1
+      for (int g0 = 0; g0 < kRows * kTiles * KC / kProd; g0 += G) {
+        uint4 lv[G];
+        float gs[G];
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const int pidx = (g0 + i) * kProd + ptid, r = pidx / KC, c = pidx % KC;
+          const int64_t grow = row0 + r;
+          lv[i] = make_uint4(0u, 0u, 0u, 0u);
+          gs[i] = 0.f;
+          if (grow < N) {
+            lv[i] = reinterpret_cast<const uint4*>(P.o_loc + (bh * N + grow) * D)[c];
+            gs[i] = __bfloat162float(P.gate[bh * N + grow]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const int pidx = (g0 + i) * kProd + ptid, r = pidx / KC, c = pidx % KC;
+          const int64_t grow = row0 + r;
+          if (grow >= N) continue;
+          const int rin = r & (kRows - 1);
+          const uint4 gv = *reinterpret_cast<const uint4*>(
+              stage + (r >> 7) * S::kQTile + rin * (D * 2) + ((c + rin) % KC) * 16);
+          const float g = 1.f / (1.f + __expf(-gs[i]));
+          const uint32_t lw[4] = {lv[i].x, lv[i].y, lv[i].z, lv[i].w};
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+          uint32_t outw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g0f = __uint_as_float(gw[e] << 16), g1f = __uint_as_float(gw[e] & 0xffff0000u);
+            const float l0 = __uint_as_float(lw[e] << 16), l1 = __uint_as_float(lw[e] & 0xffff0000u);
+            outw[e] = tc::pack_bf16(g * l0 + (1.f - g) * g0f, g * l1 + (1.f - g) * g1f);
+          }
+          const int64_t off = (bh * N + grow) * D;
+          reinterpret_cast<uint4*>(P.o + off)[c] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          if (P.o_glob) reinterpret_cast<uint4*>(P.o_glob + off)[c] = gv;
+        }
+      }
+    };
+    // one thread waits for unit k's staging; the named barrier hands its verdict to all
+    auto wait_staged = [&](int k) -> bool {
+      if (ptid == 0) *prod_ok = ab.wait(&bars[B_QEMPTY + (k & 1)], (k >> 1) & 1) ? 1 : 0;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      return *prod_ok != 0;
+    };
     int pc = 0;
+    bool pok = true;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int b = pc & 1;
       if (pc >= 2) {
-        // one thread waits; the named barrier hands its verdict to all producer warps
-        if (ptid == 0) *prod_ok = ab.wait(&bars[B_QEMPTY + b], ((pc >> 1) - 1) & 1) ? 1 : 0;
+        // q buffer b still holds unit pc-2's staged o_glob: mix it, then refill the buffer
+        if (!wait_staged(pc - 2)) { pok = false; break; }
+        mix(pc - 2);
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (!*prod_ok) break;
       }
       if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4);
       const int64_t bh = u / P.units_per_bh;
@@ -437,15 +475,23 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       tc::mbar_arrive(&bars[B_QFULL + b]);
       if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4 + 2);
     }
-  } else if (warp == 12) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Fixed order per chunk j: PV_0(j), PV_1(j), then QK_0(j+2), QK_1(j+2). QK_t(j+2) reuses
-    // the S buffer of chunk j, so it only waits for PV_t(j) to complete; it is thus issued
-    // while the softmax of tile t works on chunk j+1, and S_t(j+2) is ready when that softmax
-    // finishes. The whole warp runs the schedule with warp-uniform values (descriptors are
-    // formed once and advanced by adding address offsets: the start address is the low 14
-    // bits and every offset keeps it in range); one elected lane issues the tcgen05 MMAs and
-    // commits. This keeps the issuing instruction stream short and uniform.
+    // the last one or two units are still staged
+    for (int k = pc >= 2 ? pc - 2 : 0; k < pc && pok; ++k) {
+      if (!wait_staged(k)) break;
+      mix(k);
+    }
+  } else if (warp < 12 + kTiles) {
+    // ------------------------------------------------------------------ MMA issuers
+    // One warp per query tile (warp 12: tile 0, warp 13: tile 1), so each tile's chain
+    // softmax(j) -> PV(j) -> QK(j+2) advances on its own and neither waits behind the other's
+    // MMAs or barrier probes. Per chunk j: PV_t(j) once the softmax has written P_t(j), then --
+    // once PV_t(j) has completed, which frees the S buffer of chunk j -- QK_t(j+2), so S_t(j+1)
+    // and S_t(j+2) are ready while the softmax works. The whole warp runs the schedule with
+    // warp-uniform values (descriptors formed once and advanced by adding address offsets: the
+    // start address is the low 14 bits and every offset keeps it in range); one elected lane
+    // issues the MMAs and commits. A summary stage is released once both tiles' PVs of the
+    // chunk have completed (KVEMPTY expects one commit from each issuer).
+    const int t = warp - 12;
     const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
     const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
@@ -461,25 +507,25 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++pc) {
       const int qb = pc & 1;
       if (!wwait(&bars[B_QFULL + qb], (pc >> 1) & 1)) break;
-      if (lane == 0 && pc < 3) P3D_TRACE(2600 + pc);
+      if (lane == 0 && t == 0 && pc < 3) P3D_TRACE(2600 + pc);
       tc::tc_fence_after();
-      const uint64_t qd0 =
-          tc::smem_desc(tc::smem_u32(smem + S::kQ + qb * kTiles * S::kQTile), 2048, 128);
+      const uint64_t a0 =
+          tc::smem_desc(tc::smem_u32(smem + S::kQ + qb * kTiles * S::kQTile + t * S::kQTile),
+                        2048, 128);
       // QK_t(j): S_t[buffer of j] = q~_t K_j^T
-      auto issue_qk = [&](int t, int j) -> bool {
+      auto issue_qk = [&](int j) -> bool {
         const uint32_t kv = kv_it + j;
         const uint32_t gi = (uint32_t)(pc * NC + j);
         const int b = gi & 1;
         const bool fq = lane == 0 && pc == 1 && j >= 4 && j < 8;
-        const int fs = 3000 + j * 40 + t * 10;
+        [[maybe_unused]] const int fs = 3000 + j * 40 + t * 10;
         if (fq) P3D_TRACE_C(fs);
-        if (t == 0 && !wwait(&bars[B_KVFULL + kv % kStages], (kv / kStages) & 1)) return false;
+        if (!wwait(&bars[B_KVFULL + kv % kStages], (kv / kStages) & 1)) return false;
         if (fq) P3D_TRACE_C(fs + 1);
         // this S buffer held P of chunk gi - 2 until that PV completed
         if (gi >= 2 && !wwait(&bars[B_PVDONE + 2 * t + b], ((gi >> 1) - 1) & 1)) return false;
         if (fq) P3D_TRACE_C(fs + 2);
         tc::tc_fence_after();
-        const uint64_t a0 = qd0 + (uint64_t)((t * S::kQTile) >> 4);
         const uint64_t b0 = kd0 + (uint64_t)(((kv % kStages) * S::kCTile) >> 4);
         const uint32_t dt = tb + s_col(t, b);
         if (tc::elect_one()) {
@@ -498,48 +544,41 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         issued = true;
         return true;
       };
-      for (int j = 0; j < 2 && j < NC && ok; ++j)
-        for (int t = 0; t < kTiles && ok; ++t) ok = issue_qk(t, j);
+      for (int j = 0; j < 2 && j < NC && ok; ++j) ok = issue_qk(j);
       for (int j = 0; j < NC && ok; ++j) {
         const uint32_t kv = kv_it + j;
         const uint32_t gi = (uint32_t)(pc * NC + j);
         const int b = gi & 1;
+        const bool fp = lane == 0 && pc == 1 && j >= 2 && j < 6;
+        [[maybe_unused]] const int fs = 3000 + (j + 2) * 40 + 20 + t * 10;
+        if (fp) P3D_TRACE_C(fs);
+        if (!wwait(&bars[B_PFULL + 2 * t + b], (gi >> 1) & 1)) { ok = false; break; }
+        if (fp) P3D_TRACE_C(fs + 1);
+        // the first PV of a unit overwrites O_t: the previous epilogue must have read it
+        if (j == 0 && pc > 0 && !wwait(&bars[B_OFREE + t], (pc - 1) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
         const uint64_t v0 = vd0 + (uint64_t)(((kv % kStages) * S::kCTile) >> 4);
-        for (int t = 0; t < kTiles; ++t) {
-          const bool fp = lane == 0 && pc == 1 && j >= 2 && j < 6;
-          const int fs = 3000 + (j + 2) * 40 + 20 + t * 10;
-          if (fp) P3D_TRACE_C(fs);
-          if (!wwait(&bars[B_PFULL + 2 * t + b], (gi >> 1) & 1)) { ok = false; break; }
-          if (fp) P3D_TRACE_C(fs + 1);
-          // the first PV of a unit overwrites O_t: the previous epilogue must have read it
-          if (j == 0 && pc > 0 && !wwait(&bars[B_OFREE + t], (pc - 1) & 1)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint32_t at = tb + s_col(t, b), dt = tb + o_col(t);
-          if (tc::elect_one()) {
+        const uint32_t at = tb + s_col(t, b), dt = tb + o_col(t);
+        if (tc::elect_one()) {
 #pragma unroll
-            for (int ks = 0; ks < kChunk / 16; ++ks)
-              tc::mma_ts(dt, at + ks * 8, v0 + (uint64_t)(ks * (256 >> 4)), id_pv,
-                         (j > 0 || ks > 0) ? 1u : 0u);
-            tc::tc_commit(&bars[B_PVDONE + 2 * t + b]);
-          }
-          __syncwarp();
-          if (fp) P3D_TRACE_C(fs + 4);
-          if (lane == 0 && pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2 + 1);
+          for (int ks = 0; ks < kChunk / 16; ++ks)
+            tc::mma_ts(dt, at + ks * 8, v0 + (uint64_t)(ks * (256 >> 4)), id_pv,
+                       (j > 0 || ks > 0) ? 1u : 0u);
+          tc::tc_commit(&bars[B_PVDONE + 2 * t + b]);
+          tc::tc_commit(&bars[B_KVEMPTY + kv % kStages]);
         }
-        if (!ok) break;
-        // both tiles' PVs of chunk j are issued: the stage is free once they complete
-        if (tc::elect_one()) tc::tc_commit(&bars[B_KVEMPTY + kv % kStages]);
         __syncwarp();
-        if (j + 2 < NC)
-          for (int t = 0; t < kTiles && ok; ++t) ok = issue_qk(t, j + 2);
+        if (fp) P3D_TRACE_C(fs + 4);
+        if (lane == 0 && pc < 3) P3D_TRACE(2000 + pc * 128 + t * 64 + j * 2 + 1);
+        if (j + 2 < NC) ok = issue_qk(j + 2);
       }
       kv_it += NC;
     }
     // every MMA issued by this warp has completed before TMEM is released
     if (issued) {
-      if (tc::elect_one()) tc::tc_commit(&bars[B_DONE]);
+      if (tc::elect_one()) tc::tc_commit(&bars[B_DONE + t]);
       __syncwarp();
-      tc::mbar_wait(&bars[B_DONE], 0, 4000000000LL);
+      tc::mbar_wait(&bars[B_DONE + t], 0, 4000000000LL);
     }
   } else {
     // ------------------------------------------------------------------ summary loader

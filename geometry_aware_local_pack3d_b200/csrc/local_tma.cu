@@ -272,9 +272,11 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         tc::tmem_wait_ld();
         const uint64_t win = nb[i];
 #pragma unroll
-        for (int k = 0; k < kNK; ++k) {
+        for (int k = 0; k < kNK; k += 2) {
           if (!((win >> k) & 1ull)) r[k] = 0xff800000u;
-          mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(r[k]));
+          if (!((win >> (k + 1)) & 1ull)) r[k + 1] = 0xff800000u;
+          mx[(k >> 1) & 3] =
+              tc::max3f(mx[(k >> 1) & 3], __uint_as_float(r[k]), __uint_as_float(r[k + 1]));
         }
         const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
         const float m_new = fmaxf(m_run, cmax);
@@ -303,16 +305,20 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
           m_run = m_new;
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // scaling and row sum two columns per instruction (packed fp32)
+        float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        const float2 sl2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(neg_m, neg_m);
         uint32_t p[kNK / 2];
 #pragma unroll
         for (int k = 0; k < kNK; k += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(r[k]), P.scale_log2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(r[k + 1]), P.scale_log2, neg_m));
-          ls[(k >> 1) & 3] += p0 + p1;
-          p[k >> 1] = tc::pack_bf16(p0, p1);
+          const float2 x =
+              tc::fma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, nm2);
+          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          ls[(k >> 1) & 3] = tc::add2(ls[(k >> 1) & 3], e);
+          p[k >> 1] = tc::pack_bf16(e.x, e.y);
         }
-        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l_run += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
         tc::tmem_st16(tl + s_col(b), *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
         lg::tmem_st8(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[8]>(&p[16]));
         tc::tmem_wait_st();

@@ -401,3 +401,19 @@ def test_split_local_global_calls_equal_fused_forward(dtype, d, rotated):
                               exclude_near=True, o=o_loc)
     torch.cuda.synchronize()
     assert torch.equal(o2, g["o"])
+
+
+@pytest.mark.parametrize("grid,block,d,exclude_near", [
+    ((8, 12, 20), (2, 2, 2), 96, True),    # N 1,920, M 240: two 128-summary tiles, ragged ranges
+    ((8, 12, 20), (2, 2, 2), 48, False),
+    ((3, 5, 7), (1, 1, 1), 48, True),      # M = N = 105: unit blocks, one partial query tile
+    ((4, 4, 4), (2, 2, 2), 96, True),      # every summary excluded for some rows
+])
+def test_backward_bf16_tensor_core_edges(grid, block, d, exclude_near):
+    # bf16 runs the global branch's backward on tensor cores (k_bwd_dsum_tc, k_bwd_dq_tc)
+    w = small(grid, block, 1, 2, d, "bf16", "random", qkv_std=d ** -0.5)
+    gr, dO = gpu_backward(w, exclude_near)
+    ref = orc.backward(w["q"].numpy(), w["k"].numpy(), w["v"].numpy(), w["a"].numpy(),
+                       dO.numpy(), w["coords"], w["grid"], w["block"], exclude_near=exclude_near)
+    for key, rk in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dgate", "da")):
+        assert_close(np64(gr[key]), ref[rk], "bf16", key)
