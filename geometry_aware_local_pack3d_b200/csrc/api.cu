@@ -17,7 +17,7 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               const float* lse_loc, const float* lse_glob, const void* dO,
                               int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
                               void* dv, void* dgate, void* ws, bool tc, cudaStream_t s);
-size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, bool tc);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, int dtype, bool tc);
 cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                  const void* ksum, const void* vsum, const void* o_loc,
                                  int dtype, int64_t bh, float scale, int excl, void* o,
@@ -221,7 +221,7 @@ extern "C" size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int b
 extern "C" size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch,
                                              int heads) {
   if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;
-  return bwd_workspace_bytes(*idx, (int64_t)batch * heads, bwd_tensor_path(dtype));
+  return bwd_workspace_bytes(*idx, (int64_t)batch * heads, dtype, bwd_tensor_path(dtype));
 }
 
 extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
@@ -243,7 +243,7 @@ extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q,
   if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
   const int64_t bh = (int64_t)batch * heads;
   const bool tc = bwd_tensor_path(dtype);
-  if (workspace_bytes < bwd_workspace_bytes(*idx, bh, tc)) return PACK3D_ERR_WORKSPACE;
+  if (workspace_bytes < bwd_workspace_bytes(*idx, bh, dtype, tc)) return PACK3D_ERR_WORKSPACE;
   const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
   return cuda_status(bwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc,
                                        lse_glob, dO, dtype, bh, scale, excl, dq, dk, dv, dgate,

@@ -284,25 +284,24 @@ __global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __re
   wr_rotate<D>(ix, c, a, lane, 1.f);
   wr_load<T, D>(k + row * D, b, lane);
   wr_rotate<D>(ix, c, b, lane, 1.f);
+  T* qr = static_cast<T*>(w.qr);
+  T* kr = static_cast<T*>(w.kr);
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) {
     const int e = lane + 32 * t;
     if (e < D) {
-      w.qr[row * D + e] = a.x[t];
-      w.kr[row * D + e] = b.x[t];
+      qr[row * D + e] = from_f<T>(a.x[t]);
+      kr[row * D + e] = from_f<T>(b.x[t]);
     }
   }
   wr_load<T, D>(dO + row * D, d, lane);
   const float g = 1.f / (1.f + expf(-to_f(gate[row])));
-  if (w.qtb) {
-    // tensor-core path: the rotated q and (1 - g) dO rows in bf16, the MMA operands
+  if (w.dogb) {
+    // tensor-core path: (1 - g) dO rows in bf16, an MMA operand (the rotated q is qr)
 #pragma unroll
     for (int t = 0; t < WarpRow<D>::KT; ++t) {
       const int e = lane + 32 * t;
-      if (e < D) {
-        w.qtb[row * D + e] = __float2bfloat16_rn(w.qr[row * D + e]);
-        w.dogb[row * D + e] = __float2bfloat16_rn((1.f - g) * d.x[t]);
-      }
+      if (e < D) w.dogb[row * D + e] = __float2bfloat16_rn((1.f - g) * d.x[t]);
     }
   }
   wr_load<T, D>(o_loc + row * D, a, lane);
@@ -339,7 +338,7 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
     const float lse = lse_glob[row];
     if (lse == -INFINITY) continue;
     if (exclude_near && block_is_near(ix, m, decode(ix.coord[i]))) continue;
-    wr_load_f<D>(w.qr + row * D, x, lane);
+    wr_load<T, D>(static_cast<const T*>(w.qr) + row * D, x, lane);
     wr_load<T, D>(dO + row * D, d, lane);
     const float g1 = 1.f - 1.f / (1.f + expf(-to_f(gate[row])));
     const float s = wr_dot<D>(x, km) * scale;
@@ -380,7 +379,7 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
   const Coord c = decode(ix.coord[i]);
   const float g = 1.f / (1.f + expf(-to_f(gate[row])));
   WarpRow<D> qr, d, acc, x, y;
-  wr_load_f<D>(w.qr + row * D, qr, lane);
+  wr_load<T, D>(static_cast<const T*>(w.qr) + row * D, qr, lane);
   wr_load<T, D>(dO + row * D, d, lane);
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = 0.f;
@@ -389,7 +388,7 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
   for (int o = 0; o < kNbr; ++o) {
     const int j = ix.nbr[i * kNbr + o];
     if (j < 0) continue;
-    wr_load_f<D>(w.kr + (rowbase + j) * D, x, lane);
+    wr_load<T, D>(static_cast<const T*>(w.kr) + (rowbase + j) * D, x, lane);
     wr_load<T, D>(v + (rowbase + j) * D, y, lane);
     const float p = expf(wr_dot<D>(qr, x) * scale - ll);
     const float ds = p * (g * wr_dot<D>(d, y) - Dl) * scale;
@@ -433,7 +432,7 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
   const int64_t rowbase = bh * ix.n;
   const Coord c = decode(ix.coord[j]);
   WarpRow<D> kr, vj, ak, av, x, d;
-  wr_load_f<D>(w.kr + row * D, kr, lane);
+  wr_load<T, D>(static_cast<const T*>(w.kr) + row * D, kr, lane);
   wr_load<T, D>(v + row * D, vj, lane);
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
@@ -442,7 +441,7 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
     const int i = ix.nbr[j * kNbr + o];
     if (i < 0) continue;
     const int64_t ri = rowbase + i;
-    wr_load_f<D>(w.qr + ri * D, x, lane);
+    wr_load<T, D>(static_cast<const T*>(w.qr) + ri * D, x, lane);
     wr_load<T, D>(dO + ri * D, d, lane);
     const float g = 1.f / (1.f + expf(-to_f(gate[ri])));
     const float p = expf(wr_dot<D>(x, kr) * scale - lse_loc[ri]);
@@ -481,8 +480,8 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
 }
 
 // ------------------------------------------------------------------------------ launchers
-size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, bool tc) {
-  return bwd_workspace_bytes_for(ix, bh, tc);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, int dtype, bool tc) {
+  return bwd_workspace_bytes_for(ix, bh, dtype == PACK3D_BF16 ? 2 : 4, tc);
 }
 
 cudaError_t bwd_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* ksum,
@@ -495,7 +494,7 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
                      const void* o_glob, const float* lse_loc, const float* lse_glob,
                      const void* dO, int64_t bh, float scale, int excl, void* dq, void* dk,
                      void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
-  const BwdWork w = bwd_carve(ix, bh, ws, tc);
+  const BwdWork w = bwd_carve(ix, bh, ws, sizeof(T), tc);
   const int64_t rows = bh * ix.n;
   const unsigned rb = (unsigned)((rows + 3) / 4);
   const unsigned mb = (unsigned)((bh * ix.m + 3) / 4);

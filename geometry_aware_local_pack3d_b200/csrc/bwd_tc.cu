@@ -15,9 +15,10 @@
 //               form dS in bf16 over S, and dq~ += dS K (TS MMA, K read as the MN-major
 //               operand). Output: the global part of dq~ in fp32.
 // k_bwd_dsum_tc summary-major: a CTA owns 128 summaries of one (batch, head) and one query
-//               range; per 64-query tile S^T = K q~^T and dP^T = V dO_g^T, then P^T and dS^T
-//               in bf16 over them, dV += P^T dO_g and dK += dS^T q~ (TS MMAs, q~ and dO_g read
-//               as MN-major operands). Output: per-range partial dK, dV in fp32.
+//               range; per 64-query tile S^T = K q~^T and dP^T = V dO_g^T (double-buffered in
+//               TMEM, issued two tiles ahead), then P^T and dS^T in bf16 over them,
+//               dV += P^T dO_g and dK += dS^T q~ (TS MMAs, q~ and dO_g read as MN-major
+//               operands). Output: per-range partial dK, dV in fp32.
 // Operands use the no-swizzle core-matrix layout; the summary tiles are already in it.
 #include <math.h>
 
@@ -362,26 +363,24 @@ template <int D> struct Smem {
   static constexpr int kV = kK + kATile;
   static constexpr int kQ = kV + kATile;               // [stages]
   static constexpr int kG = kQ + kStages * kBTile;     // [stages]
-  static constexpr int kRowInfo = kG + kStages * kBTile;  // [stages][64] RowInfo
-  static constexpr int kBar = kRowInfo + kStages * btc::kChunk * 36;
+  static constexpr int kRowF = kG + kStages * kBTile;          // [stages][64] (nl, D)
+  static constexpr int kRowX = kRowF + kStages * btc::kChunk * 8;  // [stages][64][6] ranges
+  static constexpr int kBar = kRowX + kStages * btc::kChunk * 24;
   static constexpr int kBytes = kBar + 256;
 };
 enum {
-  B_QFULL = 0, B_QEMPTY = 3, B_AFULL = 6, B_SFULL = 7, B_PFULL = 8, B_DONE = 9, B_DRAIN = 10,
-  B_COUNT = 11
+  B_QFULL = 0, B_QEMPTY = 3, B_AFULL = 6, B_SFULL = 7, B_PFULL = 9, B_DONE = 11, B_DRAIN = 13,
+  B_COUNT = 14
 };
 constexpr int kThreads = 288;  // elementwise 0-3, producer 4-7, MMA 8
 constexpr int kProd = 128;
-constexpr uint32_t kS = 0, kP = 64, kK = 128, kV = 256;  // TMEM columns
-// per query of a tile: -lse log2(e), D, whether it has any global gradient, and the block
-// coordinate ranges of the summaries exclude_near drops for it (empty when off)
-struct RowInfo {
-  float nl;
-  float Dg;
-  int32_t live;
-  int32_t z0, z1, y0, y1, x0, x1;
-};
-static_assert(sizeof(RowInfo) == 36, "row info");
+// TMEM columns: dK, dV accumulators; S^T and dP^T double-buffered (buffer b of tile i = i % 2)
+constexpr uint32_t kK = 0, kV = 128;
+__device__ __forceinline__ uint32_t s_col(int b) { return 256u + 128u * b; }
+__device__ __forceinline__ uint32_t p_col(int b) { return 320u + 128u * b; }
+// Per query of a tile (staged by the producer): (-lse log2(e), D) -- -inf in place of the
+// first term when the query has no global gradient, so that P = 0 -- and the block
+// coordinate ranges [z0, z1] x [y0, y1] x [x0, x1] of the summaries exclude_near drops.
 }  // namespace bds
 
 template <int D>
@@ -412,9 +411,11 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
       tc::mbar_init(&bars[B_QEMPTY + i], 1);
     }
     tc::mbar_init(&bars[B_AFULL], kProd);
-    tc::mbar_init(&bars[B_SFULL], 1);
-    tc::mbar_init(&bars[B_PFULL], 128);
-    tc::mbar_init(&bars[B_DONE], 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars[B_SFULL + i], 1);
+      tc::mbar_init(&bars[B_PFULL + i], 128);
+      tc::mbar_init(&bars[B_DONE + i], 1);
+    }
     tc::mbar_init(&bars[B_DRAIN], 1);
     abort_flag[0] = 0;
     tc::fence_mbar_init();
@@ -424,7 +425,6 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  RowInfo* rinfo = reinterpret_cast<RowInfo*>(smem + S::kRowInfo);
 
   if (warp < 4) {
     // ------------------------------------------------------------ elementwise + epilogue
@@ -435,18 +435,21 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
     const int nby = g.gy / g.by, nbx = g.gx / g.bx;
     const int bz = m / (nby * nbx), byy = (m / nbx) % nby, bxx = m % nbx;  // block coords
     const bool excl = P.exclude_near != 0;
+    const float2* rowf = reinterpret_cast<const float2*>(smem + S::kRowF);
+    const int* rowx = reinterpret_cast<const int*>(smem + S::kRowX);
     bool ok = true;
     for (int i = 0; i < NT; ++i) {
-      const int st = i % kStages;
-      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL], i & 1))) { ok = false; break; }
+      const int st = i % kStages, b = i & 1;
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + b], (i >> 1) & 1))) { ok = false; break; }
       tc::tc_fence_after();
-      const RowInfo* ri = rinfo + st * btc::kChunk;
+      const float2* rf = rowf + st * btc::kChunk;
+      const int* rx = rowx + st * btc::kChunk * 6;
       // two halves of 32 query columns: P^T over S^T, dS^T over dP^T (columns already read)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t sv[32], dv[32];
-        tc::tmem_ld32(tl + kS + 32 * h, sv);
-        tc::tmem_ld32(tl + kP + 32 * h, dv);
+        tc::tmem_ld32(tl + s_col(b) + 32 * h, sv);
+        tc::tmem_ld32(tl + p_col(b) + 32 * h, dv);
         tc::tmem_wait_ld();
         uint32_t pp[16], pd[16];
 #pragma unroll
@@ -454,27 +457,31 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
           float pv[2], dsv[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const RowInfo& r = ri[32 * h + k + e];  // broadcast: every thread reads the same
-            bool use = r.live != 0;
-            if (excl && use)
-              use = !(bz >= r.z0 && bz <= r.z1 && byy >= r.y0 && byy <= r.y1 && bxx >= r.x0 &&
-                      bxx <= r.x1);
-            const float p = use ? btc::ex2(fmaf(__uint_as_float(sv[k + e]), P.scale_log2, r.nl)) : 0.f;
+            const int col = 32 * h + k + e;
+            const float2 r = rf[col];  // broadcast: every thread reads the same
+            float p = btc::ex2(fmaf(__uint_as_float(sv[k + e]), P.scale_log2, r.x));
+            if (excl) {
+              const int* x = rx + col * 6;
+              if (bz >= x[0] && bz <= x[1] && byy >= x[2] && byy <= x[3] && bxx >= x[4] &&
+                  bxx <= x[5])
+                p = 0.f;
+            }
             pv[e] = p;
-            dsv[e] = p * (__uint_as_float(dv[k + e]) - r.Dg) * P.scale;
+            dsv[e] = p * (__uint_as_float(dv[k + e]) - r.y) * P.scale;
           }
           pp[k >> 1] = tc::pack_bf16(pv[0], pv[1]);
           pd[k >> 1] = tc::pack_bf16(dsv[0], dsv[1]);
         }
-        tc::tmem_st16(tl + kS + 16 * h, pp);
-        tc::tmem_st16(tl + kP + 16 * h, pd);
+        tc::tmem_st16(tl + s_col(b) + 16 * h, pp);
+        tc::tmem_st16(tl + p_col(b) + 16 * h, pd);
       }
       tc::tmem_wait_st();
       tc::tc_fence_before();
-      tc::mbar_arrive(&bars[B_PFULL]);
+      tc::mbar_arrive(&bars[B_PFULL + b]);
     }
     // epilogue: this range's partial dK, dV of the tile's summaries
-    if (ok && NT > 0 && __all_sync(0xffffffffu, ab.wait(&bars[B_DONE], (NT - 1) & 1))) {
+    if (ok && NT > 0 &&
+        __all_sync(0xffffffffu, ab.wait(&bars[B_DONE + ((NT - 1) & 1)], ((NT - 1) >> 1) & 1))) {
       tc::tc_fence_after();
       const int64_t part = (int64_t)split * P.bh_count * M * D;
       float* dk = P.out0 + part + (bh * M + m) * D;
@@ -549,21 +556,16 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
       }
       if (ptid < btc::kChunk) {
         const int64_t row = row0 + ptid;
-        RowInfo r;
-        r.live = 0;
-        r.nl = 0.f;
-        r.Dg = 0.f;
-        r.z0 = r.y0 = r.x0 = 0;
-        r.z1 = r.y1 = r.x1 = -1;
+        float2 rf = make_float2(-INFINITY, 0.f);
+        btc::ExclBox ex{0, -1, 0, -1, 0, -1};
         if (row < N) {
           const float lse = P.lse[bh * N + row];
-          r.live = lse != -INFINITY ? 1 : 0;
-          r.nl = r.live ? -lse * kLog2e : 0.f;
-          r.Dg = P.Dg[bh * N + row];
-          const btc::ExclBox ex = btc::excl_box(P.ix, P.ix.coord[row], P.exclude_near != 0);
-          r.z0 = ex.z0; r.z1 = ex.z1; r.y0 = ex.y0; r.y1 = ex.y1; r.x0 = ex.x0; r.x1 = ex.x1;
+          rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY, P.Dg[bh * N + row]);
+          ex = btc::excl_box(P.ix, P.ix.coord[row], P.exclude_near != 0);
         }
-        rinfo[st * btc::kChunk + ptid] = r;
+        reinterpret_cast<float2*>(smem + S::kRowF)[st * btc::kChunk + ptid] = rf;
+        int* x = reinterpret_cast<int*>(smem + S::kRowX) + (st * btc::kChunk + ptid) * 6;
+        x[0] = ex.z0; x[1] = ex.z1; x[2] = ex.y0; x[3] = ex.y1; x[4] = ex.x0; x[5] = ex.x1;
       }
       tc::cp_async_commit();
       tc::cp_async_wait_all();
@@ -585,40 +587,47 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity, false));
     };
-    bool ok = wwait(&bars[B_AFULL], 0);
-    for (int i = 0; i < NT && ok; ++i) {
-      const int st = i % kStages;
-      if (!wwait(&bars[B_QFULL + st], (i / kStages) & 1)) break;
-      // S^T and dP^T hold the previous tile's P^T and dS^T until its MMAs have completed
-      if (i >= 1 && !wwait(&bars[B_DONE], (i - 1) & 1)) break;
+    // SS(i): S^T and dP^T of query tile i into buffer i % 2 (free once TS(i - 2) completed)
+    auto issue_ss = [&](int i) -> bool {
+      const int st = i % kStages, b = i & 1;
+      if (!wwait(&bars[B_QFULL + st], (i / kStages) & 1)) return false;
+      if (i >= 2 && !wwait(&bars[B_DONE + b], ((i - 2) >> 1) & 1)) return false;
       tc::tc_fence_after();
       const uint64_t so = (uint64_t)((st * S::kBTile) >> 4);
       if (tc::elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          tc::mma_ss(tb + kS, kd + (uint64_t)(ks * (4096 >> 4)),
+          tc::mma_ss(tb + s_col(b), kd + (uint64_t)(ks * (4096 >> 4)),
                      qk0 + so + (uint64_t)(ks * (2 * CB >> 4)), id_s, ks > 0);
-          tc::mma_ss(tb + kP, vd + (uint64_t)(ks * (4096 >> 4)),
+          tc::mma_ss(tb + p_col(b), vd + (uint64_t)(ks * (4096 >> 4)),
                      gk0 + so + (uint64_t)(ks * (2 * CB >> 4)), id_s, ks > 0);
         }
-        tc::tc_commit(&bars[B_SFULL]);
+        tc::tc_commit(&bars[B_SFULL + b]);
       }
       __syncwarp();
-      if (!wwait(&bars[B_PFULL], i & 1)) break;
+      return true;
+    };
+    bool ok = wwait(&bars[B_AFULL], 0);
+    for (int i = 0; i < 2 && i < NT && ok; ++i) ok = issue_ss(i);
+    for (int i = 0; i < NT && ok; ++i) {
+      const int st = i % kStages, b = i & 1;
+      if (!wwait(&bars[B_PFULL + b], (i >> 1) & 1)) break;
       tc::tc_fence_after();
+      const uint64_t so = (uint64_t)((st * S::kBTile) >> 4);
       if (tc::elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < btc::kChunk / 16; ++ks) {
           // dV += P^T dO_g;  dK += dS^T q~   (K = the tile's 64 queries)
-          tc::mma_ts(tb + kV, tb + kS + ks * 8, gm0 + so + (uint64_t)(ks * (256 >> 4)), id_o,
-                     (i > 0 || ks > 0) ? 1u : 0u);
-          tc::mma_ts(tb + kK, tb + kP + ks * 8, qm0 + so + (uint64_t)(ks * (256 >> 4)), id_o,
-                     (i > 0 || ks > 0) ? 1u : 0u);
+          tc::mma_ts(tb + kV, tb + s_col(b) + ks * 8, gm0 + so + (uint64_t)(ks * (256 >> 4)),
+                     id_o, (i > 0 || ks > 0) ? 1u : 0u);
+          tc::mma_ts(tb + kK, tb + p_col(b) + ks * 8, qm0 + so + (uint64_t)(ks * (256 >> 4)),
+                     id_o, (i > 0 || ks > 0) ? 1u : 0u);
         }
         tc::tc_commit(&bars[B_QEMPTY + st]);
-        tc::tc_commit(&bars[B_DONE]);
+        tc::tc_commit(&bars[B_DONE + b]);
       }
       __syncwarp();
+      if (i + 2 < NT) ok = issue_ss(i + 2);
     }
     if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
     __syncwarp();

@@ -14,47 +14,47 @@ namespace p3d {
 constexpr int kDsumSplit = 2;
 
 struct BwdWork {
-  float* qr;    // [BH, N, d]  rotated q
-  float* kr;    // [BH, N, d]  rotated k
+  void* qr;     // [BH, N, d]  rotated q, in the I/O type (bf16 or fp32)
+  void* kr;     // [BH, N, d]  rotated k, in the I/O type
   float* Dl;    // [BH, N]     <g dO, o_loc>
   float* Dg;    // [BH, N]     <(1 - g) dO, o_glob>
   float* dks;   // [nsplit][BH, M, d]  gradient of the key summaries (per query range)
   float* dvs;   // [nsplit][BH, M, d]  gradient of the value summaries
   int nsplit;   // query ranges in dks / dvs (1: CUDA-core path)
   // tensor-core path only (null otherwise)
-  __nv_bfloat16* qtb;   // [BH, N, d]  rotated q, bf16
+  __nv_bfloat16* qtb;   // [BH, N, d]  rotated q, bf16 (the qr array itself)
   __nv_bfloat16* dogb;  // [BH, N, d]  (1 - g) dO, bf16
   float* dqg;           // [BH, N, d]  global branch's part of dq~ (rotated space)
 };
 
 inline size_t bwd_align(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Bytes of workspace; `tc` adds the tensor-core path's arrays.
-inline size_t bwd_workspace_bytes_for(const pack3d_index& ix, int64_t bh, bool tc) {
+// Bytes of workspace for I/O elements of `el` bytes; `tc` (bf16 only) adds the tensor-core
+// path's arrays.
+inline size_t bwd_workspace_bytes_for(const pack3d_index& ix, int64_t bh, size_t el, bool tc) {
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
   const int ns = tc ? kDsumSplit : 1;
-  size_t b = 2 * bwd_align(sizeof(float) * rows * D) + 2 * bwd_align(sizeof(float) * rows) +
+  size_t b = 2 * bwd_align(el * rows * D) + 2 * bwd_align(sizeof(float) * rows) +
              2 * bwd_align(sizeof(float) * ns * sums * D);
-  if (tc)
-    b += 2 * bwd_align(sizeof(__nv_bfloat16) * rows * D) + bwd_align(sizeof(float) * rows * D);
+  if (tc) b += bwd_align(sizeof(__nv_bfloat16) * rows * D) + bwd_align(sizeof(float) * rows * D);
   return b;
 }
 
-inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, bool tc) {
+inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, size_t el, bool tc) {
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
   char* p = static_cast<char*>(ws);
   BwdWork w;
   w.nsplit = tc ? kDsumSplit : 1;
-  w.qr = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows * D);
-  w.kr = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows * D);
+  w.qr = p; p += bwd_align(el * rows * D);
+  w.kr = p; p += bwd_align(el * rows * D);
   w.Dl = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows);
   w.Dg = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows);
   w.dks = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * w.nsplit * sums * D);
   w.dvs = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * w.nsplit * sums * D);
   w.qtb = w.dogb = nullptr;
   w.dqg = nullptr;
-  if (tc) {
-    w.qtb = reinterpret_cast<__nv_bfloat16*>(p); p += bwd_align(sizeof(__nv_bfloat16) * rows * D);
+  if (tc) {  // bf16 I/O: qr already holds the rotated q in bf16
+    w.qtb = static_cast<__nv_bfloat16*>(w.qr);
     w.dogb = reinterpret_cast<__nv_bfloat16*>(p); p += bwd_align(sizeof(__nv_bfloat16) * rows * D);
     w.dqg = reinterpret_cast<float*>(p);
   }
