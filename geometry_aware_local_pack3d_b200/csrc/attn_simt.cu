@@ -11,9 +11,12 @@
 // Backward (paper summary §3.4), one warp per row, lanes over head dims:
 //   k_bwd_prep    rotated q, k; dgate; D_loc = <g dO, o_loc>, D_glob = <(1-g) dO, o_glob>.
 //   k_bwd_dsum    dK_sum[m] = sum_i dS_im q~_i and dV_sum[m] = sum_i P_im (1-g_i) dO_i.
-//   k_bwd_dq      dq = R(c)^T (sum_j dS_ij k~_j + sum_m dS_im K_sum[m]).
+//   k_bwd_dq      dq = R(c)^T (sum_j dS_ij k~_j + sum_m dS_im K_sum[m]); 8 lanes per row.
 //   k_bwd_dkv     dk, dv gathered over the key's own neighbourhood (the 3x3x3 relation is
-//                 symmetric, so no scatter/atomics) plus 1/|S| of its block's summary grads.
+//                 symmetric, so no scatter/atomics) plus 1/|S| of its block's summary grads;
+//                 8 lanes per row.
+// On the bf16 tensor-core path the global branch's summary gradients and its part of dq come
+// from the kernels of bwd_tc.cu instead of k_bwd_dsum and the summary loop of k_bwd_dq.
 // Every reduction order depends on coordinates (offset order, canonical slots, summary ids),
 // never on memory slots, except the sums over all queries in k_bwd_dsum.
 #include <math.h>
@@ -266,6 +269,74 @@ __device__ __forceinline__ void wr_rotate(const pack3d_index& ix, const Coord& c
   }
 }
 
+// Group layout for the neighbour loops of the backward: 8 lanes per row, 4 rows per warp;
+// lane g of a group owns the KD = d/8 consecutive dims [g KD, g KD + KD). Dot products reduce
+// over the 8 lanes in 3 shuffle steps, and every rotation pair (2p, 2p+1) stays in one lane.
+template <int D> struct GRow {
+  static constexpr int KD = D / 8;
+  static_assert(KD % 2 == 0, "a lane must own whole rotation pairs");
+  float x[KD];
+};
+template <typename T> struct Pair2;
+template <> struct Pair2<float> {
+  __device__ static float2 get(const float* p, int k) { return reinterpret_cast<const float2*>(p)[k]; }
+  __device__ static void put(float* p, int k, float a, float b) {
+    reinterpret_cast<float2*>(p)[k] = make_float2(a, b);
+  }
+};
+template <> struct Pair2<__nv_bfloat16> {
+  __device__ static float2 get(const __nv_bfloat16* p, int k) {
+    return __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(p)[k]);
+  }
+  __device__ static void put(__nv_bfloat16* p, int k, float a, float b) {
+    reinterpret_cast<__nv_bfloat162*>(p)[k] = __floats2bfloat162_rn(a, b);
+  }
+};
+template <typename T, int D>
+__device__ __forceinline__ void gr_load(const T* __restrict__ row, GRow<D>& r, int g) {
+  const T* p = row + g * GRow<D>::KD;
+#pragma unroll
+  for (int k = 0; k < GRow<D>::KD / 2; ++k) {
+    const float2 v = Pair2<T>::get(p, k);
+    r.x[2 * k] = v.x;
+    r.x[2 * k + 1] = v.y;
+  }
+}
+template <typename T, int D>
+__device__ __forceinline__ void gr_store(T* row, const GRow<D>& r, int g) {
+  T* p = row + g * GRow<D>::KD;
+#pragma unroll
+  for (int k = 0; k < GRow<D>::KD / 2; ++k) Pair2<T>::put(p, k, r.x[2 * k], r.x[2 * k + 1]);
+}
+__device__ __forceinline__ float group_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  return x;
+}
+template <int D>
+__device__ __forceinline__ float gr_dot(const GRow<D>& a, const GRow<D>& b) {
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < GRow<D>::KD; ++k) s = fmaf(a.x[k], b.x[k], s);
+  return group_sum(s);
+}
+// r <- R(c) r (sign 1) or R(c)^T r (sign -1)
+template <int D>
+__device__ __forceinline__ void gr_rotate(const pack3d_index& ix, const Coord& c, GRow<D>& r,
+                                          int g, float sign) {
+  constexpr int DA = D / 3;
+#pragma unroll
+  for (int k = 0; k < GRow<D>::KD; k += 2) {
+    const int e = g * GRow<D>::KD + k;
+    const int axis = e / DA, p = (e % DA) / 2;
+    const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+    const float sn = sign * cs.y, x0 = r.x[k], x1 = r.x[k + 1];
+    r.x[k] = x0 * cs.x - x1 * sn;
+    r.x[k + 1] = x0 * sn + x1 * cs.x;
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __restrict__ q,
                                                   const T* __restrict__ k,
@@ -361,6 +432,7 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
   }
 }
 
+// dq = R(c)^T (sum_j dS_ij k~_j + global part); 8 lanes per query row.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __restrict__ v,
                                                 const T* __restrict__ ksum,
@@ -371,53 +443,65 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
                                                 const float* __restrict__ lse_glob, float scale,
                                                 int exclude_near, int64_t rows, BwdWork w,
                                                 T* __restrict__ dq) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
+  const int g = threadIdx.x & 7;
+  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x >> 3) + (threadIdx.x >> 3);
+  const bool active = row0 < rows;  // inactive groups follow along on row 0 and store nothing
+  const int64_t row = active ? row0 : 0;
   const int64_t bh = row / ix.n, i = row % ix.n;
   const int64_t rowbase = bh * ix.n;
   const Coord c = decode(ix.coord[i]);
-  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
-  WarpRow<D> qr, d, acc, x, y;
-  wr_load<T, D>(static_cast<const T*>(w.qr) + row * D, qr, lane);
-  wr_load<T, D>(dO + row * D, d, lane);
+  const float gt = 1.f / (1.f + expf(-to_f(gate[row])));
+  const T* qr = static_cast<const T*>(w.qr);
+  const T* kr = static_cast<const T*>(w.kr);
+  GRow<D> q, d, acc, x, y;
+  gr_load<T, D>(qr + row * D, q, g);
+  gr_load<T, D>(dO + row * D, d, g);
 #pragma unroll
-  for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = 0.f;
+  for (int k = 0; k < GRow<D>::KD; ++k) acc.x[k] = 0.f;
   // local branch
   const float ll = lse_loc[row], Dl = w.Dl[row];
   for (int o = 0; o < kNbr; ++o) {
     const int j = ix.nbr[i * kNbr + o];
-    if (j < 0) continue;
-    wr_load<T, D>(static_cast<const T*>(w.kr) + (rowbase + j) * D, x, lane);
-    wr_load<T, D>(v + (rowbase + j) * D, y, lane);
-    const float p = expf(wr_dot<D>(qr, x) * scale - ll);
-    const float ds = p * (g * wr_dot<D>(d, y) - Dl) * scale;
+    const int64_t rj = rowbase + (j >= 0 ? j : 0);
+    gr_load<T, D>(kr + rj * D, x, g);
+    gr_load<T, D>(v + rj * D, y, g);
+    const float sd = gr_dot<D>(q, x), dp = gr_dot<D>(d, y);
+    const float p = j >= 0 ? expf(sd * scale - ll) : 0.f;
+    const float ds = p * (gt * dp - Dl) * scale;
 #pragma unroll
-    for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = fmaf(ds, x.x[t], acc.x[t]);
+    for (int k = 0; k < GRow<D>::KD; ++k) acc.x[k] = fmaf(ds, x.x[k], acc.x[k]);
   }
   // global branch (computed by the tensor-core kernel into the workspace on that path)
-  const float lg = lse_glob[row], Dg = w.Dg[row];
   if (w.dqg) {
-    WarpRow<D> gq;
-    wr_load_f<D>(w.dqg + row * D, gq, lane);
+    gr_load<float, D>(w.dqg + row * D, x, g);
 #pragma unroll
-    for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] += gq.x[t];
-  } else if (lg != -INFINITY) {
-    const int M = (int)ix.m;
-    for (int m = 0; m < M; ++m) {
-      if (exclude_near && block_is_near(ix, m, c)) continue;
-      wr_load_sum<T, D>(ksum, bh, m, sum_tiles(M), x, lane);
-      wr_load_sum<T, D>(vsum, bh, m, sum_tiles(M), y, lane);
-      const float p = expf(wr_dot<D>(qr, x) * scale - lg);
-      const float ds = p * ((1.f - g) * wr_dot<D>(d, y) - Dg) * scale;
+    for (int k = 0; k < GRow<D>::KD; ++k) acc.x[k] += x.x[k];
+  } else {
+    const float lg = lse_glob[row], Dg = w.Dg[row];
+    if (lg != -INFINITY) {
+      const int M = (int)ix.m;
+      const int64_t mt = sum_tiles(M);
+      for (int m = 0; m < M; ++m) {
+        if (exclude_near && block_is_near(ix, m, c)) continue;
 #pragma unroll
-      for (int t = 0; t < WarpRow<D>::KT; ++t) acc.x[t] = fmaf(ds, x.x[t], acc.x[t]);
+        for (int k = 0; k < GRow<D>::KD; ++k) {
+          const int e = g * GRow<D>::KD + k;
+          x.x[k] = to_f(ksum[sum_index(bh, m, e, D, mt)]);
+          y.x[k] = to_f(vsum[sum_index(bh, m, e, D, mt)]);
+        }
+        const float p = expf(gr_dot<D>(q, x) * scale - lg);
+        const float ds = p * ((1.f - gt) * gr_dot<D>(d, y) - Dg) * scale;
+#pragma unroll
+        for (int k = 0; k < GRow<D>::KD; ++k) acc.x[k] = fmaf(ds, x.x[k], acc.x[k]);
+      }
     }
   }
-  wr_rotate<D>(ix, c, acc, lane, -1.f);
-  wr_store<T, D>(dq + row * D, acc, lane);
+  gr_rotate<D>(ix, c, acc, g, -1.f);
+  if (active) gr_store<T, D>(dq + row * D, acc, g);
 }
 
+// dk, dv of key j: gathered over its own neighbourhood (the 3x3x3 relation is symmetric, so
+// no scatter/atomics) plus 1/|S| of its block's summary gradients; 8 lanes per key row.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __restrict__ v,
                                                  const T* __restrict__ gate,
@@ -425,58 +509,62 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
                                                  const float* __restrict__ lse_loc, float scale,
                                                  int64_t rows, BwdWork w, T* __restrict__ dk,
                                                  T* __restrict__ dv) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
+  const int g = threadIdx.x & 7;
+  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x >> 3) + (threadIdx.x >> 3);
+  const bool active = row0 < rows;
+  const int64_t row = active ? row0 : 0;
   const int64_t bh = row / ix.n, j = row % ix.n;
   const int64_t rowbase = bh * ix.n;
   const Coord c = decode(ix.coord[j]);
-  WarpRow<D> kr, vj, ak, av, x, d;
-  wr_load<T, D>(static_cast<const T*>(w.kr) + row * D, kr, lane);
-  wr_load<T, D>(v + row * D, vj, lane);
+  const T* qr = static_cast<const T*>(w.qr);
+  const T* kr = static_cast<const T*>(w.kr);
+  GRow<D> kj, vj, ak, av, x, d;
+  gr_load<T, D>(kr + row * D, kj, g);
+  gr_load<T, D>(v + row * D, vj, g);
 #pragma unroll
-  for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
-  // j is a neighbour of query i exactly when i is a neighbour of j
+  for (int k = 0; k < GRow<D>::KD; ++k) ak.x[k] = av.x[k] = 0.f;
   for (int o = 0; o < kNbr; ++o) {
     const int i = ix.nbr[j * kNbr + o];
-    if (i < 0) continue;
-    const int64_t ri = rowbase + i;
-    wr_load<T, D>(static_cast<const T*>(w.qr) + ri * D, x, lane);
-    wr_load<T, D>(dO + ri * D, d, lane);
-    const float g = 1.f / (1.f + expf(-to_f(gate[ri])));
-    const float p = expf(wr_dot<D>(x, kr) * scale - lse_loc[ri]);
-    const float ds = p * (g * wr_dot<D>(d, vj) - w.Dl[ri]) * scale;
+    const int64_t ri = rowbase + (i >= 0 ? i : 0);
+    gr_load<T, D>(qr + ri * D, x, g);
+    gr_load<T, D>(dO + ri * D, d, g);
+    const float gt = 1.f / (1.f + expf(-to_f(gate[ri])));
+    const float sd = gr_dot<D>(x, kj), dp = gr_dot<D>(d, vj);
+    const float p = i >= 0 ? expf(sd * scale - lse_loc[ri]) : 0.f;
+    const float ds = p * (gt * dp - w.Dl[ri]) * scale;
 #pragma unroll
-    for (int t = 0; t < WarpRow<D>::KT; ++t) {
-      ak.x[t] = fmaf(ds, x.x[t], ak.x[t]);
-      av.x[t] = fmaf(p * g, d.x[t], av.x[t]);
+    for (int k = 0; k < GRow<D>::KD; ++k) {
+      ak.x[k] = fmaf(ds, x.x[k], ak.x[k]);
+      av.x[k] = fmaf(p * gt, d.x[k], av.x[k]);
     }
   }
-  // un-pool: 1/|S| of the block summary's gradient
+  // un-pool: 1/|S| of the block summary's gradient (per-query-range partials summed in range
+  // order)
   const int b = ix.block_of[j];
   const float inv = 1.f / (float)ix.count[b];
-  // the summary gradients may come in per-query-range partials: summed in range order
   const int64_t part = (int64_t)(rows / ix.n) * ix.m * D;
-  WarpRow<D> sk, sv;
+  GRow<D> sk, sv;
 #pragma unroll
-  for (int t = 0; t < WarpRow<D>::KT; ++t) sk.x[t] = sv.x[t] = 0.f;
+  for (int k = 0; k < GRow<D>::KD; ++k) sk.x[k] = sv.x[k] = 0.f;
   for (int sp = 0; sp < w.nsplit; ++sp) {
-    wr_load_f<D>(w.dks + sp * part + (bh * ix.m + b) * D, x, lane);
-    wr_load_f<D>(w.dvs + sp * part + (bh * ix.m + b) * D, d, lane);
+    gr_load<float, D>(w.dks + sp * part + (bh * ix.m + b) * D, x, g);
+    gr_load<float, D>(w.dvs + sp * part + (bh * ix.m + b) * D, d, g);
 #pragma unroll
-    for (int t = 0; t < WarpRow<D>::KT; ++t) {
-      sk.x[t] += x.x[t];
-      sv.x[t] += d.x[t];
+    for (int k = 0; k < GRow<D>::KD; ++k) {
+      sk.x[k] += x.x[k];
+      sv.x[k] += d.x[k];
     }
   }
 #pragma unroll
-  for (int t = 0; t < WarpRow<D>::KT; ++t) {
-    ak.x[t] = fmaf(sk.x[t], inv, ak.x[t]);
-    av.x[t] = fmaf(sv.x[t], inv, av.x[t]);
+  for (int k = 0; k < GRow<D>::KD; ++k) {
+    ak.x[k] = fmaf(sk.x[k], inv, ak.x[k]);
+    av.x[k] = fmaf(sv.x[k], inv, av.x[k]);
   }
-  wr_rotate<D>(ix, c, ak, lane, -1.f);
-  wr_store<T, D>(dk + row * D, ak, lane);
-  wr_store<T, D>(dv + row * D, av, lane);
+  gr_rotate<D>(ix, c, ak, g, -1.f);
+  if (active) {
+    gr_store<T, D>(dk + row * D, ak, g);
+    gr_store<T, D>(dv + row * D, av, g);
+  }
 }
 
 // ------------------------------------------------------------------------------ launchers
@@ -517,10 +605,11 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
                                          excl, bh, w);
     count_launch();
   }
-  k_bwd_dq<T, D><<<rb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
+  const unsigned gb = (unsigned)((rows + 15) / 16);  // 16 rows (8 lanes each) per block
+  k_bwd_dq<T, D><<<gb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
                                      static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
                                      scale, excl, rows, w, static_cast<T*>(dq));
-  k_bwd_dkv<T, D><<<rb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, w,
+  k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, w,
                                       static_cast<T*>(dk), static_cast<T*>(dv));
   count_launch(2);
   return cudaGetLastError();
