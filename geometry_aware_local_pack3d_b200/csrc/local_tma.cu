@@ -10,14 +10,15 @@
 // walk bricks with a grid stride, two CTAs per SM. Per brick:
 //   * one 3D TMA box load brings the memory slots of the brick's 10x6x6 halo from the inverse
 //     map (x start rounded down to a 16-byte boundary: box 12x6x10 int32);
-//   * TMA row gathers (tile::gather4, 4 rows of 64 columns each, 128-byte swizzle) bring the
-//     128 q rows (rows outside the grid are requested past the end of the tensor and arrive as
-//     zeros), and two warps rotate the q tile in shared memory (axial RoPE by the brick
-//     coordinates);
-//   * the same two warps fetch, per halo z-slice, the 36 rotated key rows and value rows
-//     (padded to 48 with zero rows) with one cp.async per 16-byte piece, straight into the
-//     128-byte-swizzle layout (measured on B200: scattered 192-byte rows arrive about 1.7x
-//     faster this way than through gather4, whose per-operation cost caps it);
+//   * two producer warps fetch, per halo z-slice, the 36 rotated key rows and value rows
+//     (padded to 48 with zero rows) with one cp.async per 16-byte piece (rows off the grid are
+//     zero-filled), straight into the no-swizzle core-matrix layout (measured on B200:
+//     scattered 192-byte rows arrive about 1.7x faster this way than through TMA row gathers,
+//     whose per-operation cost caps them);
+//   * the q tile is double-buffered: while brick t runs, the box warp fetches the 128 q rows of
+//     the CTA's next brick (cp.async, zero-filled off the grid) and rotates them in place (axial
+//     RoPE by the brick coordinates), so the MMA warp starts a brick as soon as the previous
+//     one's last PV has been issued.
 // Chunk s = halo z-slice s (s = 0..9). Row r = 32 w + 16 dz + 4 y + x holds brick position
 // (2w + dz, y, x), so warp w needs exactly slices 2w .. 2w+3 and chunk s is owned by warps
 // max(0, (s-2)/2) .. min(3, s/2). Per chunk:
@@ -45,7 +46,7 @@ constexpr int kChunks = BZ + 2;        // halo z-slices
 constexpr int kSliceKeys = HY * HX;    // 36
 constexpr int kNK = 48;                // chunk rows (MMA N of QK, K of PV)
 constexpr int kStages = 3;
-constexpr int kThreads = 256;          // softmax 0-3, TMA 4, k/v fetch + q rotation 5-6, MMA 7
+constexpr int kThreads = 256;          // softmax 0-3, box + q 4, k/v fetch 5-6, MMA 7
 constexpr int kRot = 64;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kOCol = 128;
@@ -56,31 +57,42 @@ constexpr int kBoxPitch = 3072;
 
 __device__ __forceinline__ uint32_t s_col(int b) { return b ? 64u : 0u; }
 
+// Shared memory. Operands use the no-swizzle core-matrix layout: the 16-byte piece (row r,
+// column chunk c) of the q tile sits at c * kQCol + (r / 8) * 128 + (r % 8) * 16 and that of a
+// k or v chunk at c * kChunkCol + (row / 8) * 128 + (row % 8) * 16. Each column-chunk stride
+// carries 16 bytes of padding, so consecutive pieces of one row -- the order in which they are
+// read from global memory -- fall on distinct shared-memory banks.
 template <int D> struct Smem {
-  static constexpr int CBN = (D + 63) / 64;  // 64-column blocks of a row (2 for 96, 1 for 48)
-  static constexpr int kQBlk = 128 * 128;    // one column block of the q tile
-  static constexpr int kCBlk = kNK * 128;    // one column block of a k or v chunk
-  static constexpr int kStage = CBN * kCBlk;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + CBN * kQBlk;
-  static constexpr int kV = kK + kStages * kStage;
-  static constexpr int kBox = kV + kStages * kStage;  // [2] slot boxes
-  static constexpr int kRope = kBox + 2 * kBoxPitch;  // [16][d/6] (cos, sin) of the q tile
+  static constexpr int KC = D / 8;                 // 16-byte pieces of a row
+  static constexpr int kQCol = 128 * 16 + 16;      // one 16-byte column of the q tile
+  static constexpr int kQBuf = KC * kQCol;         // one q tile
+  static constexpr int kChunkCol = kNK * 16 + 16;  // one 16-byte column of a 48-row k or v chunk
+  static constexpr int kStage = KC * kChunkCol;
+  static constexpr int kQ = 0;                         // [2] q tiles
+  static constexpr int kK = kQ + 2 * kQBuf;            // [kStages] key chunks
+  static constexpr int kV = kK + kStages * kStage;     // [kStages] value chunks
+  static constexpr int kBox = kV + kStages * kStage;   // [2] slot boxes (TMA: 128-byte aligned)
+  static constexpr int kRope = kBox + 2 * kBoxPitch;   // [16][d/6] (cos, sin) of a q tile
   static constexpr int kBar = kRope + 16 * (D / 6) * 8;
   static constexpr int kBytes = kBar + 512;
+  static_assert(kBox % 128 == 0, "box alignment");
+  __device__ static int q_off(int r, int c) { return c * kQCol + (r >> 3) * 128 + (r & 7) * 16; }
 };
 
 enum {
-  B_QLOAD = 0, B_QFULL = 1, B_QEMPTY = 2, B_KVFULL = 3, B_KVEMPTY = 6, B_BOX = 9, B_BOXFREE = 11,
-  B_SFULL = 13,  // [warp][buffer]
-  B_PFULL = 21,  // [warp][buffer]
-  B_PVALL = 29, B_EPI = 30,  // B_EPI: [warp]
-  B_DRAIN = 34, B_COUNT = 35
+  B_QFULL = 0, B_QEMPTY = 2,  // [q buffer]
+  B_KVFULL = 4, B_KVEMPTY = 7, B_BOX = 10, B_BOXFREE = 12,
+  B_SFULL = 14,  // [warp][buffer]
+  B_PFULL = 22,  // [warp][buffer]
+  B_PVALL = 30, B_EPI = 31,  // B_EPI: [warp]
+  B_DRAIN = 35, B_COUNT = 36
 };
+
 static_assert(8 * B_COUNT + 16 <= 512, "barrier area");
 
 struct Params {
   pack3d_index ix;
+  const __nv_bfloat16* q;      // [B, H, N, d]
   const __nv_bfloat16* k_rot;  // rotated keys [B, H, N, d]
   const __nv_bfloat16* v;
   __nv_bfloat16* o_loc;
@@ -89,7 +101,6 @@ struct Params {
   int nbz, nby, nbx;
   int box_tma;        // slot boxes by TMA (else plain loads)
   int64_t tiles;      // batch * heads * bricks
-  int64_t rows;       // batch * heads * N: first row index past the gathered tensors
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -132,6 +143,23 @@ struct Abort {
     if ((ti) < 4) P3D_TRACE_C((ti) * 400 + (off));         \
   } while (0)
 
+#ifdef P3D_TRACE_ENABLED
+// global-timer stamp of each CTA's first 32 brick starts (MMA warp), tracing builds only
+static __device__ unsigned long long g_brick_t[512 * 32];
+#define BRICK_T(ti)                                                                       \
+  do {                                                                                    \
+    if ((ti) < 32 && blockIdx.x < 512) {                                                  \
+      unsigned long long t_;                                                              \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
+      g_brick_t[blockIdx.x * 32 + (ti)] = t_;                                             \
+    }                                                                                     \
+  } while (0)
+#else
+#define BRICK_T(ti) \
+  do {              \
+  } while (0)
+#endif
+
 // first and last softmax warp owning halo slice s
 __device__ __forceinline__ int owner_lo(int s) { return max(0, (s - 2) >> 1); }
 __device__ __forceinline__ int owner_hi(int s) { return min(3, s >> 1); }
@@ -140,12 +168,10 @@ __device__ __forceinline__ int owner_hi(int s) { return min(3, s >> 1); }
 
 template <int D>
 __global__ void __launch_bounds__(lg::kThreads, 2)
-    k_local_tma(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mg,
-                const lg::Params P) {
+    k_local_tma(const __grid_constant__ CUtensorMap mg, const lg::Params P) {
   using namespace lg;
   using S = Smem<D>;
-  constexpr int CBN = S::CBN;
-  constexpr int KC = D / 8;  // 16-byte pieces of a q row
+  constexpr int KC = S::KC;
   constexpr int DA = D / 3;
   constexpr int PR = D / 6;  // rotation pairs per axis
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -169,9 +195,10 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
   };
 
   if (tid == 0) {
-    tc::mbar_init(&bars[B_QLOAD], 1);
-    tc::mbar_init(&bars[B_QFULL], kRot);
-    tc::mbar_init(&bars[B_QEMPTY], 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars[B_QFULL + i], 32);  // the box warp
+      tc::mbar_init(&bars[B_QEMPTY + i], 1);
+    }
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bars[B_KVFULL + i], kRot);
       tc::mbar_init(&bars[B_KVEMPTY + i], 1);
@@ -190,18 +217,14 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
     abort_flag[0] = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
-    tc::tma_prefetch_desc(&mq);
-    if (P.box_tma) tc::tma_prefetch_desc(&mg);
-  }
+  if (warp == 4 && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
   // the padding rows 36..47 of every k/v stage are never written by the producers: zero them
   // once (the MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
-  for (int i = tid; i < kStages * 2 * CBN * (kNK - kSliceKeys) * 8; i += kThreads) {
-    const int piece = i & 7, row = kSliceKeys + (i >> 3) % (kNK - kSliceKeys);
-    const int blk = (i >> 3) / (kNK - kSliceKeys);  // stage * 2 * CBN + tensor * CBN + cb
-    const int st = blk / (2 * CBN), ten = (blk / CBN) & 1, cb = blk % CBN;
-    *reinterpret_cast<uint4*>(smem + (ten ? S::kV : S::kK) + st * S::kStage + cb * S::kCBlk +
-                              (row >> 3) * 1024 + (row & 7) * 128 + piece * 16) =
+  for (int i = tid; i < kStages * 2 * KC * (kNK - kSliceKeys); i += kThreads) {
+    const int row = kSliceKeys + i % (kNK - kSliceKeys), c = (i / (kNK - kSliceKeys)) % KC;
+    const int blk = i / ((kNK - kSliceKeys) * KC);  // stage * 2 + tensor
+    *reinterpret_cast<uint4*>(smem + ((blk & 1) ? S::kV : S::kK) + (blk >> 1) * S::kStage +
+                              c * S::kChunkCol + (row >> 3) * 128 + (row & 7) * 16) =
         make_uint4(0u, 0u, 0u, 0u);
   }
   tc::fence_proxy_async_smem();
@@ -281,7 +304,9 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * P.scale_log2;
         const float m_new = fmaxf(m_run, cmax);
         const bool need = m_new > m_run + kRescaleLog2;
-        if (i > 0 && __any_sync(0xffffffffu, need)) {
+        // a row that has met no neighbour yet holds O = 0 and needs no rescaling
+        const bool rescale = need && m_run != -INFINITY;
+        if (i > 0 && __any_sync(0xffffffffu, rescale)) {
           // O rows hold earlier chunks at the old max: rescale once the previous PV is done
           // (PVALL phase gs - 1 is the only incomplete or just-completed phase here)
           if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVALL], (gs - 1) & 1))) {
@@ -289,7 +314,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
             break;
           }
           tc::tc_fence_after();
-          const float f = need ? ex2(m_run - m_new) : 1.f;
+          const float f = rescale ? ex2(m_run - m_new) : 1.f;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t o[16];
@@ -357,12 +382,17 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
       }
     }
   } else if (warp == 4) {
-    // --------------------------------------------------------- TMA: slot boxes and q rows
+    // --------------------------------------------------------- slot boxes and q tiles
+    // Per brick: the slot box (3D TMA), then the brick's 128 q rows (one cp.async per 16-byte
+    // piece, rows off the grid zero-filled), rotated in place by the lane that copied them. The
+    // box and q buffers are double-buffered, so this runs one brick ahead of the MMAs.
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity));
     };
+    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope);  // [16][PR]
+    constexpr int QN = 128 * KC / 32;  // q pieces per lane, row-contiguous order
     int ti = 0;
-    uint32_t q_loads = 0, box_loads[2] = {0u, 0u};  // copies issued, for the exit
+    uint32_t box_loads[2] = {0u, 0u};  // copies issued, for the exit
     for (int64_t t = blockIdx.x; t < P.tiles; t += gridDim.x, ++ti) {
       int64_t bh;
       int z0, y0, x0;
@@ -387,45 +417,78 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars[B_BOX + bb]);
       }
+      // rotation table of this brick: rows z0..z0+7, y0..y0+3, x0..x0+3 (the previous brick's
+      // rotation, its only reader, is complete)
+      for (int i = lane; i < 16 * PR; i += 32) {
+        const int idx = i / PR, pp = i % PR;
+        int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : x0 + idx - 12);
+        cv = min(cv, P.ix.rope_rows - 1);
+        rope_q[i] = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp);
+      }
+      // the q buffer was last read by the QK MMAs of brick ti - 2
       if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
+      if (ti >= 2 && !wwait(&bars[B_QEMPTY + bb], ((ti >> 1) - 1) & 1)) break;
       if (lane == 0) GTR(ti, 2);
-      // q rows: lane l gathers rows 4l .. 4l+3 of the tile (rows off the grid: past the end)
-      if (ti >= 1 && !wwait(&bars[B_QEMPTY], (ti - 1) & 1)) break;
-      int qr[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = 4 * lane + j, rw = r >> 5, rl = r & 31;
+      uint8_t* qd = smem + S::kQ + bb * S::kQBuf;
+      // q row r of a brick holds position (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4)
+#pragma unroll 4
+      for (int j = 0; j < QN; ++j) {
+        const int i = lane + 32 * j, r = i / KC, c = i % KC;
+        const int rw = r >> 5, rl = r & 31;
         const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = rl & 3;
         const int slot = in_grid(z0 + z, y0 + y, x0 + x)
                              ? box[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
                              : -1;
-        qr[j] = slot >= 0 ? (int)(bh * N + slot) : (int)P.rows;
+        const int64_t src = (bh * N + (slot >= 0 ? slot : 0)) * D + c * 8;
+        tc::cp_async16(qd + S::q_off(r, c), P.q + src, slot >= 0);
       }
-      if (lane == 0) tc::mbar_expect_tx(&bars[B_QLOAD], 128 * 128 * CBN);
-      ++q_loads;
-      __syncwarp();
-#pragma unroll
-      for (int cb = 0; cb < CBN; ++cb)
-        tc::tma_gather4(smem + S::kQ + cb * S::kQBlk + lane * 512, &mq, cb * 64, qr[0], qr[1],
-                        qr[2], qr[3], &bars[B_QLOAD]);
+      tc::cp_async_commit();
+      tc::cp_async_wait_group<0>();
+      __syncwarp();  // rope_q complete
       if (lane == 0) GTR(ti, 3);
+      // rotate the pieces this lane copied (rows off the grid are zero and stay zero)
+#pragma unroll 2
+      for (int j = 0; j < QN; ++j) {
+        const int i = lane + 32 * j, r = i / KC, c = i % KC;
+        uint4* ptr = reinterpret_cast<uint4*>(qd + S::q_off(r, c));
+        const int rw = r >> 5, rl = r & 31;
+        const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
+        const int idx =
+            axis == 0 ? 2 * rw + (rl >> 4) : (axis == 1 ? 8 + ((rl >> 2) & 3) : 12 + (rl & 3));
+        const float4* cs4 = reinterpret_cast<const float4*>(rope_q + idx * PR + p0);
+        const float4 ca = cs4[0], cbv = cs4[1];
+        const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
+        const uint4 xv = *ptr;
+        const uint32_t xin[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t xo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float e0 = __uint_as_float(xin[k] << 16);
+          const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+          xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
+                                e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
+        }
+        *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[B_QFULL + bb]);
+      __syncwarp();  // rope_q is rewritten for the next brick
+      if (lane == 0) GTR(ti, 4);
     }
+    tc::cp_async_wait_all();
     // nothing may still be landing in shared memory when the CTA exits (bounded waits)
-    if (lane == 0) {
-      if (q_loads) tc::mbar_wait(&bars[B_QLOAD], (q_loads - 1) & 1, 100000000LL);
+    if (lane == 0)
       for (int b2 = 0; b2 < 2; ++b2)
         if (box_loads[b2])
           tc::mbar_wait(&bars[B_BOX + b2], (box_loads[b2] - 1) & 1, 100000000LL);
-    }
   } else if (warp < 7) {
-    // --------------------------------------------------------- k/v rows and q rotation (64 thr)
-    // Halo slice s of rotated keys and values: 36 rows x d, one cp.async per 16-byte piece
-    // (rows off the grid are zero-filled), written at its 128-byte-swizzle position; each
-    // thread publishes a slice once its own copies have landed. Between slices 1 and 2 the same
-    // threads rotate the brick's q tile, which the TMA warp has gathered meanwhile.
+    // --------------------------------------------------------- k/v rows (64 threads)
+    // Halo slice s of rotated keys and values: 36 rows x d, one cp.async per 16-byte piece in
+    // row-contiguous order (rows off the grid are zero-filled). Each thread's copies arrive on
+    // the stage's barrier by themselves when they land, so the warps run ahead as far as the
+    // free stages allow.
     const int pt = tid - 160;
-    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope);  // [16][PR]
-    volatile int* pflag = abort_flag + 1;                          // [2], used alternately
+    volatile int* pflag = abort_flag + 1;  // [2], used alternately
     int nwait = 0;
     // one bounded wait by one thread, its verdict shared with all 64 (named barrier 2)
     auto pwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -434,8 +497,8 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
       asm volatile("bar.sync 2, 64;" ::: "memory");
       return *f != 0;
     };
-    // this thread's pieces, the same in every slice: (row, 16-byte column) and the swizzled
-    // shared-memory offset, packed as off16 | row << 16 | col << 24
+    // this thread's pieces, the same in every slice: shared-memory offset / 16, row and column,
+    // packed as off16 | row << 16 | col << 24
     constexpr int KPIECES = kSliceKeys * KC;
     constexpr int NP = (KPIECES + kRot - 1) / kRot;
     uint32_t pc[NP];
@@ -443,8 +506,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
     for (int j = 0; j < NP; ++j) {
       const int p = pt + j * kRot;
       const int row = p / KC, c = p % KC;
-      const int off = (c >> 3) * S::kCBlk + (row >> 3) * 1024 + (row & 7) * 128 +
-                      (((c & 7) ^ (row & 7)) << 4);
+      const int off = c * S::kChunkCol + (row >> 3) * 128 + (row & 7) * 16;
       pc[j] = p < KPIECES ? ((uint32_t)(off >> 4) | ((uint32_t)row << 16) | ((uint32_t)c << 24))
                           : 0xffffffffu;
     }
@@ -485,63 +547,13 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
           tc::cp_async16(kd + off, kg + src, slot >= 0);
           tc::cp_async16(vd + off, vg + src, slot >= 0);
         }
-        tc::cp_async_commit();
+        tc::cp_async_arrive_noinc(&bars[B_KVFULL + st]);
         if (pt == 0) GTR(ti, 11 + s * 2);
-        if (s > 0) {
-          // the previous slice has landed: publish it to the MMA warp
-          tc::cp_async_wait_group<1>();
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(&bars[B_KVFULL + (gs - 1) % kStages]);
-        }
-        if (s == 1) {
-          // q tile of this brick: rotation rows z0..z0+7, y0..y0+3, x0..x0+3 (rows off the
-          // grid are zero and any finite rotation keeps them zero)
-          for (int i = pt; i < 16 * PR; i += kRot) {
-            const int idx = i / PR, pp = i % PR;
-            int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : x0 + idx - 12);
-            cv = min(cv, P.ix.rope_rows - 1);
-            rope_q[i] = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp);
-          }
-          if (!pwait(&bars[B_QLOAD], ti & 1)) { ok = false; break; }
-          if (pt == 0) GTR(ti, 40);
-#pragma unroll 4
-          for (int i = pt; i < 128 * KC; i += kRot) {
-            const int c = i >> 7, r = i & 127;
-            const int cb = c >> 3, cc = c & 7;
-            uint4* ptr = reinterpret_cast<uint4*>(smem + S::kQ + cb * S::kQBlk + (r >> 3) * 1024 +
-                                                  (r & 7) * 128 + ((cc ^ (r & 7)) << 4));
-            const int rw = r >> 5, rl = r & 31;
-            const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
-            const int idx =
-                axis == 0 ? 2 * rw + (rl >> 4) : (axis == 1 ? 8 + ((rl >> 2) & 3) : 12 + (rl & 3));
-            const float4* cs4 = reinterpret_cast<const float4*>(rope_q + idx * PR + p0);
-            const float4 ca = cs4[0], cbv = cs4[1];
-            const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
-            const uint4 x = *ptr;
-            const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
-            uint32_t xo[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float e0 = __uint_as_float(xin[k] << 16);
-              const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
-              xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
-                                    e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
-            }
-            *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
-          }
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(&bars[B_QFULL]);
-          if (pt == 0) GTR(ti, 41);
-        }
       }
       if (!ok) break;
-      // the brick's last slice, and this warp's reads of the slot box, are done
-      tc::cp_async_wait_group<0>();
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[B_KVFULL + (gs - 1) % kStages]);
+      // this warp's reads of the slot box are done
       __syncwarp();
       if ((pt & 31) == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
-      asm volatile("bar.sync 2, 64;" ::: "memory");  // rope_q is rewritten for the next brick
     }
     tc::cp_async_wait_all();  // nothing may still be landing in shared memory at exit
   } else {
@@ -552,42 +564,48 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
     const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
     const uint32_t id_qk = tc::idesc_bf16_f32(128, kNK, false, false);
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
-    const uint64_t qd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kQ), 16, 1024);
-    const uint64_t kd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kK), 16, 1024);
-    const uint64_t vd0 = tc::smem_desc_sw128(tc::smem_u32(smem + S::kV), S::kCBlk, 1024);
+    // no-swizzle descriptors: q and k K-major (lbo = column-chunk stride, sbo = 8 rows), v
+    // MN-major (lbo = 8 key rows, sbo = column-chunk stride)
+    const uint64_t qd0 = tc::smem_desc(tc::smem_u32(smem + S::kQ), S::kQCol, 128);
+    const uint64_t kd0 = tc::smem_desc(tc::smem_u32(smem + S::kK), S::kChunkCol, 128);
+    const uint64_t vd0 = tc::smem_desc(tc::smem_u32(smem + S::kV), 128, S::kChunkCol);
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity, false));
     };
     int ti = 0;
     uint32_t gs = 0;
     bool ok = true;
-    // QK(s) of chunk counter gc into S buffer s % 2; the buffer was freed by the PVALL wait
-    // of chunk gc - 2
-    auto issue_qk = [&](int s, uint32_t gc) -> bool {
+    // QK(s) of chunk counter gc into S buffer s % 2 (q tile descriptor qd, buffer qb); the S
+    // buffer was freed by the PVALL wait of chunk gc - 2
+    auto issue_qk = [&](int s, uint32_t gc, uint64_t qd, int qb) -> bool {
       const int st = gc % kStages;
       if (!wwait(&bars[B_KVFULL + st], (gc / kStages) & 1)) return false;
+      // the chunk arrived through cp.async (generic proxy); the MMAs read it through the async
+      // proxy
+      tc::fence_proxy_async_smem();
       tc::tc_fence_after();
       const uint64_t b0 = kd0 + (uint64_t)((st * S::kStage) >> 4);
       const uint32_t dt = tb + s_col(s & 1);
       if (tc::elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks & 3) * 32;  // 16 columns = 32 bytes into the swizzled row
-          tc::mma_ss(dt, qd0 + (uint64_t)(((ks >> 2) * S::kQBlk + off) >> 4),
-                     b0 + (uint64_t)(((ks >> 2) * S::kCBlk + off) >> 4), id_qk, ks > 0);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)  // 16 columns = two column chunks
+          tc::mma_ss(dt, qd + (uint64_t)(ks * ((2 * S::kQCol) >> 4)),
+                     b0 + (uint64_t)(ks * ((2 * S::kChunkCol) >> 4)), id_qk, ks > 0);
         for (int w = owner_lo(s); w <= owner_hi(s); ++w)
           tc::tc_commit(&bars[B_SFULL + 2 * w + (s & 1)]);
-        if (s == kChunks - 1) tc::tc_commit(&bars[B_QEMPTY]);  // q tile free for the next brick
+        if (s == kChunks - 1) tc::tc_commit(&bars[B_QEMPTY + qb]);  // q buffer free again
       }
       __syncwarp();
       return true;
     };
     for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
-      if (!wwait(&bars[B_QFULL], ti & 1)) break;
+      const int qb = ti & 1;
+      const uint64_t qd = qd0 + (uint64_t)((qb * S::kQBuf) >> 4);
+      if (!wwait(&bars[B_QFULL + qb], (ti >> 1) & 1)) break;
       if (lane == 0) GTR(ti, 50);
+      if (lane == 0) BRICK_T(ti);
       tc::tc_fence_after();
-      ok = issue_qk(0, gs) && issue_qk(1, gs + 1);
+      ok = issue_qk(0, gs, qd, qb) && issue_qk(1, gs + 1, qd, qb);
       if (lane == 0) GTR(ti, 51);
       for (int s = 0; s < kChunks && ok; ++s, ++gs) {
         const int st = gs % kStages, b = s & 1;
@@ -605,7 +623,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         if (tc::elect_one()) {
 #pragma unroll
           for (int ks = 0; ks < kNK / 16; ++ks)
-            tc::mma_ts_masked(tb + kOCol, tb + s_col(b) + ks * 8, v0 + (uint64_t)(ks * (2048 >> 4)),
+            tc::mma_ts_masked(tb + kOCol, tb + s_col(b) + ks * 8, v0 + (uint64_t)(ks * (256 >> 4)),
                               id_pv, 1u, m0, m1, m2, m3);
           tc::tc_commit(&bars[B_KVEMPTY + st]);
           tc::tc_commit(&bars[B_PVALL]);
@@ -616,7 +634,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         // PV(s) complete: S buffer s % 2 may take QK(s + 2); observed for every chunk, in order
         if (!wwait(&bars[B_PVALL], gs & 1)) { ok = false; break; }
         if (lane == 0) GTR(ti, 62 + s * 4);
-        if (s + 2 < kChunks) ok = issue_qk(s + 2, gs + 2);
+        if (s + 2 < kChunks) ok = issue_qk(s + 2, gs + 2, qd, qb);
         if (lane == 0) GTR(ti, 63 + s * 4);
       }
     }
@@ -658,20 +676,18 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;
   p.tiles = bh * p.nbz * p.nby * p.nbx;
-  p.rows = bh * ix.n;
   if (p.tiles <= 0) return cudaSuccess;
-  if (p.rows >= 0x7fffffffLL) return cudaErrorInvalidValue;  // gather row indices are int32
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_rot = static_cast<const __nv_bfloat16*>(k_rot);
   p.v = static_cast<const __nv_bfloat16*>(v);
-  CUtensorMap mq, mg;
+  CUtensorMap mg;
   memset(&mg, 0, sizeof(mg));
-  if (!encode_gather_rows_bf16(&mq, q, p.rows, D)) return cudaErrorInvalidValue;
   p.box_tma = encode_grid_i32(&mg, ix.inv, ix.geom.gz, ix.geom.gy, ix.geom.gx, kBoxX, kBoxY, kBoxZ)
                   ? 1
                   : 0;
   const int64_t cap = 2 * (int64_t)sm_count();
   const unsigned grid = (unsigned)(p.tiles < cap ? p.tiles : cap);
-  k_local_tma<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mq, mg, p);
+  k_local_tma<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mg, p);
   count_launch();
   return cudaGetLastError();
 }
@@ -690,6 +706,10 @@ cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void
 extern "C" int p3d_trace_read_t(unsigned long long* host) {
   cudaDeviceSynchronize();
   return (int)cudaMemcpyFromSymbol(host, p3d::g_trace, sizeof(unsigned long long) * 4096);
+}
+extern "C" int p3d_trace_read_b(unsigned long long* host) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(host, p3d::lg::g_brick_t, sizeof(unsigned long long) * 512 * 32);
 }
 extern "C" int p3d_trace_clear_t() {
   static unsigned long long z[4096];
