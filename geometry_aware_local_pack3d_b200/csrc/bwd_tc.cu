@@ -342,7 +342,8 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
     }
     if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
     __syncwarp();
-    tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL);
+    if (!tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL))
+      set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -631,7 +632,8 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
     }
     if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
     __syncwarp();
-    tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL);
+    if (!tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL))
+      set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
   }
   tc::tc_fence_before();
   __syncthreads();

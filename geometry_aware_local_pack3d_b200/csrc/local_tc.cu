@@ -576,7 +576,8 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
     // every MMA this warp issued has completed once this commit arrives (bounded wait)
     if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
     __syncwarp();
-    tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL);
+    if (!tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL))
+      set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
   }
 
   tc::tc_fence_before();

@@ -6,30 +6,36 @@
 // never by adjacency in memory; paper summary §3.5: streamed online softmax, no gathered
 // neighbour tensor in memory.
 //
-// Work unit: one 8x4x4 (z, y, x) brick of 128 queries of one (batch, head); persistent CTAs
-// walk bricks with a grid stride, two CTAs per SM. Per brick:
-//   * one 3D TMA box load brings the memory slots of the brick's 10x6x6 halo from the inverse
-//     map (x start rounded down to a 16-byte boundary: box 12x6x10 int32);
-//   * two producer warps fetch, per halo z-slice, the 36 rotated key rows and value rows
-//     (padded to 48 with zero rows) with one cp.async per 16-byte piece (rows off the grid are
-//     zero-filled), straight into the no-swizzle core-matrix layout (measured on B200:
-//     scattered 192-byte rows arrive about 1.7x faster this way than through TMA row gathers,
-//     whose per-operation cost caps them);
-//   * the q tile is double-buffered: while brick t runs, the box warp fetches the 128 q rows of
-//     the CTA's next brick (cp.async, zero-filled off the grid) and rotates them in place (axial
-//     RoPE by the brick coordinates), so the MMA warp starts a brick as soon as the previous
-//     one's last PV has been issued.
-// Chunk s = halo z-slice s (s = 0..9). Row r = 32 w + 16 dz + 4 y + x holds brick position
-// (2w + dz, y, x), so warp w needs exactly slices 2w .. 2w+3 and chunk s is owned by warps
-// max(0, (s-2)/2) .. min(3, s/2). Per chunk:
-//   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2 at column 0 or 64)
+// Work unit: one 8x4x8 (z, y, x) brick of one (batch, head), split into two 128-query tiles
+// (x0..x0+3 and x0+4..x0+7); one persistent CTA per SM. The two
+// tiles share one stream of halo z-slices (10 slices of 6x10 = 60 keys), so a key row is
+// fetched once for 256 queries. Units are handed out by a device-wide counter (status word 2
+// of the index; the last CTA to finish puts it back to zero), so SMs that run slower take
+// fewer units. Per unit:
+//   * one 3D TMA box load brings the memory slots of the unit's 10x6x10 halo from the inverse
+//     map (x start rounded down to a 16-byte boundary: box 16x6x10 int32);
+//   * four producer warps fetch, per halo z-slice, the 60 rotated key rows and value rows with
+//     one cp.async per 16-byte piece (rows off the grid are zero-filled) into the no-swizzle
+//     core-matrix layout, four stages deep; each thread's copies arrive on the stage's barrier
+//     by themselves when they land;
+//   * the q tiles are double-buffered: two q warps (one per tile) fetch the next unit's 128 q
+//     rows each (cp.async) and rotate them in place (axial RoPE by the brick coordinates)
+//     while the current unit runs.
+// Slice key order: x columns 0-3, then 4-5, then 6-9 of the halo (each block y-major), so tile
+// 0's neighbours (halo x 0..5) are slice rows 0..35 and tile 1's (halo x 4..9) rows 24..59:
+// each tile works on a 48-row window (rows 24 t .. 24 t + 47; rows 60..71 are zero padding).
+// Per tile, chunk s = halo z-slice s. Row r = 32 w + 16 dz + 4 y + x holds brick position
+// (2w + dz, y, x), so warp w of a tile needs exactly slices 2w .. 2w+3 and chunk s is owned by
+// warps max(0, (s-2)/2) .. min(3, s/2). Per tile and chunk:
+//   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2)
 //   owners: 3x3x3 mask, online softmax, P = exp2(s - m) as bf16 over the buffer's first 24
-//   columns;  O += P_s v_s  (TS MMA, N = d, TMEM columns 128..) with the rows of the other
-//   warps disabled through the MMA's output-lane mask, so non-owners never touch chunk s.
-// QK runs two chunks ahead of PV, so S_{s+2} is ready when the owners finish chunk s + 1. Each
-// warp zeroes its O rows when it starts a brick; its epilogue runs after the PV of its last
-// chunk. Every query sits at the same row and every neighbour at the same column whatever the
-// packing, so a coordinate-carrying repack permutes the output bit for bit.
+//   columns;  O += P_s v_s  (TS MMA, N = d) with the rows of the other warps disabled through
+//   the MMA's output-lane mask, so non-owners never touch chunk s.
+// Each tile has its own MMA warp; QK runs two chunks ahead of PV, so S_{s+2} is ready when the
+// owners finish chunk s + 1. Each softmax warp zeroes its O rows when it starts a unit; its
+// epilogue runs after the PV of its last chunk. Every query sits at the same row and every
+// neighbour at the same column whatever the packing, so a coordinate-carrying repack permutes
+// the output bit for bit.
 #include <math.h>
 
 #include "common.cuh"
@@ -40,55 +46,69 @@
 namespace p3d {
 
 namespace lg {
-constexpr int BZ = 8, BY = 4, BX = 4;  // brick
+constexpr int BZ = 8, BY = 4, BX = 8;  // unit; two tiles of 8 x 4 x 4
+constexpr int kTiles = 2;
 constexpr int HY = BY + 2, HX = BX + 2;
 constexpr int kChunks = BZ + 2;        // halo z-slices
-constexpr int kSliceKeys = HY * HX;    // 36
-constexpr int kNK = 48;                // chunk rows (MMA N of QK, K of PV)
-constexpr int kStages = 3;
-constexpr int kThreads = 256;          // softmax 0-3, box + q 4, k/v fetch 5-6, MMA 7
-constexpr int kRot = 64;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kSliceKeys = HY * HX;    // 60
+constexpr int kNK = 48;                // tile window (MMA N of QK, K of PV)
+constexpr int kWin = 24;               // first slice row of tile 1's window
+constexpr int kRows = kWin + kNK;      // 72 rows per stage
+constexpr int kStages = 4;
+// warps: softmax 0-7 (tile = warp / 4), q 8-9 (tile = warp - 8; warp 8 also loads the slot
+// boxes), k/v producers 10-13, MMA 14-15 (tile = warp - 14)
+constexpr int kThreads = 512;
+constexpr int W_Q = 8, W_PROD = 10, W_MMA = 14;
+constexpr int kProd = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTileCols = 256;  // per tile: S buffers at 0 / 64, O at 128
 constexpr uint32_t kOCol = 128;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kBoxX = 12, kBoxY = 6, kBoxZ = 10;  // slot box: x from x0 - 4
+constexpr int kBoxX = 16, kBoxY = 6, kBoxZ = 10;  // slot box: x from x0 - 4
 constexpr int kBoxBytes = kBoxX * kBoxY * kBoxZ * 4;
-constexpr int kBoxPitch = 3072;
+constexpr int kBoxPitch = 4096;  // box, then the unit index (int64) at kBoxBytes
 
 __device__ __forceinline__ uint32_t s_col(int b) { return b ? 64u : 0u; }
 
+// slice row of halo position (hy, hx): halo x 0-3, then 4-5, then 6-9, each block y-major
+__host__ __device__ constexpr int slice_row(int hy, int hx) {
+  return hx < 4 ? hy * 4 + hx : (hx < 6 ? 24 + hy * 2 + (hx - 4) : 36 + hy * 4 + (hx - 6));
+}
+
 // Shared memory. Operands use the no-swizzle core-matrix layout: the 16-byte piece (row r,
-// column chunk c) of the q tile sits at c * kQCol + (r / 8) * 128 + (r % 8) * 16 and that of a
-// k or v chunk at c * kChunkCol + (row / 8) * 128 + (row % 8) * 16. Each column-chunk stride
+// column chunk c) of a q tile sits at c * kQCol + (r / 8) * 128 + (r % 8) * 16 and that of a
+// k or v stage at c * kChunkCol + (row / 8) * 128 + (row % 8) * 16. Each column-chunk stride
 // carries 16 bytes of padding, so consecutive pieces of one row -- the order in which they are
 // read from global memory -- fall on distinct shared-memory banks.
 template <int D> struct Smem {
   static constexpr int KC = D / 8;                 // 16-byte pieces of a row
-  static constexpr int kQCol = 128 * 16 + 16;      // one 16-byte column of the q tile
+  static constexpr int PR = D / 6;                 // rotation pairs per axis
+  static constexpr int kQCol = 128 * 16 + 16;      // one 16-byte column of a q tile
   static constexpr int kQBuf = KC * kQCol;         // one q tile
-  static constexpr int kChunkCol = kNK * 16 + 16;  // one 16-byte column of a 48-row k or v chunk
+  static constexpr int kChunkCol = kRows * 16 + 16;
   static constexpr int kStage = KC * kChunkCol;
-  static constexpr int kQ = 0;                         // [2] q tiles
-  static constexpr int kK = kQ + 2 * kQBuf;            // [kStages] key chunks
-  static constexpr int kV = kK + kStages * kStage;     // [kStages] value chunks
-  static constexpr int kBox = kV + kStages * kStage;   // [2] slot boxes (TMA: 128-byte aligned)
-  static constexpr int kRope = kBox + 2 * kBoxPitch;   // [16][d/6] (cos, sin) of a q tile
-  static constexpr int kBar = kRope + 16 * (D / 6) * 8;
-  static constexpr int kBytes = kBar + 512;
+  static constexpr int kQ = 0;                            // [2 buffers][2 tiles] q tiles
+  static constexpr int kK = kQ + 4 * kQBuf;               // [kStages] key chunks
+  static constexpr int kV = kK + kStages * kStage;        // [kStages] value chunks
+  static constexpr int kBox = kV + kStages * kStage;      // [2] slot boxes (TMA: 128-aligned)
+  static constexpr int kRope = kBox + 2 * kBoxPitch;      // [2 tiles][16][PR] (cos, sin)
+  static constexpr int kBar = kRope + 2 * 16 * PR * 8;
+  static constexpr int kBytes = kBar + 1024;
   static_assert(kBox % 128 == 0, "box alignment");
   __device__ static int q_off(int r, int c) { return c * kQCol + (r >> 3) * 128 + (r & 7) * 16; }
 };
 
 enum {
-  B_QFULL = 0, B_QEMPTY = 2,  // [q buffer]
-  B_KVFULL = 4, B_KVEMPTY = 7, B_BOX = 10, B_BOXFREE = 12,
-  B_SFULL = 14,  // [warp][buffer]
-  B_PFULL = 22,  // [warp][buffer]
-  B_PVALL = 30, B_EPI = 31,  // B_EPI: [warp]
-  B_DRAIN = 35, B_COUNT = 36
+  B_QFULL = 0, B_QEMPTY = 4,  // [q buffer][tile]
+  B_KVFULL = 8, B_KVEMPTY = 12, B_BOX = 16, B_BOXFREE = 18,
+  B_SFULL = 20,  // [tile][warp][buffer]
+  B_PFULL = 36,  // [tile][warp][buffer]
+  B_PVALL = 52,  // [tile]
+  B_EPI = 54,    // [tile][warp]
+  B_DRAIN = 62,  // [tile]
+  B_COUNT = 64
 };
-
-static_assert(8 * B_COUNT + 16 <= 512, "barrier area");
+static_assert(8 * B_COUNT + 16 <= 1024, "barrier area");
 
 struct Params {
   pack3d_index ix;
@@ -100,7 +120,7 @@ struct Params {
   float scale_log2;
   int nbz, nby, nbx;
   int box_tma;        // slot boxes by TMA (else plain loads)
-  int64_t tiles;      // batch * heads * bricks
+  int64_t units;      // batch * heads * units per field
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -137,20 +157,20 @@ struct Abort {
   }
 };
 
-// clock64 trace slots of the first four bricks a CTA processes (tracing builds only)
+// clock64 trace slots of the first four units a CTA processes (tracing builds only)
 #define GTR(ti, off)                                       \
   do {                                                     \
     if ((ti) < 4) P3D_TRACE_C((ti) * 400 + (off));         \
   } while (0)
 
 #ifdef P3D_TRACE_ENABLED
-// global-timer stamp of each CTA's first 32 brick starts (MMA warp), tracing builds only
+// global-timer stamp of each CTA's first 32 unit starts (MMA warp of tile 0), tracing builds
 static __device__ unsigned long long g_brick_t[512 * 32];
 #define BRICK_T(ti)                                                                       \
   do {                                                                                    \
     if ((ti) < 32 && blockIdx.x < 512) {                                                  \
       unsigned long long t_;                                                              \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                              \
       g_brick_t[blockIdx.x * 32 + (ti)] = t_;                                             \
     }                                                                                     \
   } while (0)
@@ -167,13 +187,13 @@ __device__ __forceinline__ int owner_hi(int s) { return min(3, s >> 1); }
 }  // namespace lg
 
 template <int D>
-__global__ void __launch_bounds__(lg::kThreads, 2)
+__global__ void __launch_bounds__(lg::kThreads, 1)
     k_local_tma(const __grid_constant__ CUtensorMap mg, const lg::Params P) {
   using namespace lg;
   using S = Smem<D>;
   constexpr int KC = S::KC;
   constexpr int DA = D / 3;
-  constexpr int PR = D / 6;  // rotation pairs per axis
+  constexpr int PR = S::PR;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
@@ -182,10 +202,10 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
   Abort ab{abort_flag, P.ix.status};
   const pack3d_geom& g = P.ix.geom;
   const int64_t N = P.ix.n;
-  const int64_t bricks = (int64_t)P.nbz * P.nby * P.nbx;
-  auto origin = [&](int64_t t, int64_t& bh, int& z0, int& y0, int& x0) {
-    bh = t / bricks;
-    const int64_t br = t % bricks;
+  const int64_t per_field = (int64_t)P.nbz * P.nby * P.nbx;
+  auto origin = [&](int64_t u, int64_t& bh, int& z0, int& y0, int& x0) {
+    bh = u / per_field;
+    const int64_t br = u % per_field;
     z0 = (int)(br / (P.nby * P.nbx)) * BZ;
     y0 = (int)((br / P.nbx) % P.nby) * BY;
     x0 = (int)(br % P.nbx) * BX;
@@ -193,68 +213,77 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
   auto in_grid = [&](int z, int y, int x) {
     return z >= 0 && z < g.gz && y >= 0 && y < g.gy && x >= 0 && x < g.gx;
   };
+  // unit published with slot box bb (-1: no more units), valid once B_BOX[bb] has completed
+  auto unit_of = [&](int bb) -> int64_t {
+    return *reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes);
+  };
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bars[B_QFULL + i], 32);  // the box warp
+    for (int i = 0; i < 4; ++i) {
+      tc::mbar_init(&bars[B_QFULL + i], 32);  // the tile's q warp
       tc::mbar_init(&bars[B_QEMPTY + i], 1);
     }
     for (int i = 0; i < kStages; ++i) {
-      tc::mbar_init(&bars[B_KVFULL + i], kRot);
-      tc::mbar_init(&bars[B_KVEMPTY + i], 1);
+      tc::mbar_init(&bars[B_KVFULL + i], kProd);
+      tc::mbar_init(&bars[B_KVEMPTY + i], kTiles);  // one commit per tile's MMA warp
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bars[B_BOX + i], 1);
-      tc::mbar_init(&bars[B_BOXFREE + i], 4 + 2);  // softmax warps + producer warps
+      tc::mbar_init(&bars[B_BOXFREE + i], 8 + 2 + 4);  // softmax, q and producer warps
     }
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 16; ++i) {
       tc::mbar_init(&bars[B_SFULL + i], 1);
       tc::mbar_init(&bars[B_PFULL + i], 32);
     }
-    tc::mbar_init(&bars[B_PVALL], 1);
-    for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[B_EPI + i], 1);
-    tc::mbar_init(&bars[B_DRAIN], 1);
+    for (int i = 0; i < kTiles; ++i) {
+      tc::mbar_init(&bars[B_PVALL + i], 1);
+      tc::mbar_init(&bars[B_DRAIN + i], 1);
+    }
+    for (int i = 0; i < 8; ++i) tc::mbar_init(&bars[B_EPI + i], 1);
     abort_flag[0] = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
-  // the padding rows 36..47 of every k/v stage are never written by the producers: zero them
-  // once (the MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
-  for (int i = tid; i < kStages * 2 * KC * (kNK - kSliceKeys); i += kThreads) {
-    const int row = kSliceKeys + i % (kNK - kSliceKeys), c = (i / (kNK - kSliceKeys)) % KC;
-    const int blk = i / ((kNK - kSliceKeys) * KC);  // stage * 2 + tensor
+  if (warp == W_Q && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
+  // rows 60..71 of every k/v stage are never written by the producers: zero them once (tile 1's
+  // MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
+  for (int i = tid; i < kStages * 2 * KC * (kRows - kSliceKeys); i += kThreads) {
+    const int row = kSliceKeys + i % (kRows - kSliceKeys), c = (i / (kRows - kSliceKeys)) % KC;
+    const int blk = i / ((kRows - kSliceKeys) * KC);  // stage * 2 + tensor
     *reinterpret_cast<uint4*>(smem + ((blk & 1) ? S::kV : S::kK) + (blk >> 1) * S::kStage +
                               c * S::kChunkCol + (row >> 3) * 128 + (row & 7) * 16) =
         make_uint4(0u, 0u, 0u, 0u);
   }
   tc::fence_proxy_async_smem();
-  if (warp == 7) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == W_MMA) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp < 4) {
-    // --------------------------------------------------------- softmax + epilogue (row = tid)
-    const int w = warp;
+  if (warp < 8) {
+    // --------------------------------------------------------- softmax + epilogue (row = lane)
+    const int tile = warp >> 2, w = warp & 3;
     int ti = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
-      // lane-derived values from opaque copies each brick (keeps the score row in registers)
+    for (; ok; ++ti) {
+      // lane-derived values from opaque copies each unit (keeps the score row in registers)
       int ln = lane;
       uint32_t tl = tbase;
       asm volatile("" : "+r"(ln), "+r"(tl));
-      tl += (uint32_t)(w * 32) << 16;
-      const int dz = ln >> 4, qy = (ln >> 2) & 3, qx = ln & 3;
-      int64_t bh;
-      int z0, y0, x0;
-      origin(t, bh, z0, y0, x0);
+      tl += ((uint32_t)(w * 32) << 16) + tile * kTileCols;
+      const int dz = ln >> 4, qy = (ln >> 2) & 3, qx = 4 * tile + (ln & 3);
       const int bb = ti & 1;
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + bb], (ti >> 1) & 1))) break;
+      const int64_t u = unit_of(bb);
+      if (u < 0) break;
+      int64_t bh;
+      int z0, y0, x0;
+      origin(u, bh, z0, y0, x0);
       const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
       const int cz = z0 + 2 * w + dz, cy = y0 + qy, cx = x0 + qx;
       const bool valid = cz < g.gz && cy < g.gy && cx < g.gx;
-      // neighbour bits of the warp's four slices: bit hy * 6 + hx of slice 2w + i
+      // neighbour bits of the warp's four slices: bit slice_row(hy, hx) - 24 tile of slice
+      // 2w + i
       uint64_t nb[4] = {0ull, 0ull, 0ull, 0ull};
       if (valid) {
 #pragma unroll
@@ -264,29 +293,31 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
           const int hz = 2 * w + dz + 1 + ddz;  // halo slice
           if (!in_grid(cz + ddz, cy + ddy, cx + ddx)) continue;
           if (box[(hz * kBoxY + hy) * kBoxX + hx + 3] < 0) continue;
-          const uint64_t bit = 1ull << (hy * HX + hx);
+          const uint64_t bit = 1ull << (slice_row(hy, hx) - kWin * tile);
           nb[1 + ddz] |= dz == 0 ? bit : 0ull;  // slice index i = dz + 1 + ddz
           nb[2 + ddz] |= dz == 1 ? bit : 0ull;
         }
       }
-      // this warp's O rows start at zero (the previous brick's epilogue has read them)
+      // this warp's O rows start at zero (the previous unit's epilogue has read them)
       {
         const uint32_t zr[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 16) tc::tmem_st16(tl + kOCol + c0, zr);
       }
+      uint64_t* sfull = &bars[B_SFULL + (tile * 4 + w) * 2];
+      uint64_t* pfull = &bars[B_PFULL + (tile * 4 + w) * 2];
       float m_run = -INFINITY, l_run = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int s = 2 * w + i, b = i & 1;
         const uint32_t gs = (uint32_t)ti * kChunks + s;
-        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL + 2 * w + b], (i >> 1) & 1))) {
+        if (!__all_sync(0xffffffffu, ab.wait(&sfull[b], (i >> 1) & 1))) {
           ok = false;
           break;
         }
-        if (ln == 0) GTR(ti, 110 + w * 20 + i * 4);
+        if (ln == 0 && tile == 0) GTR(ti, 110 + w * 20 + i * 4);
         tc::tc_fence_after();
-        // the chunk's 48 scores; entries off the 3x3x3 cube become -inf
+        // the chunk's 48 window scores; entries off the 3x3x3 cube become -inf
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         uint32_t r[kNK];
 #pragma unroll
@@ -309,7 +340,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         if (i > 0 && __any_sync(0xffffffffu, rescale)) {
           // O rows hold earlier chunks at the old max: rescale once the previous PV is done
           // (PVALL phase gs - 1 is the only incomplete or just-completed phase here)
-          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVALL], (gs - 1) & 1))) {
+          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_PVALL + tile], (gs - 1) & 1))) {
             ok = false;
             break;
           }
@@ -348,12 +379,12 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         lg::tmem_st8(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[8]>(&p[16]));
         tc::tmem_wait_st();
         tc::tc_fence_before();
-        tc::mbar_arrive(&bars[B_PFULL + 2 * w + b]);
-        if (ln == 0) GTR(ti, 111 + w * 20 + i * 4);
+        tc::mbar_arrive(&pfull[b]);
+        if (ln == 0 && tile == 0) GTR(ti, 111 + w * 20 + i * 4);
       }
       if (!ok) break;
       // epilogue after the PV of the warp's last slice: o_loc = O / l, lse_loc
-      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_EPI + w], ti & 1))) break;
+      if (!__all_sync(0xffffffffu, ab.wait(&bars[B_EPI + tile * 4 + w], ti & 1))) break;
       tc::tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       uint32_t ow[D / 2];
@@ -371,7 +402,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
           valid ? box[((2 * w + dz + 1) * kBoxY + qy + 1) * kBoxX + qx + 4] : -1;
       __syncwarp();
       if (ln == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
-      if (ln == 0) GTR(ti, 190 + w);
+      if (ln == 0 && tile == 0) GTR(ti, 190 + w);
       if (slot >= 0) {
         uint4* dst = reinterpret_cast<uint4*>(P.o_loc + (bh * N + slot) * D);
 #pragma unroll
@@ -381,71 +412,102 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
           P.lse_loc[bh * N + slot] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
-  } else if (warp == 4) {
+  } else if (warp < W_PROD) {
     // --------------------------------------------------------- slot boxes and q tiles
-    // Per brick: the slot box (3D TMA), then the brick's 128 q rows (one cp.async per 16-byte
-    // piece, rows off the grid zero-filled), rotated in place by the lane that copied them. The
-    // box and q buffers are double-buffered, so this runs one brick ahead of the MMAs.
+    // q warp `tile` (warp 8 also loads the slot box): per unit, the tile's 128 q rows (one
+    // cp.async per 16-byte piece, rows off the grid zero-filled), rotated in place by the lane
+    // that copied them. Box and q buffers are double-buffered, so this runs one unit ahead of
+    // the MMAs.
+    const int tile = warp - W_Q;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity));
     };
-    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope);  // [16][PR]
+    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope) + tile * 16 * PR;  // [16][PR]
     constexpr int QN = 128 * KC / 32;  // q pieces per lane, row-contiguous order
     int ti = 0;
-    uint32_t box_loads[2] = {0u, 0u};  // copies issued, for the exit
-    for (int64_t t = blockIdx.x; t < P.tiles; t += gridDim.x, ++ti) {
-      int64_t bh;
-      int z0, y0, x0;
-      origin(t, bh, z0, y0, x0);
+    uint32_t box_phases[2] = {0u, 0u};  // phases started on B_BOX (lane 0), for the exit
+    for (;; ++ti) {
       const int bb = ti & 1;
       int32_t* box = reinterpret_cast<int32_t*>(smem + S::kBox + bb * kBoxPitch);
-      if (lane == 0) GTR(ti, 0);
-      if (ti >= 2 && !wwait(&bars[B_BOXFREE + bb], ((ti >> 1) - 1) & 1)) break;
-      if (lane == 0) GTR(ti, 1);
-      ++box_loads[bb];
-      if (P.box_tma) {
-        if (lane == 0) {
-          tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
-          tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
+      int64_t u, bh;
+      int z0, y0, x0;
+      if (tile == 0) {
+        // the next unit from the device-wide counter, published with its slot box
+        if (lane == 0) GTR(ti, 0);
+        if (ti >= 2 && !wwait(&bars[B_BOXFREE + bb], ((ti >> 1) - 1) & 1)) break;
+        if (lane == 0) GTR(ti, 1);
+        unsigned int nu = 0;
+        if (lane == 0) nu = atomicAdd(reinterpret_cast<unsigned int*>(P.ix.status + 2), 1u);
+        u = (int64_t)__shfl_sync(0xffffffffu, nu, 0);
+        if (u >= P.units) {
+          if (lane == 0) {
+            *reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes) = -1;
+            ++box_phases[bb];
+            tc::mbar_arrive(&bars[B_BOX + bb]);
+          }
+          break;
+        }
+        origin(u, bh, z0, y0, x0);
+        if (lane == 0)
+          *reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes) = u;
+        __syncwarp();
+        if (P.box_tma) {
+          if (lane == 0) {
+            ++box_phases[bb];
+            tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
+            tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
+          }
+        } else {
+          for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
+            const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
+            const int z = z0 - 1 + bz, y = y0 - 1 + by, x = x0 - 4 + bx;
+            box[i] = in_grid(z, y, x) ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : 0;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            ++box_phases[bb];
+            tc::mbar_arrive(&bars[B_BOX + bb]);
+          }
         }
       } else {
-        for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
-          const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
-          const int z = z0 - 1 + bz, y = y0 - 1 + by, x = x0 - 4 + bx;
-          box[i] = in_grid(z, y, x) ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : 0;
-        }
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars[B_BOX + bb]);
+        if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
+        u = unit_of(bb);
+        if (u < 0) break;
+        origin(u, bh, z0, y0, x0);
       }
-      // rotation table of this brick: rows z0..z0+7, y0..y0+3, x0..x0+3 (the previous brick's
+      const int xt = x0 + 4 * tile;  // the tile's first x
+      // rotation table of the tile: rows z0..z0+7, y0..y0+3, xt..xt+3 (the previous unit's
       // rotation, its only reader, is complete)
       for (int i = lane; i < 16 * PR; i += 32) {
         const int idx = i / PR, pp = i % PR;
-        int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : x0 + idx - 12);
+        int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : xt + idx - 12);
         cv = min(cv, P.ix.rope_rows - 1);
         rope_q[i] = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp);
       }
-      // the q buffer was last read by the QK MMAs of brick ti - 2
+      // the q buffer was last read by the tile's QK MMAs of unit ti - 2
       if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
-      if (ti >= 2 && !wwait(&bars[B_QEMPTY + bb], ((ti >> 1) - 1) & 1)) break;
-      if (lane == 0) GTR(ti, 2);
-      uint8_t* qd = smem + S::kQ + bb * S::kQBuf;
-      // q row r of a brick holds position (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4)
+      if (ti >= 2 && !wwait(&bars[B_QEMPTY + bb * 2 + tile], ((ti >> 1) - 1) & 1)) break;
+      if (lane == 0 && tile == 0) GTR(ti, 2);
+      uint8_t* qd = smem + S::kQ + (bb * 2 + tile) * S::kQBuf;
+      const __nv_bfloat16* qg = P.q + bh * N * D;
+      // q row r of a tile holds position (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4)
 #pragma unroll 4
       for (int j = 0; j < QN; ++j) {
         const int i = lane + 32 * j, r = i / KC, c = i % KC;
         const int rw = r >> 5, rl = r & 31;
-        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = rl & 3;
+        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = 4 * tile + (rl & 3);
         const int slot = in_grid(z0 + z, y0 + y, x0 + x)
                              ? box[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
                              : -1;
-        const int64_t src = (bh * N + (slot >= 0 ? slot : 0)) * D + c * 8;
-        tc::cp_async16(qd + S::q_off(r, c), P.q + src, slot >= 0);
+        tc::cp_async16(qd + S::q_off(r, c), qg + (int64_t)(slot >= 0 ? slot : 0) * D + c * 8,
+                       slot >= 0);
       }
       tc::cp_async_commit();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);  // this warp's box reads are done
       tc::cp_async_wait_group<0>();
       __syncwarp();  // rope_q complete
-      if (lane == 0) GTR(ti, 3);
+      if (lane == 0 && tile == 0) GTR(ti, 3);
       // rotate the pieces this lane copied (rows off the grid are zero and stay zero)
 #pragma unroll 2
       for (int j = 0; j < QN; ++j) {
@@ -471,43 +533,49 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
       }
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[B_QFULL + bb]);
-      __syncwarp();  // rope_q is rewritten for the next brick
-      if (lane == 0) GTR(ti, 4);
+      tc::mbar_arrive(&bars[B_QFULL + bb * 2 + tile]);
+      __syncwarp();  // rope_q is rewritten for the next unit
+      if (lane == 0 && tile == 0) GTR(ti, 4);
     }
     tc::cp_async_wait_all();
-    // nothing may still be landing in shared memory when the CTA exits (bounded waits)
-    if (lane == 0)
+    // nothing may still be landing in shared memory when the CTA exits: wait for the latest
+    // phase of each box barrier (phases complete in order; bounded waits; lane 0's counts)
+    if (tile == 0 && lane == 0)
       for (int b2 = 0; b2 < 2; ++b2)
-        if (box_loads[b2])
-          tc::mbar_wait(&bars[B_BOX + b2], (box_loads[b2] - 1) & 1, 100000000LL);
-  } else if (warp < 7) {
-    // --------------------------------------------------------- k/v rows (64 threads)
-    // Halo slice s of rotated keys and values: 36 rows x d, one cp.async per 16-byte piece in
+        if (box_phases[b2])
+          if (!tc::mbar_wait(&bars[B_BOX + b2], (box_phases[b2] - 1) & 1, 100000000LL))
+            set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
+  } else if (warp < W_MMA) {
+    // --------------------------------------------------------- k/v rows (128 threads)
+    // Halo slice s of rotated keys and values: 60 rows x d, one cp.async per 16-byte piece in
     // row-contiguous order (rows off the grid are zero-filled). Each thread's copies arrive on
     // the stage's barrier by themselves when they land, so the warps run ahead as far as the
     // free stages allow.
-    const int pt = tid - 160;
+    const int pt = tid - W_PROD * 32;
     volatile int* pflag = abort_flag + 1;  // [2], used alternately
     int nwait = 0;
-    // one bounded wait by one thread, its verdict shared with all 64 (named barrier 2)
+    // one bounded wait by one thread, its verdict shared with all 128 (named barrier 2)
     auto pwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       volatile int* f = pflag + (nwait++ & 1);
       if (pt == 0) *f = ab.wait(bar, parity) ? 1 : 0;
-      asm volatile("bar.sync 2, 64;" ::: "memory");
+      asm volatile("bar.sync 2, 128;" ::: "memory");
       return *f != 0;
     };
-    // this thread's pieces, the same in every slice: shared-memory offset / 16, row and column,
-    // packed as off16 | row << 16 | col << 24
+    // this thread's pieces, the same in every slice: shared-memory offset / 16, halo (hy, hx)
+    // and column, packed as off16 | hy << 16 | hx << 20 | col << 24 (pieces in halo order,
+    // y-major over x; the stage row is slice_row(hy, hx))
     constexpr int KPIECES = kSliceKeys * KC;
-    constexpr int NP = (KPIECES + kRot - 1) / kRot;
+    constexpr int NP = (KPIECES + kProd - 1) / kProd;
     uint32_t pc[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-      const int p = pt + j * kRot;
-      const int row = p / KC, c = p % KC;
+      const int p = pt + j * kProd;
+      const int key = p / KC, c = p % KC;
+      const int hy = key / HX, hx = key % HX;
+      const int row = slice_row(hy, hx);
       const int off = c * S::kChunkCol + (row >> 3) * 128 + (row & 7) * 16;
-      pc[j] = p < KPIECES ? ((uint32_t)(off >> 4) | ((uint32_t)row << 16) | ((uint32_t)c << 24))
+      pc[j] = p < KPIECES ? ((uint32_t)(off >> 4) | ((uint32_t)hy << 16) | ((uint32_t)hx << 20) |
+                             ((uint32_t)c << 24))
                           : 0xffffffffu;
     }
     const __nv_bfloat16* kg = P.k_rot;
@@ -515,13 +583,15 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
     int ti = 0;
     uint32_t gs = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
-      int64_t bh;
-      int z0, y0, x0;
-      origin(t, bh, z0, y0, x0);
+    for (; ok; ++ti) {
       const int bb = ti & 1;
       const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
       if (!pwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
+      const int64_t u = unit_of(bb);
+      if (u < 0) break;
+      int64_t bh;
+      int z0, y0, x0;
+      origin(u, bh, z0, y0, x0);
       const int64_t rbase = bh * N;
       for (int s = 0; s < kChunks; ++s, ++gs) {
         const int st = gs % kStages;
@@ -536,8 +606,7 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
           if (pc[j] == 0xffffffffu) continue;
-          const int row = (pc[j] >> 16) & 0xff, c = pc[j] >> 24;
-          const int hy = row / HX, hx = row % HX;
+          const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf, c = pc[j] >> 24;
           const int y = y0 - 1 + hy, x = x0 - 1 + hx;
           int slot = -1;
           if (zin && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
@@ -557,27 +626,34 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
     }
     tc::cp_async_wait_all();  // nothing may still be landing in shared memory at exit
   } else {
-    // --------------------------------------------------------- MMA issuer (warp 7)
-    // Per slice s: PV(s) for its owners (other rows disabled), then -- once PV(s) has
-    // completed, which frees S buffer s % 2 -- QK(s + 2). The whole warp runs the schedule with
-    // warp-uniform values; one elected lane issues the MMAs and commits.
-    const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
+    // --------------------------------------------------------- MMA issuers (warps 14, 15)
+    // One warp per tile. Per slice s: PV(s) for its owners (other rows disabled), then -- once
+    // PV(s) has completed, which frees S buffer s % 2 -- QK(s + 2). The whole warp runs the
+    // schedule with warp-uniform values; one elected lane issues the MMAs and commits.
+    const int tile = warp - W_MMA;
+    const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0) + tile * kTileCols;
     const uint32_t id_qk = tc::idesc_bf16_f32(128, kNK, false, false);
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
     // no-swizzle descriptors: q and k K-major (lbo = column-chunk stride, sbo = 8 rows), v
-    // MN-major (lbo = 8 key rows, sbo = column-chunk stride)
+    // MN-major (lbo = 8 key rows, sbo = column-chunk stride); the tile's window starts at
+    // slice row 24 tile
     const uint64_t qd0 = tc::smem_desc(tc::smem_u32(smem + S::kQ), S::kQCol, 128);
-    const uint64_t kd0 = tc::smem_desc(tc::smem_u32(smem + S::kK), S::kChunkCol, 128);
-    const uint64_t vd0 = tc::smem_desc(tc::smem_u32(smem + S::kV), 128, S::kChunkCol);
+    const uint64_t kd0 =
+        tc::smem_desc(tc::smem_u32(smem + S::kK + (kWin * tile / 8) * 128), S::kChunkCol, 128);
+    const uint64_t vd0 =
+        tc::smem_desc(tc::smem_u32(smem + S::kV + (kWin * tile / 8) * 128), 128, S::kChunkCol);
+    uint64_t* sfull = &bars[B_SFULL + tile * 8];
+    uint64_t* pfull = &bars[B_PFULL + tile * 8];
+    uint64_t* pvall = &bars[B_PVALL + tile];
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity, false));
     };
     int ti = 0;
     uint32_t gs = 0;
     bool ok = true;
-    // QK(s) of chunk counter gc into S buffer s % 2 (q tile descriptor qd, buffer qb); the S
+    // QK(s) of chunk counter gc into S buffer s % 2 (q tile descriptor qd, q barrier qi); the S
     // buffer was freed by the PVALL wait of chunk gc - 2
-    auto issue_qk = [&](int s, uint32_t gc, uint64_t qd, int qb) -> bool {
+    auto issue_qk = [&](int s, uint32_t gc, uint64_t qd, int qi) -> bool {
       const int st = gc % kStages;
       if (!wwait(&bars[B_KVFULL + st], (gc / kStages) & 1)) return false;
       // the chunk arrived through cp.async (generic proxy); the MMAs read it through the async
@@ -591,29 +667,28 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         for (int ks = 0; ks < D / 16; ++ks)  // 16 columns = two column chunks
           tc::mma_ss(dt, qd + (uint64_t)(ks * ((2 * S::kQCol) >> 4)),
                      b0 + (uint64_t)(ks * ((2 * S::kChunkCol) >> 4)), id_qk, ks > 0);
-        for (int w = owner_lo(s); w <= owner_hi(s); ++w)
-          tc::tc_commit(&bars[B_SFULL + 2 * w + (s & 1)]);
-        if (s == kChunks - 1) tc::tc_commit(&bars[B_QEMPTY + qb]);  // q buffer free again
+        for (int w = owner_lo(s); w <= owner_hi(s); ++w) tc::tc_commit(&sfull[2 * w + (s & 1)]);
+        if (s == kChunks - 1) tc::tc_commit(&bars[B_QEMPTY + qi]);  // q tile free again
       }
       __syncwarp();
       return true;
     };
-    for (int64_t t = blockIdx.x; t < P.tiles && ok; t += gridDim.x, ++ti) {
-      const int qb = ti & 1;
-      const uint64_t qd = qd0 + (uint64_t)((qb * S::kQBuf) >> 4);
-      if (!wwait(&bars[B_QFULL + qb], (ti >> 1) & 1)) break;
-      if (lane == 0) GTR(ti, 50);
-      if (lane == 0) BRICK_T(ti);
+    for (; ok; ++ti) {
+      if (!wwait(&bars[B_BOX + (ti & 1)], (ti >> 1) & 1) || unit_of(ti & 1) < 0) break;
+      const int qi = (ti & 1) * 2 + tile;
+      const uint64_t qd = qd0 + (uint64_t)((qi * S::kQBuf) >> 4);
+      if (!wwait(&bars[B_QFULL + qi], (ti >> 1) & 1)) break;
+      if (lane == 0 && tile == 0) GTR(ti, 50);
+      if (lane == 0 && tile == 0) BRICK_T(ti);
       tc::tc_fence_after();
-      ok = issue_qk(0, gs, qd, qb) && issue_qk(1, gs + 1, qd, qb);
-      if (lane == 0) GTR(ti, 51);
+      ok = issue_qk(0, gs, qd, qi) && issue_qk(1, gs + 1, qd, qi);
+      if (lane == 0 && tile == 0) GTR(ti, 51);
       for (int s = 0; s < kChunks && ok; ++s, ++gs) {
         const int st = gs % kStages, b = s & 1;
         const int wlo = owner_lo(s), whi = owner_hi(s);
-        for (int w = wlo; w <= whi && ok; ++w)
-          ok = wwait(&bars[B_PFULL + 2 * w + b], ((s - 2 * w) >> 1) & 1);
+        for (int w = wlo; w <= whi && ok; ++w) ok = wwait(&pfull[2 * w + b], ((s - 2 * w) >> 1) & 1);
         if (!ok) break;
-        if (lane == 0) GTR(ti, 60 + s * 4);
+        if (lane == 0 && tile == 0) GTR(ti, 60 + s * 4);
         tc::tc_fence_after();
         const uint32_t m0 = (0 < wlo || 0 > whi) ? 0xffffffffu : 0u;
         const uint32_t m1 = (1 < wlo || 1 > whi) ? 0xffffffffu : 0u;
@@ -622,34 +697,44 @@ __global__ void __launch_bounds__(lg::kThreads, 2)
         const uint64_t v0 = vd0 + (uint64_t)((st * S::kStage) >> 4);
         if (tc::elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < kNK / 16; ++ks)
+          for (int ks = 0; ks < kNK / 16; ++ks)  // 16 key rows = two row groups
             tc::mma_ts_masked(tb + kOCol, tb + s_col(b) + ks * 8, v0 + (uint64_t)(ks * (256 >> 4)),
                               id_pv, 1u, m0, m1, m2, m3);
           tc::tc_commit(&bars[B_KVEMPTY + st]);
-          tc::tc_commit(&bars[B_PVALL]);
-          if ((s & 1) && s >= 3) tc::tc_commit(&bars[B_EPI + ((s - 3) >> 1)]);
+          tc::tc_commit(pvall);
+          if ((s & 1) && s >= 3) tc::tc_commit(&bars[B_EPI + tile * 4 + ((s - 3) >> 1)]);
         }
         __syncwarp();
-        if (lane == 0) GTR(ti, 61 + s * 4);
+        if (lane == 0 && tile == 0) GTR(ti, 61 + s * 4);
         // PV(s) complete: S buffer s % 2 may take QK(s + 2); observed for every chunk, in order
-        if (!wwait(&bars[B_PVALL], gs & 1)) { ok = false; break; }
-        if (lane == 0) GTR(ti, 62 + s * 4);
-        if (s + 2 < kChunks) ok = issue_qk(s + 2, gs + 2, qd, qb);
-        if (lane == 0) GTR(ti, 63 + s * 4);
+        if (!wwait(pvall, gs & 1)) { ok = false; break; }
+        if (lane == 0 && tile == 0) GTR(ti, 62 + s * 4);
+        if (s + 2 < kChunks) ok = issue_qk(s + 2, gs + 2, qd, qi);
+        if (lane == 0 && tile == 0) GTR(ti, 63 + s * 4);
       }
     }
     // every MMA this warp issued has completed once this commit arrives (bounded wait)
-    if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN]);
+    if (tc::elect_one()) tc::tc_commit(&bars[B_DRAIN + tile]);
     __syncwarp();
-    tc::mbar_wait(&bars[B_DRAIN], 0, 100000000LL);
+    if (!tc::mbar_wait(&bars[B_DRAIN + tile], 0, 100000000LL))
+      set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 7) {
+  if (warp == W_MMA) {
     __syncwarp();
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, kTmemCols);
+  }
+  if (tid == 0) {
+    // the last CTA out puts the unit counter (and this count) back to zero for the next call
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(P.ix.status + 2);
+    __threadfence();
+    if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
+      atomicExch(ctr, 0u);
+      atomicExch(ctr + 1, 0u);
+    }
   }
 }
 
@@ -661,9 +746,7 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(k_local_tma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<D>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(k_local_tma<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             100) != cudaSuccess)
+                             Smem<D>::kBytes) != cudaSuccess)
       return cudaErrorInvalidValue;
     attr = true;
   }
@@ -675,8 +758,9 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   p.nbz = (ix.geom.gz + BZ - 1) / BZ;
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;
-  p.tiles = bh * p.nbz * p.nby * p.nbx;
-  if (p.tiles <= 0) return cudaSuccess;
+  p.units = bh * p.nbz * p.nby * p.nbx;
+  if (p.units <= 0) return cudaSuccess;
+  if (!ix.status || p.units >= 0x7fffffffLL) return cudaErrorInvalidValue;  // unit counter
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_rot = static_cast<const __nv_bfloat16*>(k_rot);
   p.v = static_cast<const __nv_bfloat16*>(v);
@@ -685,8 +769,8 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   p.box_tma = encode_grid_i32(&mg, ix.inv, ix.geom.gz, ix.geom.gy, ix.geom.gx, kBoxX, kBoxY, kBoxZ)
                   ? 1
                   : 0;
-  const int64_t cap = 2 * (int64_t)sm_count();
-  const unsigned grid = (unsigned)(p.tiles < cap ? p.tiles : cap);
+  const int64_t cap = sm_count();
+  const unsigned grid = (unsigned)(p.units < cap ? p.units : cap);
   k_local_tma<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mg, p);
   count_launch();
   return cudaGetLastError();

@@ -96,7 +96,10 @@ typedef struct {
   int32_t* members;       /* device [M, v]   slot of the member at each canonical slot */
   int32_t* count;         /* device [M]      members present */
   float* rope;            /* device [rope_rows, rope_pairs, 2] (cos, sin) of c * theta_p */
-  int32_t* status;        /* device [4]      status words written by kernels */
+  int32_t* status;        /* device [4]      status words written by kernels: [0] first error;
+                             [2], [3] the work counter of the bf16 rotated-key local kernel
+                             (zero between calls; calls that use one index must therefore be
+                             ordered, e.g. on one stream) */
 } pack3d_index;
 
 /* Human-readable name of a status code (static string, never NULL). */
