@@ -378,23 +378,28 @@ def test_repacking_equivariance_is_exact_rotated_keys():
 
 
 @pytest.mark.parametrize("bh", [(1, 1), (3, 5), (40, 4)])
-def test_local_work_counter_returns_to_zero(bh):
+def test_forward_work_counter_returns_to_zero(bh):
     # the rotated-key local kernel takes its work units from a counter in status words 2 and 3
-    # of the index: after every call both are zero again, and a repeated call (units handed
-    # to other CTAs) gives the same output bit for bit; (40, 4) has more units than SMs
+    # of the index: after every call (and after the global call that follows) both are zero
+    # again, and a repeated call (units handed to other CTAs) gives the same output bit for
+    # bit; (40, 4) has more units than SMs
     m = p3d()
     B, H = bh
     w = small((8, 8, 16), (4, 4, 4), B, H, 96, "bf16", "random", qkv_std=96 ** -0.5)
     ix = gpu_index(w, 96)
-    q, k, v = (w[n].to(torch.bfloat16).cuda().contiguous() for n in "qkv")
-    _, _, k_rot = m.pack3d_summarize_rotated(ix, k, v)
+    q, k, v, a = (w[n].to(torch.bfloat16).cuda().contiguous() for n in "qkva")
+    ks, vs, k_rot = m.pack3d_summarize_rotated(ix, k, v)
     outs = []
     for _ in range(3):
         o_loc, _ = m.pack3d_attn_local(ix, q, k_rot, v, k_rotated=True)
         torch.cuda.synchronize()
         st = ix.table("status", (4,)).cpu()
         assert int(st[0]) == 0 and int(st[2]) == 0 and int(st[3]) == 0, st
-        outs.append(o_loc.clone())
+        o = m.pack3d_attn_global(ix, q, a, ks, vs, o_loc)
+        torch.cuda.synchronize()
+        st = ix.table("status", (4,)).cpu()
+        assert int(st[0]) == 0 and int(st[2]) == 0 and int(st[3]) == 0, st
+        outs.append(o.clone())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
