@@ -18,9 +18,11 @@
 //     one cp.async per 16-byte piece (rows off the grid are zero-filled) into the no-swizzle
 //     core-matrix layout, four stages deep; each thread's copies arrive on the stage's barrier
 //     by themselves when they land;
-//   * the q tiles are double-buffered: two q warps (one per tile) fetch the next unit's 128 q
-//     rows each (cp.async) and rotate them in place (axial RoPE by the brick coordinates)
-//     while the current unit runs.
+//   * the q tiles are double-buffered: softmax warps 0 and 1 of each tile, idle once their
+//     slices of a unit are done, load the next unit's q rows (64 rows each, one row per lane),
+//     rotate them in registers (axial RoPE by the row's coordinates) and store them into the
+//     tile's other q buffer, so the MMAs start a unit as soon as the previous one's last PV
+//     has been issued.
 // Slice key order: x columns 0-3, then 4-5, then 6-9 of the halo (each block y-major), so tile
 // 0's neighbours (halo x 0..5) are slice rows 0..35 and tile 1's (halo x 4..9) rows 24..59:
 // each tile works on a 48-row window (rows 24 t .. 24 t + 47; rows 60..71 are zero padding).
@@ -28,8 +30,9 @@
 // (2w + dz, y, x), so warp w of a tile needs exactly slices 2w .. 2w+3 and chunk s is owned by
 // warps max(0, (s-2)/2) .. min(3, s/2). Per tile and chunk:
 //   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2)
-//   owners: 3x3x3 mask, online softmax, P = exp2(s - m) as bf16 over the buffer's first 24
-//   columns;  O += P_s v_s  (TS MMA, N = d) with the rows of the other warps disabled through
+//   owners: 3x3x3 mask, online softmax over the window's first 36 columns (the only ones that
+//   can hold a neighbour of the tile), P = exp2(s - m) as bf16 over the buffer's first 24
+//   columns (P = 0 in window columns 36..47);  O += P_s v_s  (TS MMA, N = d) with the rows of the other warps disabled through
 //   the MMA's output-lane mask, so non-owners never touch chunk s.
 // Each tile has its own MMA warp; QK runs two chunks ahead of PV, so S_{s+2} is ready when the
 // owners finish chunk s + 1. Each softmax warp zeroes its O rows when it starts a unit; its
@@ -52,13 +55,14 @@ constexpr int HY = BY + 2, HX = BX + 2;
 constexpr int kChunks = BZ + 2;        // halo z-slices
 constexpr int kSliceKeys = HY * HX;    // 60
 constexpr int kNK = 48;                // tile window (MMA N of QK, K of PV)
+constexpr int kNV = 36;                // window columns that can hold a neighbour
 constexpr int kWin = 24;               // first slice row of tile 1's window
 constexpr int kRows = kWin + kNK;      // 72 rows per stage
 constexpr int kStages = 4;
-// warps: softmax 0-7 (tile = warp / 4), q 8-9 (tile = warp - 8; warp 8 also loads the slot
-// boxes), k/v producers 10-13, MMA 14-15 (tile = warp - 14)
+// warps: softmax 0-7 (tile = warp / 4; warps 0, 1, 4, 5 also prepare q tiles), slot boxes 8
+// (warp 9 idle), k/v producers 10-13, MMA 14-15 (tile = warp - 14)
 constexpr int kThreads = 512;
-constexpr int W_Q = 8, W_PROD = 10, W_MMA = 14;
+constexpr int W_BOX = 8, W_PROD = 10, W_MMA = 14;
 constexpr int kProd = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTileCols = 256;  // per tile: S buffers at 0 / 64, O at 128
@@ -82,7 +86,6 @@ __host__ __device__ constexpr int slice_row(int hy, int hx) {
 // read from global memory -- fall on distinct shared-memory banks.
 template <int D> struct Smem {
   static constexpr int KC = D / 8;                 // 16-byte pieces of a row
-  static constexpr int PR = D / 6;                 // rotation pairs per axis
   static constexpr int kQCol = 128 * 16 + 16;      // one 16-byte column of a q tile
   static constexpr int kQBuf = KC * kQCol;         // one q tile
   static constexpr int kChunkCol = kRows * 16 + 16;
@@ -91,8 +94,7 @@ template <int D> struct Smem {
   static constexpr int kK = kQ + 4 * kQBuf;               // [kStages] key chunks
   static constexpr int kV = kK + kStages * kStage;        // [kStages] value chunks
   static constexpr int kBox = kV + kStages * kStage;      // [2] slot boxes (TMA: 128-aligned)
-  static constexpr int kRope = kBox + 2 * kBoxPitch;      // [2 tiles][16][PR] (cos, sin)
-  static constexpr int kBar = kRope + 2 * 16 * PR * 8;
+  static constexpr int kBar = kBox + 2 * kBoxPitch;
   static constexpr int kBytes = kBar + 1024;
   static_assert(kBox % 128 == 0, "box alignment");
   __device__ static int q_off(int r, int c) { return c * kQCol + (r >> 3) * 128 + (r & 7) * 16; }
@@ -127,6 +129,12 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
@@ -193,7 +201,6 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
   using S = Smem<D>;
   constexpr int KC = S::KC;
   constexpr int DA = D / 3;
-  constexpr int PR = S::PR;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) {
-      tc::mbar_init(&bars[B_QFULL + i], 32);  // the tile's q warp
+      tc::mbar_init(&bars[B_QFULL + i], 64);  // softmax warps 0 and 1 of the tile
       tc::mbar_init(&bars[B_QEMPTY + i], 1);
     }
     for (int i = 0; i < kStages; ++i) {
@@ -229,7 +236,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bars[B_BOX + i], 1);
-      tc::mbar_init(&bars[B_BOXFREE + i], 8 + 2 + 4);  // softmax, q and producer warps
+      tc::mbar_init(&bars[B_BOXFREE + i], 8 + 4);  // softmax and producer warps
     }
     for (int i = 0; i < 16; ++i) {
       tc::mbar_init(&bars[B_SFULL + i], 1);
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     abort_flag[0] = 0;
     tc::fence_mbar_init();
   }
-  if (warp == W_Q && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
+  if (warp == W_BOX && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
   // rows 60..71 of every k/v stage are never written by the producers: zero them once (tile 1's
   // MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
   for (int i = tid; i < kStages * 2 * KC * (kRows - kSliceKeys); i += kThreads) {
@@ -263,6 +270,56 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
   if (warp < 8) {
     // --------------------------------------------------------- softmax + epilogue (row = lane)
     const int tile = warp >> 2, w = warp & 3;
+    // q tile of unit `un` (slot box nb) into q buffer qi: warp w (0 or 1) takes rows
+    // 64 w .. 64 w + 63, one row per lane and pass -- loaded, rotated in registers by the row's
+    // coordinates (axial RoPE) and stored in the operand layout -- then publishes its share
+    // (QFULL: 64 arrivals per tile). Row r of a tile holds brick position
+    // (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4); rows off the grid are zero.
+    auto prepare_q = [&](int64_t un, int nb, int qi) {
+      int64_t qbh;
+      int qz0, qy0, qx0;
+      origin(un, qbh, qz0, qy0, qx0);
+      const int32_t* qbox = reinterpret_cast<const int32_t*>(smem + S::kBox + nb * kBoxPitch);
+      uint8_t* qd = smem + S::kQ + qi * S::kQBuf;
+      const int pairs = P.ix.rope_pairs, rmax = P.ix.rope_rows - 1;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int r = 64 * w + 32 * pass + lane;
+        const int rw = r >> 5, rl = r & 31;
+        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = 4 * tile + (rl & 3);
+        const int slot = in_grid(qz0 + z, qy0 + y, qx0 + x)
+                             ? qbox[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
+                             : -1;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(P.q + (qbh * N + (slot >= 0 ? slot : 0)) * D);
+        uint4 row[KC];
+#pragma unroll
+        for (int c = 0; c < KC; ++c) row[c] = src[c];
+        const int cz = min(qz0 + z, rmax), cy = min(qy0 + y, rmax), cx = min(qx0 + x, rmax);
+#pragma unroll
+        for (int c = 0; c < KC; ++c) {
+          const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
+          const int cv = axis == 0 ? cz : (axis == 1 ? cy : cx);
+          // (cos, sin) of the piece's 4 rotation pairs: 32 contiguous bytes of the table
+          const float4* cs4 = reinterpret_cast<const float4*>(P.ix.rope + 2 * (cv * pairs + p0));
+          const float4 ca = __ldg(cs4), cbv = __ldg(cs4 + 1);
+          const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
+          const uint32_t xin[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
+          uint32_t xo[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float e0 = __uint_as_float(xin[k] << 16);
+            const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+            xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
+                                  e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
+          }
+          if (slot < 0) xo[0] = xo[1] = xo[2] = xo[3] = 0u;
+          *reinterpret_cast<uint4*>(qd + S::q_off(r, c)) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[B_QFULL + qi]);
+    };
     int ti = 0;
     bool ok = true;
     for (; ok; ++ti) {
@@ -276,6 +333,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + bb], (ti >> 1) & 1))) break;
       const int64_t u = unit_of(bb);
       if (u < 0) break;
+      if (ti == 0 && w < 2) prepare_q(u, 0, tile);  // the first unit's q tile
       int64_t bh;
       int z0, y0, x0;
       origin(u, bh, z0, y0, x0);
@@ -317,16 +375,17 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         }
         if (ln == 0 && tile == 0) GTR(ti, 110 + w * 20 + i * 4);
         tc::tc_fence_after();
-        // the chunk's 48 window scores; entries off the 3x3x3 cube become -inf
+        // the chunk's first 36 window scores (the rest never hold a neighbour of this tile);
+        // entries off the 3x3x3 cube become -inf
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        uint32_t r[kNK];
-#pragma unroll
-        for (int c0 = 0; c0 < kNK; c0 += 16)
-          tc::tmem_ld16(tl + s_col(b) + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[c0]));
+        uint32_t r[kNV];
+        tc::tmem_ld16(tl + s_col(b), *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+        tc::tmem_ld16(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+        lg::tmem_ld4(tl + s_col(b) + 32, &r[32]);
         tc::tmem_wait_ld();
         const uint64_t win = nb[i];
 #pragma unroll
-        for (int k = 0; k < kNK; k += 2) {
+        for (int k = 0; k < kNV; k += 2) {
           if (!((win >> k) & 1ull)) r[k] = 0xff800000u;
           if (!((win >> (k + 1)) & 1ull)) r[k + 1] = 0xff800000u;
           mx[(k >> 1) & 3] =
@@ -367,7 +426,9 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         const float2 sl2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(neg_m, neg_m);
         uint32_t p[kNK / 2];
 #pragma unroll
-        for (int k = 0; k < kNK; k += 2) {
+        for (int k = kNV; k < kNK; k += 2) p[k >> 1] = 0u;  // P = 0 where no neighbour can be
+#pragma unroll
+        for (int k = 0; k < kNV; k += 2) {
           const float2 x =
               tc::fma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), sl2, nm2);
           const float2 e = make_float2(ex2(x.x), ex2(x.y));
@@ -411,141 +472,79 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         if (P.lse_loc)
           P.lse_loc[bh * N + slot] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
+      if (w < 2) {
+        // the next unit's q tile, into the other q buffer once its slot box is in and the
+        // buffer's previous unit (ti - 1) has finished its QK MMAs
+        const int nb = (ti + 1) & 1, qi = nb * 2 + tile;
+        if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + nb], ((ti + 1) >> 1) & 1))) break;
+        const int64_t un = unit_of(nb);
+        if (un >= 0) {
+          if (ti >= 1 &&
+              !__all_sync(0xffffffffu, ab.wait(&bars[B_QEMPTY + qi], ((ti - 1) >> 1) & 1)))
+            break;
+          prepare_q(un, nb, qi);
+        }
+      }
     }
-  } else if (warp < W_PROD) {
-    // --------------------------------------------------------- slot boxes and q tiles
-    // q warp `tile` (warp 8 also loads the slot box): per unit, the tile's 128 q rows (one
-    // cp.async per 16-byte piece, rows off the grid zero-filled), rotated in place by the lane
-    // that copied them. Box and q buffers are double-buffered, so this runs one unit ahead of
-    // the MMAs.
-    const int tile = warp - W_Q;
+  } else if (warp == W_BOX) {
+    // --------------------------------------------------------- slot boxes (warp 8)
+    // Per unit: the next unit index from the device-wide counter, posted with the unit's slot
+    // box (3D TMA, or plain loads when the grid pitch does not suit TMA); -1 when none is left.
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, ab.wait(bar, parity));
     };
-    float2* rope_q = reinterpret_cast<float2*>(smem + S::kRope) + tile * 16 * PR;  // [16][PR]
-    constexpr int QN = 128 * KC / 32;  // q pieces per lane, row-contiguous order
-    int ti = 0;
     uint32_t box_phases[2] = {0u, 0u};  // phases started on B_BOX (lane 0), for the exit
-    for (;; ++ti) {
+    for (int ti = 0;; ++ti) {
       const int bb = ti & 1;
       int32_t* box = reinterpret_cast<int32_t*>(smem + S::kBox + bb * kBoxPitch);
-      int64_t u, bh;
-      int z0, y0, x0;
-      if (tile == 0) {
-        // the next unit from the device-wide counter, published with its slot box
-        if (lane == 0) GTR(ti, 0);
-        if (ti >= 2 && !wwait(&bars[B_BOXFREE + bb], ((ti >> 1) - 1) & 1)) break;
-        if (lane == 0) GTR(ti, 1);
-        unsigned int nu = 0;
-        if (lane == 0) nu = atomicAdd(reinterpret_cast<unsigned int*>(P.ix.status + 2), 1u);
-        u = (int64_t)__shfl_sync(0xffffffffu, nu, 0);
-        if (u >= P.units) {
-          if (lane == 0) {
-            *reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes) = -1;
-            ++box_phases[bb];
-            tc::mbar_arrive(&bars[B_BOX + bb]);
-          }
-          break;
+      volatile int64_t* uslot =
+          reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes);
+      if (lane == 0) GTR(ti, 0);
+      if (ti >= 2 && !wwait(&bars[B_BOXFREE + bb], ((ti >> 1) - 1) & 1)) break;
+      if (lane == 0) GTR(ti, 1);
+      unsigned int nu = 0;
+      if (lane == 0) nu = atomicAdd(reinterpret_cast<unsigned int*>(P.ix.status + 2), 1u);
+      const int64_t u = (int64_t)__shfl_sync(0xffffffffu, nu, 0);
+      if (u >= P.units) {
+        if (lane == 0) {
+          *uslot = -1;
+          ++box_phases[bb];
+          tc::mbar_arrive(&bars[B_BOX + bb]);
         }
-        origin(u, bh, z0, y0, x0);
-        if (lane == 0)
-          *reinterpret_cast<volatile int64_t*>(smem + S::kBox + bb * kBoxPitch + kBoxBytes) = u;
-        __syncwarp();
-        if (P.box_tma) {
-          if (lane == 0) {
-            ++box_phases[bb];
-            tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
-            tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
-          }
-        } else {
-          for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
-            const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
-            const int z = z0 - 1 + bz, y = y0 - 1 + by, x = x0 - 4 + bx;
-            box[i] = in_grid(z, y, x) ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : 0;
-          }
-          __syncwarp();
-          if (lane == 0) {
-            ++box_phases[bb];
-            tc::mbar_arrive(&bars[B_BOX + bb]);
-          }
+        break;
+      }
+      int64_t bh;
+      int z0, y0, x0;
+      origin(u, bh, z0, y0, x0);
+      if (lane == 0) *uslot = u;
+      __syncwarp();
+      if (P.box_tma) {
+        if (lane == 0) {
+          ++box_phases[bb];
+          tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
+          tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
         }
       } else {
-        if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
-        u = unit_of(bb);
-        if (u < 0) break;
-        origin(u, bh, z0, y0, x0);
-      }
-      const int xt = x0 + 4 * tile;  // the tile's first x
-      // rotation table of the tile: rows z0..z0+7, y0..y0+3, xt..xt+3 (the previous unit's
-      // rotation, its only reader, is complete)
-      for (int i = lane; i < 16 * PR; i += 32) {
-        const int idx = i / PR, pp = i % PR;
-        int cv = idx < 8 ? z0 + idx : (idx < 12 ? y0 + idx - 8 : xt + idx - 12);
-        cv = min(cv, P.ix.rope_rows - 1);
-        rope_q[i] = rope_cs(P.ix.rope, P.ix.rope_pairs, cv, pp);
-      }
-      // the q buffer was last read by the tile's QK MMAs of unit ti - 2
-      if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
-      if (ti >= 2 && !wwait(&bars[B_QEMPTY + bb * 2 + tile], ((ti >> 1) - 1) & 1)) break;
-      if (lane == 0 && tile == 0) GTR(ti, 2);
-      uint8_t* qd = smem + S::kQ + (bb * 2 + tile) * S::kQBuf;
-      const __nv_bfloat16* qg = P.q + bh * N * D;
-      // q row r of a tile holds position (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4)
-#pragma unroll 4
-      for (int j = 0; j < QN; ++j) {
-        const int i = lane + 32 * j, r = i / KC, c = i % KC;
-        const int rw = r >> 5, rl = r & 31;
-        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = 4 * tile + (rl & 3);
-        const int slot = in_grid(z0 + z, y0 + y, x0 + x)
-                             ? box[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
-                             : -1;
-        tc::cp_async16(qd + S::q_off(r, c), qg + (int64_t)(slot >= 0 ? slot : 0) * D + c * 8,
-                       slot >= 0);
-      }
-      tc::cp_async_commit();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);  // this warp's box reads are done
-      tc::cp_async_wait_group<0>();
-      __syncwarp();  // rope_q complete
-      if (lane == 0 && tile == 0) GTR(ti, 3);
-      // rotate the pieces this lane copied (rows off the grid are zero and stay zero)
-#pragma unroll 2
-      for (int j = 0; j < QN; ++j) {
-        const int i = lane + 32 * j, r = i / KC, c = i % KC;
-        uint4* ptr = reinterpret_cast<uint4*>(qd + S::q_off(r, c));
-        const int rw = r >> 5, rl = r & 31;
-        const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
-        const int idx =
-            axis == 0 ? 2 * rw + (rl >> 4) : (axis == 1 ? 8 + ((rl >> 2) & 3) : 12 + (rl & 3));
-        const float4* cs4 = reinterpret_cast<const float4*>(rope_q + idx * PR + p0);
-        const float4 ca = cs4[0], cbv = cs4[1];
-        const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
-        const uint4 xv = *ptr;
-        const uint32_t xin[4] = {xv.x, xv.y, xv.z, xv.w};
-        uint32_t xo[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float e0 = __uint_as_float(xin[k] << 16);
-          const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
-          xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
-                                e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
+        for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
+          const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
+          const int z = z0 - 1 + bz, y = y0 - 1 + by, x = x0 - 4 + bx;
+          box[i] = in_grid(z, y, x) ? P.ix.inv[((int64_t)z * g.gy + y) * g.gx + x] : 0;
         }
-        *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+        __syncwarp();
+        if (lane == 0) {
+          ++box_phases[bb];
+          tc::mbar_arrive(&bars[B_BOX + bb]);
+        }
       }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[B_QFULL + bb * 2 + tile]);
-      __syncwarp();  // rope_q is rewritten for the next unit
-      if (lane == 0 && tile == 0) GTR(ti, 4);
     }
-    tc::cp_async_wait_all();
     // nothing may still be landing in shared memory when the CTA exits: wait for the latest
     // phase of each box barrier (phases complete in order; bounded waits; lane 0's counts)
-    if (tile == 0 && lane == 0)
+    if (lane == 0)
       for (int b2 = 0; b2 < 2; ++b2)
-        if (box_phases[b2])
-          if (!tc::mbar_wait(&bars[B_BOX + b2], (box_phases[b2] - 1) & 1, 100000000LL))
-            set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
-  } else if (warp < W_MMA) {
+        if (box_phases[b2] &&
+            !tc::mbar_wait(&bars[B_BOX + b2], (box_phases[b2] - 1) & 1, 100000000LL))
+          set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
+  } else if (warp >= W_PROD && warp < W_MMA) {
     // --------------------------------------------------------- k/v rows (128 threads)
     // Halo slice s of rotated keys and values: 60 rows x d, one cp.async per 16-byte piece in
     // row-contiguous order (rows off the grid are zero-filled). Each thread's copies arrive on
@@ -625,7 +624,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       if ((pt & 31) == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
     }
     tc::cp_async_wait_all();  // nothing may still be landing in shared memory at exit
-  } else {
+  } else if (warp >= W_MMA) {
     // --------------------------------------------------------- MMA issuers (warps 14, 15)
     // One warp per tile. Per slice s: PV(s) for its owners (other rows disabled), then -- once
     // PV(s) has completed, which frees S buffer s % 2 -- QK(s + 2). The whole warp runs the
