@@ -236,6 +236,12 @@ def test_forward_262k_field_sampled():
     sampled_compare(inputs.make_workload("field262k_bf16"), False, heads=((0, 3),), count=64)
 
 
+def test_forward_rotated_keys_262k_field_sampled():
+    # the benchmarked path (summaries + rotated keys, two-tile local units) on the 64^3 field
+    sampled_compare(inputs.make_workload("field262k_bf16"), False, heads=((0, 5),), count=64,
+                    rotated=True)
+
+
 def test_repacking_equivariance_is_exact_65k_field():
     # four coordinate-carrying packings: outputs are exact permutations of the raster output
     outs = {}
