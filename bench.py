@@ -345,8 +345,8 @@ def main():
         torch.cuda.synchronize()
         bms = be0.elapsed_time(be1) / nb
         M = int(np.prod([g_ // b_ for g_, b_ in zip(w["grid"], w["block"])]))
-        # SURVEY-style count: the global branch's backward is 2.5x its forward contraction
-        # (dS, dq, dK_sum, dV_sum: 5 products of N x M x d per (batch, head))
+        # the global branch's backward: five products of N x M x d per (batch, head) (S
+        # recomputed, dP, dq, dK_sum, dV_sum), 2.5x its forward contraction
         bflops = 10.0 * N * M * d * B * H
         peaks_b = measured_peaks()
         extra["attn_bwd"] = {"ms": bms, "tokens_per_s": B * N / (bms / 1e3),
