@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
   PACK3D_OK = 0,
   PACK3D_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent arguments */
-  PACK3D_ERR_UNSUPPORTED = 2,   /* valid but not supported by this build (d, partial grid) */
+  PACK3D_ERR_UNSUPPORTED = 2,   /* valid but not supported by this library (d, partial grid) */
   PACK3D_ERR_DUP_COORD = 3,     /* two tokens carry the same coordinate */
   PACK3D_ERR_COORD_RANGE = 4,   /* a coordinate (or raster id) lies outside the grid */
   PACK3D_ERR_ALIGN = 5,         /* a pointer is not 16-byte aligned */
