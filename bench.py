@@ -230,6 +230,23 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------ multi-rank
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (ms) over every rank of the default process group
+    (identity on one rank): the job is as slow as its slowest rank."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(world, tokens_per_rank, ms):
+    """Whole-job tokens/s when each of `world` ranks processes `tokens_per_rank` tokens per step
+    and a step takes `ms` (the max over ranks)."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -308,11 +325,9 @@ def main():
     ms = t0.elapsed_time(t1) / args.steps
     ms_k = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
             for i, name in enumerate(("summarize", "local", "global"))}
-    if world > 1:
-        tt = torch.tensor([ms] + [ms_k[n] for n in ("summarize", "local", "global")], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        vals = [float(x) for x in tt.tolist()]
-        ms, ms_k = vals[0], dict(zip(("summarize", "local", "global"), vals[1:]))
+    vals = max_over_ranks([ms] + [ms_k[n] for n in ("summarize", "local", "global")],
+                          dist if world > 1 else None, dev)
+    ms, ms_k = vals[0], dict(zip(("summarize", "local", "global"), vals[1:]))
 
     # Outside the headline step: the index build (once per geometry) and the backward of the
     # same field (dO ~ N(0, 1), seed 2), each timed with CUDA events on this stream.
@@ -389,11 +404,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / k_e2e
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        e2e = {"value": world * B * N / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        ems = max_over_ranks([ems], dist if world > 1 else None, dev)[0]
+        e2e = {"value": job_throughput(world, B * N, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e}
 
     if rank == 0:
@@ -423,7 +435,7 @@ def main():
         dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
         roof = dict(kernels[dominant])
         line = {
-            "metric": METRIC, "value": world * B * N / (ms / 1e3), "unit": UNIT,
+            "metric": METRIC, "value": job_throughput(world, B * N, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(args.workload, w),
