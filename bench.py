@@ -66,16 +66,60 @@ def workload_config(name, w):
 
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU while the timed region runs: NVML
+    polled every 2 ms from a thread (read-only queries), or nvidia-smi at 100 ms when NVML is
+    not available."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
     def __init__(self, device_index):
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.idx)
 
     def start(self):
+        try:
+            import threading
+
+            import pynvml
+            h = self._nvml_handle()
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.stop_flag = threading.Event()
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        self.rows.append(dict(
+                            sm=float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                            smax=smax,
+                            power=pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                            bits=int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        break
+                    time.sleep(0.002)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 2 ms"
+            return
+        except Exception:
+            self.thread = None
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -85,41 +129,46 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
+            self.source = "nvidia-smi, 100 ms"
         except Exception:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
         rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            for r in self.rows:
+                rows.append(dict(sm=r["sm"], smax=r["smax"], power=r["power"],
+                                 reasons={n for bit, n in self.REASONS.items() if r["bits"] & bit}))
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                rows.append(dict(sm=float(parts[0]), smax=float(parts[1]),
-                                 power=float(parts[2]) if parts[2] not in ("[N/A]", "") else 0.0,
-                                 hw=parts[4], hwt=parts[5], swt=parts[6], pcap=parts[7]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[0]), smax=float(parts[1]),
+                                     power=float(parts[2]) if parts[2] not in ("[N/A]", "") else 0.0,
+                                     reasons={n for n, v in zip(names, parts[4:8])
+                                              if v.lower() == "active"}))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
         if not rows:
             return None
         load = [r for r in rows if r["power"] > 0.25 * max(x["power"] for x in rows)] or rows
         reasons = set()
         for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower() == "active":
-                    reasons.add(name)
+            reasons |= r["reasons"]
         return {"sm_mhz": statistics.median(r["sm"] for r in load),
                 "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(rows), "source": self.source}
 
 
 # ---------------------------------------------------------------------------- roofline
