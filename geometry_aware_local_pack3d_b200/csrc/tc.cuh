@@ -127,16 +127,6 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// 2D tiled load (no multicast) of box {x .. x+bx, y .. y+by} into shared memory.
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // 3D tiled load (no multicast) of a box starting at (x, y, z) into shared memory.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int x, int y,
                                             int z, uint64_t* bar) {
@@ -146,19 +136,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-// Row gather (no multicast): columns [col, col + box) of rows r0..r3 of a 2D tensor whose box
-// is one row high, written as 4 consecutive box rows at smem_dst. Rows outside the tensor read
-// as zeros.
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, int col,
-                                            int r0, int r1, int r2, int r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(smem_u32(bar))
-      : "memory");
-}
-
 // -------------------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -254,12 +231,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return d;                // base offset 0, lbo mode 0, layout type 0 (no swizzle)
 }
 
-// Shared-memory matrix descriptor for the 128-byte swizzle (layout type 2): rows of 128 bytes,
-// 8-row atoms of 1024 bytes (sbo), lbo = stride between 64-element column blocks (MN-major).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return smem_desc(saddr, lbo, sbo) | (2ull << 61);
-}
-
 // Instruction descriptor of kind::f16: bf16 A and B, f32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                      bool b_mn_major) {
@@ -282,19 +253,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// As mma_ss, with D rows (TMEM lanes) whose bit is set in the 128-bit mask m0..m3 left as they
-// are (m0 covers lanes 0-31, m1 lanes 32-63, ...).
-__device__ __forceinline__ void mma_ss_masked(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate, uint32_t m0,
-                                              uint32_t m1, uint32_t m2, uint32_t m3) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3)
-      : "memory");
-}
 // D[tmem] (+)= A[tmem] * B[smem desc]   (A is K-major, 2 bf16 per 32-bit column)
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -305,7 +263,8 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// As mma_ts, with D rows whose bit is set in the 128-bit mask m0..m3 left as they are.
+// As mma_ts, with the D rows (TMEM lanes) whose bit is set in the 128-bit mask m0..m3 left as
+// they are (m0 covers lanes 0-31, m1 lanes 32-63, ...).
 __device__ __forceinline__ void mma_ts_masked(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                               uint32_t idesc, uint32_t accumulate, uint32_t m0,
                                               uint32_t m1, uint32_t m2, uint32_t m3) {

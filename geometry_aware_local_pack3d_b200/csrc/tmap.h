@@ -28,20 +28,6 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// [rows, cols] bf16 row-major as a row-gather source: box = 64 columns x 1 row, 128-byte swizzle.
-inline bool encode_gather_rows_bf16(CUtensorMap* map, const void* base, int64_t rows, int cols) {
-  EncodeTiledFn fn = encode_tiled_fn();
-  if (!fn || (reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
 // [gz, gy, gx] int32 grid as a 3D box source (box bx x by x bz, no swizzle); the row pitch
 // gx * 4 must be a multiple of 16 bytes.
 inline bool encode_grid_i32(CUtensorMap* map, const void* base, int gz, int gy, int gx, int bx,
