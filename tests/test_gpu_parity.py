@@ -409,6 +409,33 @@ def test_forward_work_counter_returns_to_zero(bh):
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
+def test_local_units_independent_of_batch_and_stream():
+    # every (batch, head, unit) is computed on its own: one head's output from a batch of 30
+    # heads (units spread over all SMs by the work counter) equals, bit for bit, the same head
+    # computed alone on a side stream with the same index
+    m = p3d()
+    w = small((8, 8, 16), (4, 4, 4), 6, 5, 96, "bf16", "random", qkv_std=96 ** -0.5)
+    ix = gpu_index(w, 96)
+    q, k, v = (w[n].to(torch.bfloat16).cuda().contiguous() for n in "qkv")
+    _, _, k_rot = m.pack3d_summarize_rotated(ix, k, v)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    o_all, _ = m.pack3d_attn_local(ix, q, k_rot, v, k_rotated=True, lse_loc=lse)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    for b, h in ((0, 0), (5, 4), (2, 3)):
+        sl = lambda t: t[b:b + 1, h:h + 1].contiguous()  # noqa: E731
+        q1, k1, v1 = sl(q), sl(k_rot), sl(v)
+        with torch.cuda.stream(side):
+            lse1 = torch.empty((1, 1, q.shape[2]), dtype=torch.float32, device=q.device)
+            o1, _ = m.pack3d_attn_local(ix, q1, k1, v1, k_rotated=True, lse_loc=lse1,
+                                        stream=side)
+        side.synchronize()
+        assert torch.equal(o1[0, 0], o_all[b, h]), (b, h)
+        assert torch.equal(lse1[0, 0], lse[b, h]), (b, h)
+    st = ix.table("status", (4,)).cpu()
+    assert int(st[0]) == 0 and int(st[2]) == 0 and int(st[3]) == 0, st
+
+
 @pytest.mark.parametrize("dtype,d,rotated", [("bf16", 96, True), ("bf16", 96, False),
                                              ("bf16", 48, True), ("fp32", 48, False)])
 def test_split_local_global_calls_equal_fused_forward(dtype, d, rotated):
