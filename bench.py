@@ -61,7 +61,8 @@ def workload_config(name, w):
                 [g // b for g, b in zip(w["grid"], w["block"])])),
             "packing": w["packing"], "exclude_near": w["exclude_near"],
             "l2": "inputs larger than L2: q, k, v alone are "
-                  f"{3 * w['batch'] * w['heads'] * int(np.prod(w['grid'])) * w['d'] * 2 / 1e6:.0f} MB per step"}
+                  f"{3 * w['batch'] * w['heads'] * int(np.prod(w['grid'])) * w['d'] * 2 / 1e6:.0f}"
+                  " MB per step"}
 
 
 # ------------------------------------------------------------------------------ clocks

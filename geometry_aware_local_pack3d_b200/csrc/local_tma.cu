@@ -32,8 +32,9 @@
 //   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2)
 //   owners: 3x3x3 mask, online softmax over the window's first 36 columns (the only ones that
 //   can hold a neighbour of the tile), P = exp2(s - m) as bf16 over the buffer's first 24
-//   columns (P = 0 in window columns 36..47);  O += P_s v_s  (TS MMA, N = d) with the rows of the other warps disabled through
-//   the MMA's output-lane mask, so non-owners never touch chunk s.
+//   columns (P = 0 in window columns 36..47);  O += P_s v_s  (TS MMA, N = d) with the rows
+//   of the other warps disabled through the MMA's output-lane mask, so non-owners never touch
+//   chunk s.
 // Each tile has its own MMA warp; QK runs two chunks ahead of PV, so S_{s+2} is ready when the
 // owners finish chunk s + 1. Each softmax warp zeroes its O rows when it starts a unit; its
 // epilogue runs after the PV of its last chunk. Every query sits at the same row and every

@@ -234,7 +234,8 @@ def test_all_summaries_excluded_gives_zero_global_output():
 def test_summary_set_order_invariance():
     # project page Ch.7: permuting summary keys and values together changes nothing
     g = np.random.default_rng(0)
-    qr, ks, vs = g.standard_normal((1, 2, 20, 12)), g.standard_normal((1, 2, 9, 12)), g.standard_normal((1, 2, 9, 12))
+    qr = g.standard_normal((1, 2, 20, 12))
+    ks, vs = g.standard_normal((1, 2, 9, 12)), g.standard_normal((1, 2, 9, 12))
     p = g.permutation(9)
     o1, l1 = orc.global_branch(qr, ks, vs, 0.3)
     o2, l2 = orc.global_branch(qr, ks[:, :, p], vs[:, :, p], 0.3)
