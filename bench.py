@@ -9,6 +9,12 @@ the packed field is built once per geometry before timing, as it is amortised ov
 heads and batches. Default workload: the 65,536-token field (32x32x64 grid, batch 2, 8 heads,
 head_dim 96, bf16, 4x4x4 blocks -> 1,024 summaries, raster-block packing).
 
+The line's `roofline` is the whole step's: the slower of the step's algorithmic bytes at the
+measured HBM peak and its global-contraction flops at the measured bf16 peak, against the step
+time; the per-kernel rooflines sit under `kernels` (and the slowest under
+`roofline.dominant_kernel`). On one GPU the same run also reports the forward + backward of
+the headline field (`fwd_bwd`, `attn_bwd`) and the 262,144-token field (`field262k_bf16`).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pack3d|reference]
 
 With N > 1 the script is launched by torch.distributed.run, one rank per GPU; every rank runs
@@ -58,7 +64,7 @@ def workload_config(name, w):
     return {"workload": name, "grid": list(w["grid"]), "block": list(w["block"]),
             "batch": w["batch"], "heads": w["heads"], "head_dim": w["d"],
             "tokens": int(np.prod(w["grid"])), "summaries": int(np.prod(
-                [g // b for g, b in zip(w["grid"], w["block"])])),
+                [-(-g // b) for g, b in zip(w["grid"], w["block"])])),
             "packing": w["packing"], "exclude_near": w["exclude_near"],
             "l2": "inputs larger than L2: q, k, v alone are "
                   f"{3 * w['batch'] * w['heads'] * int(np.prod(w['grid'])) * w['d'] * 2 / 1e6:.0f}"
@@ -198,12 +204,17 @@ def kernel_traffic(kernel_key):
     return d["bytes_per_launch_full"]
 
 
+def _sizes(w):
+    B, H, d = w["batch"], w["heads"], w["d"]
+    N = int(np.prod(w["grid"]))
+    M = int(np.prod([-(-g // b) for g, b in zip(w["grid"], w["block"])]))
+    return B, H, N, M, d
+
+
 def algorithmic(w):
     """Per-launch algorithmic work of the three kernels of a step (each row read or written
     once; index tables read once)."""
-    B, H, d = w["batch"], w["heads"], w["d"]
-    N = int(np.prod(w["grid"]))
-    M = int(np.prod([g // b for g, b in zip(w["grid"], w["block"])]))
+    B, H, N, M, d = _sizes(w)
     el = 2  # bf16
     e = B * H * N * d * el  # bytes of one [B, H, N, d] tensor
     return {
@@ -217,41 +228,71 @@ def algorithmic(w):
     }
 
 
+def step_algorithmic(w, index_bytes):
+    """Algorithmic work of one forward step whatever the kernel split: q, k, v read and o
+    written once, the gate logits read, the summaries written and read back once, the index
+    tables read once; the global contraction's 4 N M d flops per (batch, head)."""
+    B, H, N, M, d = _sizes(w)
+    el = 2
+    e = B * H * N * d * el
+    summ = B * H * M * d * el
+    return {"bytes": 4 * e + B * H * N * el + 2 * 2 * summ + index_bytes,
+            "flops": 4.0 * N * M * d * B * H}
+
+
+def step_roofline(alg, ms, peaks):
+    """Roofline of a whole step: the slower of its bytes at the HBM peak and its flops at the
+    bf16 tensor peak, against the measured step time."""
+    t_hbm = alg["bytes"] / (peaks["hbm"] * 1e9)
+    t_mma = alg["flops"] / (peaks["bf16"] * 1e12)
+    sec = ms / 1e3
+    if t_mma >= t_hbm:
+        ach = alg["flops"] / sec / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16"], "roofline_ms": t_mma * 1e3,
+                "algorithmic_flops_per_step": alg["flops"],
+                "algorithmic_bytes_per_step": alg["bytes"],
+                "peak_source": f"{peaks['source']} bf16 dense burst"}
+    ach = alg["bytes"] / sec / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": ach / peaks["hbm"], "roofline_ms": t_hbm * 1e3,
+            "algorithmic_flops_per_step": alg["flops"], "algorithmic_bytes_per_step": alg["bytes"],
+            "peak_source": f"{peaks['source']} HBM copy"}
+
+
 # -------------------------------------------------------------------------------- oracle
 def oracle_sample(w, idx, head=(0, 0)):
-    """Time the float64 oracle on one (batch, head) of the workload: summaries + all rows."""
+    """Time the float64 oracle on one (batch, head) of the workload: summaries + all rows.
+    Returns (wall seconds, process CPU seconds)."""
     from oracle import pack3d_oracle as orc
     b, h = head
     sl = lambda t: t[b:b + 1, h:h + 1].numpy()  # noqa: E731
     q, k, v, a = sl(w["q"]), sl(w["k"]), sl(w["v"]), sl(w["a"])
-    t0 = time.perf_counter()
+    c0, t0 = time.process_time(), time.perf_counter()
     orc.forward(q, k, v, a, w["coords"], w["grid"], w["block"], exclude_near=w["exclude_near"],
                 index=idx)
-    return time.perf_counter() - t0
+    return time.perf_counter() - t0, time.process_time() - c0
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+def cores_used(wall, cpu):
+    """Threads the oracle actually kept busy: process CPU time over wall time (at least 1)."""
+    return max(1, int(round(cpu / wall))) if wall > 0 else 1
 
 
-def cpu_baseline(w, reps=1):
+def cpu_baseline(w, reps=3):
     from oracle import pack3d_oracle as orc
     idx = orc.build_index(w["coords"], w["grid"], w["block"])
-    ts = [oracle_sample(w, idx) for _ in range(reps)]
-    t = statistics.median(ts)
-    B, H = w["batch"], w["heads"]
-    N = int(np.prod(w["grid"]))
+    runs = [oracle_sample(w, idx) for _ in range(reps)]
+    t = statistics.median(r[0] for r in runs)
+    cores = cores_used(sum(r[0] for r in runs), sum(r[1] for r in runs))
+    B, H, N, _, _ = _sizes(w)
     # one head of one batch element is 1/(B*H) of a step
     value = (B * N) / (t * B * H)
-    return {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"float64 numpy oracle on 1 of {B * H} (batch, head) pairs of the workload "
-                      f"(summaries + local + global + mixer for all {N} tokens), {reps} rep(s), "
-                      f"{t:.2f} s each, scaled by {B * H}"}
+                      f"(summaries + local + global + mixer for all {N} tokens), median of "
+                      f"{reps} runs ({t:.2f} s), scaled by {B * H}; cores = process CPU time / "
+                      f"wall time"}
 
 
 def run_reference(args, rank):
@@ -262,19 +303,22 @@ def run_reference(args, rank):
     idx = orc.build_index(w["coords"], w["grid"], w["block"])
     for _ in range(args.warmup):
         oracle_sample(w, idx)
-    ts = [oracle_sample(w, idx, head=(s % w["batch"], s % w["heads"])) for s in range(args.steps)]
-    B, H = w["batch"], w["heads"]
-    N = int(np.prod(w["grid"]))
-    step = float(np.mean(ts)) * B * H
-    value = B * N / step
+    runs = [oracle_sample(w, idx, head=(s % w["batch"], s % w["heads"]))
+            for s in range(args.steps)]
+    B, H, N, _, _ = _sizes(w)
+    # a step is the oracle on one (batch, head): N tokens of one head = N / H token-equivalents
+    # of the metric (a token of the metric carries all H heads)
+    step = float(np.mean([r[0] for r in runs]))
+    value = (N / H) / step
+    cores = cores_used(sum(r[0] for r in runs), sum(r[1] for r in runs))
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference", "config": workload_config(args.workload, w),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
-                             "kind": "oracle",
-                             "sample": f"each step: the float64 oracle on one (batch, head) of "
-                                       f"{B * H}, all {N} tokens; value scaled by {B * H}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"each timed step: the float64 oracle on one (batch, head) "
+                                       f"of {B * H}, all {N} tokens (= {N // H} tokens of all "
+                                       f"{H} heads); cores = process CPU time / wall time"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -298,6 +342,127 @@ def job_throughput(world, tokens_per_rank, ms):
 
 
 # ------------------------------------------------------------------------------- GPU arm
+def device_workload(name, dev):
+    """A named workload with its q, k, v, a drawn on the device (N(0, sigma^2) and N(0, 1) from
+    a seeded CUDA generator, rounded to bf16, in memory order): the large fields of the extra
+    measurements, whose CPU generation would take longer than their timing. The packing and
+    coordinates come from the same host generator as every other workload."""
+    cfg = dict(inputs.WORKLOADS[name])
+    grid, block = tuple(cfg["grid"]), tuple(cfg["block"])
+    perm = inputs.packing(cfg["packing"], grid, block)
+    B, H, N, d = cfg["batch"], cfg["heads"], int(np.prod(grid)), cfg["d"]
+    g = torch.Generator(device=dev).manual_seed(0)
+    shape = (B, H, N, d)
+    out = dict(cfg)
+    out.update(perm=perm, coords=inputs.coords_of(perm, grid))
+    for n in "qkv":
+        out[n] = (torch.randn(shape, generator=g, device=dev) * cfg["qkv_std"]).to(torch.bfloat16)
+    out["a"] = torch.randn(shape[:3], generator=g, device=dev).to(torch.bfloat16)
+    return out
+
+
+class Forward:
+    """The timed forward step of one workload on one device: summaries + rotated keys, local
+    branch, global branch + mixer, each call's kernel timed with CUDA events on its stream."""
+
+    def __init__(self, p3d, w, dev):
+        self.p3d, self.w = p3d, w
+        B, H, d = w["batch"], w["heads"], w["d"]
+        dt = torch.bfloat16
+        self.geom = p3d.make_geom(w["grid"], w["block"], d)
+        self.ix = p3d.pack3d_build_index(self.geom, coords=torch.from_numpy(w["coords"]).to(dev))
+        self.q, self.k, self.v, self.a = (w[n].to(dt).to(dev).contiguous() for n in "qkva")
+        self.ksum = torch.empty(p3d.summary_tiles_shape(self.ix, B, H, d), dtype=dt, device=dev)
+        self.vsum = torch.empty_like(self.ksum)
+        self.k_rot = torch.empty_like(self.k)
+        self.o = torch.empty_like(self.q)
+        self.stream = torch.cuda.current_stream()
+
+    def step(self, ev=None):
+        p3d, st = self.p3d, self.stream
+        if ev is not None:
+            ev[0].record(st)
+        p3d.pack3d_summarize_rotated(self.ix, self.k, self.v, self.ksum, self.vsum, self.k_rot)
+        n = p3d.pack3d_last_launch_count()
+        if ev is not None:
+            ev[1].record(st)
+        p3d.pack3d_attn_local(self.ix, self.q, self.k_rot, self.v, k_rotated=True, o_loc=self.o)
+        n += p3d.pack3d_last_launch_count()
+        if ev is not None:
+            ev[2].record(st)
+        p3d.pack3d_attn_global(self.ix, self.q, self.a, self.ksum, self.vsum, self.o,
+                               exclude_near=self.w["exclude_near"], o=self.o)
+        n += p3d.pack3d_last_launch_count()
+        if ev is not None:
+            ev[3].record(st)
+        return n
+
+    def time(self, steps, warmup, sync=None):
+        for _ in range(max(warmup, 0)):
+            self.step()
+        torch.cuda.synchronize()
+        if sync:
+            sync()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launches = 0
+        t0.record(self.stream)
+        for s in range(steps):
+            launches += self.step(evs[s])
+        t1.record(self.stream)
+        torch.cuda.synchronize()
+        if sync:
+            sync()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / steps
+        ms_k = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, name in enumerate(("summarize", "local", "global"))}
+        return ms, ms_k, launches
+
+    def index_bytes(self):
+        return self.p3d.pack3d_index_bytes(self.geom, int(np.prod(self.w["grid"])))
+
+
+KERNEL_NAMES = {"summarize": "k_summarize (pack3d_summarize_rotated)",
+                "local": "k_local_tma (pack3d_attn_local)",
+                "global": "k_global_tc (pack3d_attn_global)"}
+
+
+def kernel_rooflines(w, ms_k, peaks, workload):
+    alg = algorithmic(w)
+    kernels = {}
+    for name in ("summarize", "local", "global"):
+        sec = ms_k[name] / 1e3
+        if "flops" in alg[name]:
+            ach = alg[name]["flops"] / sec / 1e12
+            ent = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                   "frac": ach / peaks["bf16"],
+                   "algorithmic_flops_per_launch": alg[name]["flops"],
+                   "peak_source": f"{peaks['source']} bf16 dense burst"}
+        else:
+            ach = alg[name]["bytes"] / sec / 1e9
+            ent = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                   "frac": ach / peaks["hbm"], "peak_source": f"{peaks['source']} HBM copy"}
+        ent.update({"kernel": KERNEL_NAMES[name], "ms_per_launch": ms_k[name],
+                    "algorithmic_bytes_per_launch": alg[name]["bytes"],
+                    "traffic": kernel_traffic(f"{name}_{workload}")})
+        kernels[name] = ent
+    return kernels
+
+
+def forward_line(w, workload, ms, ms_k, index_bytes, peaks):
+    """Step-level roofline (the headline) plus the per-kernel rooflines."""
+    kernels = kernel_rooflines(w, ms_k, peaks, workload)
+    roof = step_roofline(step_algorithmic(w, index_bytes), ms, peaks)
+    tr = [kernels[n]["traffic"] for n in kernels]
+    roof["traffic"] = float(sum(tr)) if all(t is not None for t in tr) else None
+    roof["traffic_note"] = "DRAM bytes per step: sum of the step kernels' ncu dram__bytes"
+    dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
+    roof["dominant_kernel"] = dict(kernels[dominant])
+    return roof, kernels
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -317,129 +482,120 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    sync = dist.barrier if world > 1 else None
 
     w = inputs.make_workload(args.workload)
-    B, H, d = w["batch"], w["heads"], w["d"]
-    N = int(np.prod(w["grid"]))
-    dt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
-    geom = p3d.make_geom(w["grid"], w["block"], d)
-    ix = p3d.pack3d_build_index(geom, coords=torch.from_numpy(w["coords"]).to(dev))
-    q, k, v, a = (w[n].to(dt).to(dev).contiguous() for n in "qkva")
-    ksum = torch.empty(p3d.summary_tiles_shape(ix, B, H, d), dtype=dt, device=dev)
-    vsum = torch.empty_like(ksum)
-    k_rot = torch.empty_like(k)
-    o = torch.empty_like(q)
-    excl = w["exclude_near"]
-    stream = torch.cuda.current_stream()
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        p3d.pack3d_summarize_rotated(ix, k, v, ksum, vsum, k_rot)
-        n = p3d.pack3d_last_launch_count()
-        if ev is not None:
-            ev[1].record(stream)
-        p3d.pack3d_attn_local(ix, q, k_rot, v, k_rotated=True, o_loc=o)
-        n += p3d.pack3d_last_launch_count()
-        if ev is not None:
-            ev[2].record(stream)
-        p3d.pack3d_attn_global(ix, q, a, ksum, vsum, o, exclude_near=excl, o=o)
-        n += p3d.pack3d_last_launch_count()
-        if ev is not None:
-            ev[3].record(stream)
-        return n
-
-    for _ in range(max(args.warmup, 0)):
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    B, H, N, M, d = _sizes(w)
+    F = Forward(p3d, w, dev)
 
     clocks = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     if clocks:
         clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches = 0
-    t0.record(stream)
-    for s in range(args.steps):
-        launches += step(evs[s])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    ms, ms_k, launches = F.time(args.steps, args.warmup, sync)
     clk = clocks.stop() if clocks else None
-
-    ms = t0.elapsed_time(t1) / args.steps
-    ms_k = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-            for i, name in enumerate(("summarize", "local", "global"))}
     vals = max_over_ranks([ms] + [ms_k[n] for n in ("summarize", "local", "global")],
                           dist if world > 1 else None, dev)
     ms, ms_k = vals[0], dict(zip(("summarize", "local", "global"), vals[1:]))
+    peaks = measured_peaks()
 
-    # Outside the headline step: the index build (once per geometry) and the backward of the
-    # same field (dO ~ N(0, 1), seed 2), each timed with CUDA events on this stream.
+    # Outside the headline step (rank 0's GPU alone): the index build (once per geometry), the
+    # forward + backward of the same field (dO ~ N(0, 1), seed 2) and the 262,144-token field,
+    # each timed with CUDA events on this stream.
     extra = {}
     if not args.skip_bwd and world == 1:
+        stream = F.stream
         coords_d = torch.from_numpy(w["coords"]).to(dev)
         ie0, ie1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        p3d.pack3d_build_index(geom, coords=coords_d)
+        p3d.pack3d_build_index(F.geom, coords=coords_d)
         ie0.record(stream)
         for _ in range(3):
-            p3d.pack3d_build_index(geom, coords=coords_d)
+            p3d.pack3d_build_index(F.geom, coords=coords_d)
         ie1.record(stream)
         torch.cuda.synchronize()
         extra["index_build"] = {"ms": ie0.elapsed_time(ie1) / 3,
                                 "note": "inverse map, neighbour and block tables, RoPE table; "
                                         "includes the call's one host synchronisation"}
-        saved = p3d.pack3d_attn_fwd(ix, q, k, v, a, ksum, vsum, exclude_near=excl,
-                                    save_for_backward=True)
-        dO = inputs.pack(inputs.upstream_grad(B, H, w["grid"], d), w["perm"]).to(dt).to(dev)
-        ws = torch.empty(p3d.pack3d_bwd_workspace_bytes(ix, 1 if dt == torch.bfloat16 else 0,
-                                                        B, H), dtype=torch.uint8, device=dev)
-        p3d.pack3d_attn_bwd(ix, q, k, v, a, ksum, vsum, saved, dO, exclude_near=excl, workspace=ws)
-        be0, be1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        be0.record(stream)
-        nb = 3
-        for _ in range(nb):
-            p3d.pack3d_attn_bwd(ix, q, k, v, a, ksum, vsum, saved, dO, exclude_near=excl,
-                                workspace=ws)
-        be1.record(stream)
+        excl = w["exclude_near"]
+        dO = inputs.pack(inputs.upstream_grad(B, H, w["grid"], d), w["perm"]).to(
+            torch.bfloat16).to(dev)
+        ws = torch.empty(p3d.pack3d_bwd_workspace_bytes(F.ix, 1, B, H), dtype=torch.uint8,
+                         device=dev)
+
+        def fwd_saving():
+            p3d.pack3d_summarize_rotated(F.ix, F.k, F.v, F.ksum, F.vsum, F.k_rot)
+            return p3d.pack3d_attn_fwd(F.ix, F.q, F.k_rot, F.v, F.a, F.ksum, F.vsum,
+                                       exclude_near=excl, k_rotated=True, save_for_backward=True)
+
+        saved = fwd_saving()
+        p3d.pack3d_attn_bwd(F.ix, F.q, F.k, F.v, F.a, F.ksum, F.vsum, saved, dO,
+                            exclude_near=excl, workspace=ws)
         torch.cuda.synchronize()
-        bms = be0.elapsed_time(be1) / nb
-        M = int(np.prod([g_ // b_ for g_, b_ in zip(w["grid"], w["block"])]))
+        nb = 3
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nb)]
+        for i in range(nb):
+            ev[i][0].record(stream)
+            saved = fwd_saving()
+            ev[i][1].record(stream)
+            p3d.pack3d_attn_bwd(F.ix, F.q, F.k, F.v, F.a, F.ksum, F.vsum, saved, dO,
+                                exclude_near=excl, workspace=ws)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        fms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        bms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
         # the global branch's backward: five products of N x M x d per (batch, head) (S
         # recomputed, dP, dq, dK_sum, dV_sum), 2.5x its forward contraction
         bflops = 10.0 * N * M * d * B * H
-        peaks_b = measured_peaks()
+        fflops = 4.0 * N * M * d * B * H
         extra["attn_bwd"] = {"ms": bms, "tokens_per_s": B * N / (bms / 1e3),
                              "roofline": {"bound": "tensor", "algorithmic_flops": bflops,
                                           "achieved": bflops / (bms / 1e3) / 1e12,
-                                          "peak": peaks_b["bf16"], "unit": "TFLOP/s",
-                                          "frac": bflops / (bms / 1e3) / 1e12 / peaks_b["bf16"]},
+                                          "peak": peaks["bf16"], "unit": "TFLOP/s",
+                                          "frac": bflops / (bms / 1e3) / 1e12 / peaks["bf16"]},
                              "path": "global branch on tensor cores (k_bwd_dsum_tc, "
                                      "k_bwd_dq_tc); row prologue, local branch, un-pooling and "
                                      "inverse RoPE on CUDA cores (k_bwd_prep, k_bwd_dq, "
                                      "k_bwd_dkv)"}
+        extra["fwd_bwd"] = {"workload": "field65k_fwdbwd_bf16 (the headline field, forward "
+                                        "saving o_loc, o_glob and both lse, then the backward)",
+                            "ms": fms + bms, "fwd_ms": fms, "bwd_ms": bms,
+                            "tokens_per_s": B * N / ((fms + bms) / 1e3),
+                            "roofline": {"bound": "tensor",
+                                         "algorithmic_flops": fflops + bflops,
+                                         "achieved": (fflops + bflops) / ((fms + bms) / 1e3) / 1e12,
+                                         "peak": peaks["bf16"], "unit": "TFLOP/s",
+                                         "frac": (fflops + bflops) / ((fms + bms) / 1e3) / 1e12
+                                         / peaks["bf16"]}}
         del saved, dO, ws
+
+        # the 262,144-token field (64^3, batch 1, 8 heads, 4,096 summaries)
+        name = "field262k_bf16"
+        w2 = device_workload(name, dev)
+        F2 = Forward(p3d, w2, dev)
+        ms2, ms2_k, _ = F2.time(10, 3)
+        roof2, kern2 = forward_line(w2, name, ms2, ms2_k, F2.index_bytes(), peaks)
+        B2, H2, N2, _, _ = _sizes(w2)
+        extra[name] = {"config": workload_config(name, w2), "ms_per_step": ms2,
+                       "tokens_per_s": B2 * N2 / (ms2 / 1e3), "roofline": roof2,
+                       "kernels": kern2, "steps": 10, "warmup": 3,
+                       "data": "synthetic, drawn on the device (seeded CUDA generator)"}
+        del F2, w2
 
     # end to end through the public API with host buffers: H2D of the inputs and D2H of o
     e2e = None
     if not args.skip_e2e:
+        dt = torch.bfloat16
         hq, hk, hv, ha = (t.to(dt).pin_memory() for t in (w["q"], w["k"], w["v"], w["a"]))
-        ho = torch.empty(o.shape, dtype=dt).pin_memory()
+        ho = torch.empty(F.o.shape, dtype=dt).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha))
         d2h = ho.numel() * ho.element_size()
 
         def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            a.copy_(ha, non_blocking=True)
-            step()
-            ho.copy_(o, non_blocking=True)
+            F.q.copy_(hq, non_blocking=True)
+            F.k.copy_(hk, non_blocking=True)
+            F.v.copy_(hv, non_blocking=True)
+            F.a.copy_(ha, non_blocking=True)
+            F.step()
+            ho.copy_(F.o, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -448,10 +604,10 @@ def main():
             dist.barrier()
         k_e2e = max(3, min(args.steps, 10))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(F.stream)
         for _ in range(k_e2e):
             e2e_step()
-        e1.record(stream)
+        e1.record(F.stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / k_e2e
         ems = max_over_ranks([ems], dist if world > 1 else None, dev)[0]
@@ -459,31 +615,7 @@ def main():
                "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e}
 
     if rank == 0:
-        peaks = measured_peaks()
-        alg = algorithmic(w)
-        kernel_names = {"summarize": "k_summarize (pack3d_summarize_rotated)",
-                        "local": "k_local_tma (pack3d_attn_local)",
-                        "global": "k_global_tc (pack3d_attn_global)"}
-        kernels = {}
-        for name in ("summarize", "local", "global"):
-            sec = ms_k[name] / 1e3
-            if "flops" in alg[name]:
-                ach = alg[name]["flops"] / sec / 1e12
-                ent = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16"],
-                       "unit": "TFLOP/s", "frac": ach / peaks["bf16"],
-                       "algorithmic_flops_per_launch": alg[name]["flops"],
-                       "peak_source": f"{peaks['source']} bf16 dense burst"}
-            else:
-                ach = alg[name]["bytes"] / sec / 1e9
-                ent = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                       "frac": ach / peaks["hbm"],
-                       "peak_source": f"{peaks['source']} HBM copy"}
-            ent.update({"kernel": kernel_names[name], "ms_per_launch": ms_k[name],
-                        "algorithmic_bytes_per_launch": alg[name]["bytes"],
-                        "traffic": kernel_traffic(f"{name}_{args.workload}")})
-            kernels[name] = ent
-        dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
-        roof = dict(kernels[dominant])
+        roof, kernels = forward_line(w, args.workload, ms, ms_k, F.index_bytes(), peaks)
         line = {
             "metric": METRIC, "value": job_throughput(world, B * N, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -491,8 +623,6 @@ def main():
             "data": "synthetic", "config": workload_config(args.workload, w),
             "roofline": roof,
             "kernels": kernels,
-            # the global contraction's flops over the whole forward (local + global kernels)
-            "fwd_tflops": alg["global"]["flops"] / ((ms_k["local"] + ms_k["global"]) / 1e3) / 1e12,
             "gpu_launches": launches,
             "clocks": clk,
             "e2e": e2e,

@@ -9,5 +9,6 @@ from .binding import (  # noqa: F401
     pack3d_attn_global, pack3d_attn_local,
     pack3d_build_index, pack3d_bwd_workspace_bytes, pack3d_device_status, pack3d_index_bytes,
     pack3d_last_launch_count, pack3d_strerror, pack3d_summarize, pack3d_summarize_rotated,
+    pack3d_testing_set_wait_budget,
     pack3d_summary_bytes, summary_rows, summary_tiles_shape,
 )

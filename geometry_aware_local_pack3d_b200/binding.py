@@ -96,6 +96,8 @@ def lib():
         L.pack3d_device_status.argtypes = [ip, _P]
         L.pack3d_last_launch_count.restype = ctypes.c_int
         L.pack3d_last_launch_count.argtypes = []
+        L.pack3d_testing_set_wait_budget.restype = ctypes.c_longlong
+        L.pack3d_testing_set_wait_budget.argtypes = [ctypes.c_longlong]
         _lib = L
     return _lib
 
@@ -352,6 +354,11 @@ def pack3d_device_status(index, stream=None):
 
 def pack3d_last_launch_count():
     return int(lib().pack3d_last_launch_count())
+
+
+def pack3d_testing_set_wait_budget(cycles):
+    """Testing hook: SM-cycle budget of the kernels' device-side waits (<= 0: default)."""
+    return int(lib().pack3d_testing_set_wait_budget(int(cycles)))
 
 
 def pack3d_strerror(status):

@@ -31,6 +31,7 @@ cudaError_t local_tc_dispatch(const pack3d_index& ix, const void* q, const void*
 cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void* k_rot,
                                const void* v, int64_t bh, float scale, void* o_loc,
                                float* lse_loc, cudaStream_t s);
+pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int heads);
 cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
                                float scale, int excl, void* o, float* lse_glob, void* o_glob,
@@ -39,10 +40,8 @@ cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void
 
 using namespace p3d;
 
-namespace {
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int heads) {
+// Checks shared by every operator call (also used by the no-alloc backward).
+pack3d_status p3d::check_common(const pack3d_index* idx, int dtype, int batch, int heads) {
   if (!idx || !idx->coord || !idx->nbr || !idx->members || !idx->rope)
     return PACK3D_ERR_INVALID_ARG;
   if (dtype != PACK3D_F32 && dtype != PACK3D_BF16) return PACK3D_ERR_INVALID_ARG;
@@ -51,6 +50,9 @@ pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int he
   if (idx->geom.head_dim != 48 && idx->geom.head_dim != 96) return PACK3D_ERR_UNSUPPORTED;
   return PACK3D_OK;
 }
+
+namespace {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 pack3d_status check_rows(std::initializer_list<const void*> ptrs) {
   for (const void* p : ptrs) {
@@ -62,21 +64,8 @@ pack3d_status check_rows(std::initializer_list<const void*> ptrs) {
 
 pack3d_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
 
-bool bf16_tensor_path();
-// the backward's global branch runs on tensor cores for bf16 (unless the CUDA-core path is
-// selected); float32 stays on CUDA cores for the 1e-4 bar
-bool bwd_tensor_path(int dtype) { return dtype == PACK3D_BF16 && bf16_tensor_path(); }
-
-// bf16 runs the global branch on tcgen05 tensor cores unless PACK3D_BF16_PATH=simt selects the
-// CUDA-core kernels (both compute the whole operator).
-bool bf16_tensor_path() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("PACK3D_BF16_PATH");
-    v = (e && strcmp(e, "simt") == 0) ? 0 : 1;
-  }
-  return v == 1;
-}
+// bf16 runs on tcgen05 tensor cores; float32 stays on CUDA cores for the 1e-4 bar (no TF32)
+bool tensor_path(int dtype) { return dtype == PACK3D_BF16; }
 }  // namespace
 
 extern "C" const char* pack3d_strerror(pack3d_status s) {
@@ -95,6 +84,10 @@ extern "C" const char* pack3d_strerror(pack3d_status s) {
 }
 
 extern "C" int pack3d_last_launch_count(void) { return g_launches; }
+
+extern "C" long long pack3d_testing_set_wait_budget(long long cycles) {
+  return wait_budget_store().exchange(cycles > 0 ? cycles : kDefaultWaitBudget);
+}
 
 extern "C" pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const void* v,
                                           int dtype, int batch, int heads, void* ksum,
@@ -125,7 +118,7 @@ namespace {
 pack3d_status run_local(const pack3d_index* idx, const void* q, const void* k, const void* v,
                         int dtype, int64_t bh, float scale, bool k_rotated, void* o_loc,
                         float* lse_loc, cudaStream_t s) {
-  if (dtype == PACK3D_BF16 && bf16_tensor_path())
+  if (tensor_path(dtype))
     return cuda_status(k_rotated ? local_tma_dispatch(*idx, q, k, v, bh, scale, o_loc, lse_loc, s)
                                  : local_tc_dispatch(*idx, q, k, v, bh, scale, o_loc, lse_loc, s));
   return cuda_status(local_simt_dispatch(*idx, q, k, v, dtype, bh, scale, o_loc, lse_loc, s));
@@ -136,7 +129,7 @@ pack3d_status run_global(const pack3d_index* idx, const void* q, const void* gat
                          const void* ksum, const void* vsum, const void* o_loc, int dtype,
                          int64_t bh, float scale, int excl, void* o, float* lse_glob,
                          void* o_glob, cudaStream_t s) {
-  if (dtype == PACK3D_BF16 && bf16_tensor_path())
+  if (tensor_path(dtype))
     return cuda_status(global_tc_dispatch(*idx, q, gate, ksum, vsum, o_loc, bh, scale, excl, o,
                                           lse_glob, o_glob, s));
   return cuda_status(global_simt_dispatch(*idx, q, gate, ksum, vsum, o_loc, dtype, bh, scale,
@@ -145,7 +138,7 @@ pack3d_status run_global(const pack3d_index* idx, const void* q, const void* gat
 
 pack3d_status check_flags(int dtype, uint32_t flags, uint32_t allowed) {
   if (flags & ~allowed) return PACK3D_ERR_INVALID_ARG;
-  if ((flags & PACK3D_K_ROTATED) && !(dtype == PACK3D_BF16 && bf16_tensor_path()))
+  if ((flags & PACK3D_K_ROTATED) && !tensor_path(dtype))
     return PACK3D_ERR_UNSUPPORTED;
   return PACK3D_OK;
 }
@@ -221,7 +214,7 @@ extern "C" size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int b
 extern "C" size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch,
                                              int heads) {
   if (check_common(idx, dtype, batch, heads) != PACK3D_OK) return 0;
-  return bwd_workspace_bytes(*idx, (int64_t)batch * heads, dtype, bwd_tensor_path(dtype));
+  return bwd_workspace_bytes(*idx, (int64_t)batch * heads, dtype, tensor_path(dtype));
 }
 
 extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
@@ -242,7 +235,7 @@ extern "C" pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q,
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return PACK3D_ERR_ALIGN;
   if (!(scale > 0.f) || (flags & ~PACK3D_EXCLUDE_NEAR)) return PACK3D_ERR_INVALID_ARG;
   const int64_t bh = (int64_t)batch * heads;
-  const bool tc = bwd_tensor_path(dtype);
+  const bool tc = tensor_path(dtype);
   if (workspace_bytes < bwd_workspace_bytes(*idx, bh, dtype, tc)) return PACK3D_ERR_WORKSPACE;
   const int excl = (flags & PACK3D_EXCLUDE_NEAR) ? 1 : 0;
   return cuda_status(bwd_simt_dispatch(*idx, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc,

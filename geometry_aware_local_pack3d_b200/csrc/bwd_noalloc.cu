@@ -18,6 +18,11 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.h"
+
+namespace p3d {
+pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int heads);
+}
 
 namespace {
 constexpr size_t kScratchBytes = PACK3D_NOALLOC_SCRATCH_BYTES;
@@ -49,8 +54,12 @@ extern "C" pack3d_status pack3d_attn_bwd_noalloc(
     const void* ksum, const void* vsum, const void* o_loc, const void* o_glob,
     const float* lse_loc, const float* lse_glob, const void* dO, int dtype, int batch, int heads,
     float scale, uint32_t flags, void* dq, void* dk, void* dv, void* dgate, void* stream) {
+  // a rejected call launches nothing: the launch count reads 0 afterwards, and argument errors
+  // are the ones pack3d_attn_bwd reports for the same arguments
+  p3d::reset_launches();
+  const pack3d_status common = p3d::check_common(idx, dtype, batch, heads);
+  if (common != PACK3D_OK) return common;
   const size_t need = pack3d_bwd_workspace_bytes(idx, dtype, batch, heads);
-  if (need == 0) return PACK3D_ERR_INVALID_ARG;
   if (need > kScratchBytes) return PACK3D_ERR_WORKSPACE;  // problem too large for the buffer
   void* ws = nullptr;
   const pack3d_status st = scratch_address(&ws);

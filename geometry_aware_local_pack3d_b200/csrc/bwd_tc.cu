@@ -39,24 +39,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-struct Abort {
-  volatile int* flag;
-  int32_t* status;
-  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
-    if (tc::mbar_test_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!tc::mbar_test_wait(bar, parity)) {
-      if (nap) __nanosleep(32);
-      if (*flag) return false;
-      if (clock64() - t0 > 4000000000LL) {
-        *flag = 1;
-        set_status(status, PACK3D_ERR_TIMEOUT);
-        return false;
-      }
-    }
-    return true;
-  }
-};
 
 struct Params {
   pack3d_index ix;
@@ -74,6 +56,7 @@ struct Params {
   int64_t units, units_per_bh;  // dq: 128-query tiles
   int n_chunks;                 // dq: 64-summary chunks per (batch, head)
   int m_tiles, q_tiles, q_per_split;  // dsum: 128-summary tiles, 64-query tiles
+  long long wait_budget;              // SM cycles of each bounded wait
 };
 
 // summaries of block coordinates [z0, z1] x [y0, y1] x [x0, x1] are excluded for a query at
@@ -126,7 +109,7 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  btc::Abort ab{abort_flag, P.ix.status};
+  tc::Abort ab{abort_flag, P.ix.status, P.wait_budget};
   const int64_t N = P.ix.n;
   const int M = (int)P.ix.m;
   const int NC = P.n_chunks;
@@ -395,7 +378,7 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  btc::Abort ab{abort_flag, P.ix.status};
+  tc::Abort ab{abort_flag, P.ix.status, P.wait_budget};
   const int64_t N = P.ix.n;
   const int M = (int)P.ix.m;
   // work item: (batch*head, 128-summary tile, query range)
@@ -649,15 +632,12 @@ template <int D>
 cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* ksum,
                           const void* vsum, const float* lse_glob, int64_t bh, float scale,
                           int excl, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bdq::Smem<D>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(k_bwd_dsum_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bds::Smem<D>::kBytes) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr_dq{0}, attr_dsum{0};
+  if (smem_attr_once(reinterpret_cast<const void*>(k_bwd_dq_tc<D>), bdq::Smem<D>::kBytes,
+                     attr_dq) != cudaSuccess ||
+      smem_attr_once(reinterpret_cast<const void*>(k_bwd_dsum_tc<D>), bds::Smem<D>::kBytes,
+                     attr_dsum) != cudaSuccess)
+    return cudaErrorInvalidValue;
   btc::Params p;
   p.ix = ix;
   p.qtb = w.qtb;
@@ -669,6 +649,7 @@ cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* 
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.exclude_near = excl;
+  p.wait_budget = wait_budget_cycles();
   p.bh_count = bh;
   // summary gradients: (batch*head) x 128-summary tiles x query ranges
   p.m_tiles = (int)((ix.m + btc::kRows - 1) / btc::kRows);

@@ -101,6 +101,7 @@ struct Params {
   int units_per_bh;
   int n_chunks;
   int rope_in_smem;
+  long long wait_budget;       // SM cycles of each bounded wait
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -109,27 +110,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-struct Abort {
-  volatile int* flag;
-  int32_t* status;
-  // Probing wait (a suspended try_wait wakes up measurably later). With `nap`, a short
-  // nanosleep between probes leaves the issue slots of the SM sub-partition to the warps that
-  // are working, above all the single MMA-issuing thread; the issuer itself waits without it.
-  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
-    if (tc::mbar_test_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!tc::mbar_test_wait(bar, parity)) {
-      if (nap) __nanosleep(32);
-      if (*flag) return false;
-      if (clock64() - t0 > 4000000000LL) {
-        *flag = 1;
-        set_status(status, PACK3D_ERR_TIMEOUT);
-        return false;
-      }
-    }
-    return true;
-  }
-};
 
 }  // namespace gtc
 
@@ -147,7 +127,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
   volatile int* prod_ok = abort_flag + 1;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) P3D_TRACE(999);
-  Abort ab{abort_flag, P.ix.status};
+  tc::Abort ab{abort_flag, P.ix.status, P.wait_budget};
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -623,13 +603,10 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
                              float scale, int excl, void* o, float* lse_glob, void* o_glob,
                              cudaStream_t s) {
   using namespace gtc;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_global_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<D>::kBytes) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (smem_attr_once(reinterpret_cast<const void*>(k_global_tc<D>), Smem<D>::kBytes, attr_done) !=
+      cudaSuccess)
+    return cudaErrorInvalidValue;
   Params p;
   p.ix = ix;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -642,6 +619,7 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   p.lse_glob = lse_glob;
   p.scale_log2 = scale * kLog2e;
   p.exclude_near = excl;
+  p.wait_budget = wait_budget_cycles();
   p.units_per_bh = (int)((ix.n + kRows * kTiles - 1) / (kRows * kTiles));
   p.units = bh * p.units_per_bh;
   p.n_chunks = (int)((ix.m + kChunk - 1) / kChunk);

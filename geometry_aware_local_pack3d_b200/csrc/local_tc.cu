@@ -72,6 +72,7 @@ struct Params {
   int nbz, nby, nbx;  // bricks per axis
   int64_t tiles;      // batch * heads * bricks
   int rope_in_smem;   // the whole rotation table is copied to shared memory once per CTA
+  long long wait_budget;  // SM cycles of each bounded wait
 };
 
 // trace slots of the first four tiles a CTA processes (tracing builds only)
@@ -94,27 +95,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 
-struct Abort {
-  volatile int* flag;
-  int32_t* status;
-  // Probing wait (a suspended try_wait wakes up measurably later). With `nap`, a short
-  // nanosleep between probes leaves the issue slots of the SM sub-partition to the warps that
-  // are working; the MMA issuer waits without it.
-  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
-    if (tc::mbar_test_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!tc::mbar_test_wait(bar, parity)) {
-      if (nap) __nanosleep(32);
-      if (*flag) return false;
-      if (clock64() - t0 > 4000000000LL) {
-        *flag = 1;
-        set_status(status, PACK3D_ERR_TIMEOUT);
-        return false;
-      }
-    }
-    return true;
-  }
-};
 
 // 16 bytes of one row: rotate 4 (x0, x1) pairs of axis third `axis` by coordinate value cv.
 __device__ __forceinline__ uint4 rope16(uint4 x, const float* rope, int pairs, int cv, int p0) {
@@ -145,7 +125,7 @@ __global__ void __launch_bounds__(ltc::kThreads, 2) k_local_tc(const ltc::Params
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) P3D_TRACE(3000);
   if (tid == 0) P3D_TRACE_CLK(3910);
-  Abort ab{abort_flag, P.ix.status};
+  tc::Abort ab{abort_flag, P.ix.status, P.wait_budget};
   const pack3d_geom& g = P.ix.geom;
   const int64_t N = P.ix.n;
   const int64_t bricks = (int64_t)P.nbz * P.nby * P.nbx;
@@ -594,13 +574,10 @@ cudaError_t launch_local_tc(const pack3d_index& ix, const void* q, const void* k
                             int64_t bh, float scale, void* o_loc, float* lse_loc,
                             cudaStream_t s) {
   using namespace ltc;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_local_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<D>::kBytes) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (smem_attr_once(reinterpret_cast<const void*>(k_local_tc<D>), Smem<D>::kBytes, attr_done) !=
+      cudaSuccess)
+    return cudaErrorInvalidValue;
   Params p;
   p.ix = ix;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -609,6 +586,7 @@ cudaError_t launch_local_tc(const pack3d_index& ix, const void* q, const void* k
   p.o_loc = static_cast<__nv_bfloat16*>(o_loc);
   p.lse_loc = lse_loc;
   p.scale_log2 = scale * kLog2e;
+  p.wait_budget = wait_budget_cycles();
   p.nbz = (ix.geom.gz + BZ - 1) / BZ;
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;

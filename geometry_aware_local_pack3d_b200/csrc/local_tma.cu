@@ -124,6 +124,7 @@ struct Params {
   int nbz, nby, nbx;
   int box_tma;        // slot boxes by TMA (else plain loads)
   int64_t units;      // batch * heads * units per field
+  long long wait_budget;  // SM cycles of each bounded wait
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -146,25 +147,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 
-struct Abort {
-  volatile int* flag;
-  int32_t* status;
-  // probing wait; with `nap` a short sleep between probes leaves issue slots to working warps
-  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
-    if (tc::mbar_test_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!tc::mbar_test_wait(bar, parity)) {
-      if (nap) __nanosleep(32);
-      if (*flag) return false;
-      if (clock64() - t0 > 4000000000LL) {
-        *flag = 1;
-        set_status(status, PACK3D_ERR_TIMEOUT);
-        return false;
-      }
-    }
-    return true;
-  }
-};
 
 // clock64 trace slots of the first four units a CTA processes (tracing builds only)
 #define GTR(ti, off)                                       \
@@ -207,7 +189,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kBar + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kBar + 8 * B_COUNT + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  Abort ab{abort_flag, P.ix.status};
+  tc::Abort ab{abort_flag, P.ix.status, P.wait_budget};
   const pack3d_geom& g = P.ix.geom;
   const int64_t N = P.ix.n;
   const int64_t per_field = (int64_t)P.nbz * P.nby * P.nbx;
@@ -743,18 +725,16 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
                              const void* v, int64_t bh, float scale, void* o_loc, float* lse_loc,
                              cudaStream_t s) {
   using namespace lg;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_local_tma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<D>::kBytes) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (smem_attr_once(reinterpret_cast<const void*>(k_local_tma<D>), Smem<D>::kBytes, attr_done) !=
+      cudaSuccess)
+    return cudaErrorInvalidValue;
   Params p;
   p.ix = ix;
   p.o_loc = static_cast<__nv_bfloat16*>(o_loc);
   p.lse_loc = lse_loc;
   p.scale_log2 = scale * kLog2e;
+  p.wait_budget = wait_budget_cycles();
   p.nbz = (ix.geom.gz + BZ - 1) / BZ;
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;

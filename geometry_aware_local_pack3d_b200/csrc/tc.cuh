@@ -12,6 +12,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace p3d {
 namespace tc {
 
@@ -68,6 +70,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
   return true;
 }
+
+// Bounded, abortable wait of the warp-specialised kernels. `flag` is the CTA's abort word in
+// shared memory; `budget` is the launch's wait budget in SM clock cycles. A wait that runs out
+// records PACK3D_ERR_TIMEOUT in the status word and raises the flag, and every other role's
+// wait then returns false at once, so the CTA drains its copies and MMAs and exits; nothing
+// traps. The probe is a non-suspending test_wait (a suspended try_wait wakes measurably later);
+// with `nap`, a short nanosleep between probes leaves the issue slots of the SM sub-partition
+// to the warps that are working, above all the MMA issuers, which wait without it.
+struct Abort {
+  volatile int* flag;
+  int32_t* status;
+  long long budget;
+  __device__ bool wait(uint64_t* bar, uint32_t parity, bool nap = true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+      if (nap) __nanosleep(32);
+      if (*flag) return false;
+      if (clock64() - t0 > budget) {
+        *flag = 1;
+        set_status(status, PACK3D_ERR_TIMEOUT);
+        return false;
+      }
+    }
+    return true;
+  }
+};
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -236,6 +236,16 @@ pack3d_status pack3d_device_status(const pack3d_index* idx, void* stream);
  * this host thread (for launch accounting). */
 int pack3d_last_launch_count(void);
 
+/* TESTING HOOK (not part of the operator; the paper has no counterpart). Every device-side
+ * wait of the tensor-core kernels (a warp waiting for a copy, an MMA or another warp) gives up
+ * after a budget of SM clock cycles: it records PACK3D_ERR_TIMEOUT in the index's status word
+ * (read it with pack3d_device_status), the kernel drains its in-flight copies and MMAs, frees
+ * its tensor memory and returns, so the CUDA context stays usable. This sets the budget used
+ * by the launches that follow, process-wide (cycles <= 0 restores the default of 4e9 cycles)
+ * and returns the previous value. A tiny budget makes the next launches time out on purpose;
+ * it exists so that tests can exercise that path without faulting or hanging a GPU. */
+long long pack3d_testing_set_wait_budget(long long cycles);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,3 +47,25 @@ def test_committed_traffic_entries_name_existing_sources():
         for s in e["sources"]:
             assert os.path.exists(os.path.join(root, s)), s
         assert os.path.exists(os.path.join(root, e["capture"]))
+
+
+def test_step_roofline_of_the_headline_field():
+    w = inputs.WORKLOADS["field65k_bf16"]
+    e = 201326592
+    alg = bench.step_algorithmic(dict(w), index_bytes=8_000_000)
+    # q, k, v read and o written, gate read, summaries written and read back, tables
+    assert alg["bytes"] == 4 * e + 2 * 8 * 65536 * 2 + 4 * (2 * 8 * 1024 * 96 * 2) + 8_000_000
+    assert alg["flops"] == pytest.approx(412316860416.0)
+    peaks = dict(hbm=6508.8, bf16=1624.0, source="measured")
+    r = bench.step_roofline(alg, 1.0, peaks)
+    # tensor-bound: 412.3 GFLOP at 1,624 TFLOP/s is 0.2539 ms, more than 0.83 GB at 6.5 TB/s
+    assert r["bound"] == "tensor"
+    assert r["roofline_ms"] == pytest.approx(0.25389, rel=1e-4)
+    assert r["frac"] == pytest.approx(0.25389, rel=1e-4)  # the step took 1 ms
+    assert r["achieved"] == pytest.approx(412.3169, rel=1e-4)
+
+
+def test_cores_used_is_cpu_time_over_wall_time():
+    assert bench.cores_used(10.0, 10.2) == 1
+    assert bench.cores_used(10.0, 38.0) == 4
+    assert bench.cores_used(10.0, 0.1) == 1
