@@ -13,7 +13,9 @@ The line's `roofline` is the whole step's: the slower of the step's algorithmic 
 measured HBM peak and its global-contraction flops at the measured bf16 peak, against the step
 time; the per-kernel rooflines sit under `kernels` (and the slowest under
 `roofline.dominant_kernel`). On one GPU the same run also reports the forward + backward of
-the headline field (`fwd_bwd`, `attn_bwd`) and the 262,144-token field (`field262k_bf16`).
+the headline field (`fwd_bwd`, `attn_bwd`), the 262,144-token field (`field262k_bf16`) and the
+pages' 1M-token point (`field1m_bf16`: 64x128x128, 4,096 summaries after a second pooling
+stage).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pack3d|reference]
 
@@ -57,14 +59,16 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--skip-bwd", action="store_true",
                     help="skip the (untimed-step) backward and index-build measurements")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     return ap.parse_args()
 
 
 def workload_config(name, w):
     return {"workload": name, "grid": list(w["grid"]), "block": list(w["block"]),
             "batch": w["batch"], "heads": w["heads"], "head_dim": w["d"],
-            "tokens": int(np.prod(w["grid"])), "summaries": int(np.prod(
-                [-(-g // b) for g, b in zip(w["grid"], w["block"])])),
+            "tokens": int(np.prod(w["grid"])), "summaries": _sizes(w)[3],
+            "pool2": list(w.get("pool2", (1, 1, 1))),
             "packing": w["packing"], "exclude_near": w["exclude_near"],
             "l2": "inputs larger than L2: q, k, v alone are "
                   f"{3 * w['batch'] * w['heads'] * int(np.prod(w['grid'])) * w['d'] * 2 / 1e6:.0f}"
@@ -205,9 +209,12 @@ def kernel_traffic(kernel_key):
 
 
 def _sizes(w):
+    """B, H, N, M, d of a workload (M: the summaries the global branch attends to, after the
+    second pooling stage when there is one)."""
     B, H, d = w["batch"], w["heads"], w["d"]
     N = int(np.prod(w["grid"]))
-    M = int(np.prod([-(-g // b) for g, b in zip(w["grid"], w["block"])]))
+    pool2 = w.get("pool2", (1, 1, 1))
+    M = int(np.prod([-(-(-(-g // b)) // p) for g, b, p in zip(w["grid"], w["block"], pool2)]))
     return B, H, N, M, d
 
 
@@ -369,7 +376,7 @@ class Forward:
         self.p3d, self.w = p3d, w
         B, H, d = w["batch"], w["heads"], w["d"]
         dt = torch.bfloat16
-        self.geom = p3d.make_geom(w["grid"], w["block"], d)
+        self.geom = p3d.make_geom(w["grid"], w["block"], d, pool2=w.get("pool2", (1, 1, 1)))
         self.ix = p3d.pack3d_build_index(self.geom, coords=torch.from_numpy(w["coords"]).to(dev))
         self.q, self.k, self.v, self.a = (w[n].to(dt).to(dev).contiguous() for n in "qkva")
         self.ksum = torch.empty(p3d.summary_tiles_shape(self.ix, B, H, d), dtype=dt, device=dev)
@@ -484,7 +491,12 @@ def main():
                                 device_id=dev)
     sync = dist.barrier if world > 1 else None
 
-    w = inputs.make_workload(args.workload)
+    if args.batch is not None:
+        cfg = dict(inputs.WORKLOADS[args.workload])
+        cfg["batch"] = args.batch
+        w = inputs.make_workload(cfg)
+    else:
+        w = inputs.make_workload(args.workload)
     B, H, N, M, d = _sizes(w)
     F = Forward(p3d, w, dev)
 
@@ -579,40 +591,83 @@ def main():
                        "kernels": kern2, "steps": 10, "warmup": 3,
                        "data": "synthetic, drawn on the device (seeded CUDA generator)"}
         del F2, w2
+        torch.cuda.empty_cache()
 
-    # end to end through the public API with host buffers: H2D of the inputs and D2H of o
+        # the pages' high-token point: 1,048,576 tokens, 4,096 summaries per KV head
+        name = "field1m_bf16"
+        w3 = device_workload(name, dev)
+        F3 = Forward(p3d, w3, dev)
+        ms3, ms3_k, _ = F3.time(5, 2)
+        roof3, kern3 = forward_line(w3, name, ms3, ms3_k, F3.index_bytes(), peaks)
+        B3, H3, N3, _, _ = _sizes(w3)
+        extra[name] = {"config": workload_config(name, w3), "ms_per_step": ms3,
+                       "tokens_per_s": B3 * N3 / (ms3 / 1e3), "roofline": roof3,
+                       "kernels": kern3, "steps": 5, "warmup": 2,
+                       "data": "synthetic, drawn on the device (seeded CUDA generator)"}
+        del F3, w3
+        torch.cuda.empty_cache()
+
+    # End to end through the public API with host buffers: every step copies its inputs q, k,
+    # v, a from pinned host memory to the device and its output o back. Steps are pipelined as
+    # a serving loop would run them: two device input/output sets, host->device copies on one
+    # stream, the operator on the compute stream, device->host copies on a third, so a step's
+    # input upload, the previous step's compute and an earlier step's download overlap (PCIe
+    # is full duplex). The timed region runs from the first upload to the last download.
     e2e = None
     if not args.skip_e2e:
         dt = torch.bfloat16
         hq, hk, hv, ha = (t.to(dt).pin_memory() for t in (w["q"], w["k"], w["v"], w["a"]))
-        ho = torch.empty(F.o.shape, dtype=dt).pin_memory()
+        ho = [torch.empty(F.o.shape, dtype=dt).pin_memory() for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha))
-        d2h = ho.numel() * ho.element_size()
+        d2h = ho[0].numel() * ho[0].element_size()
+        sets = [dict(q=F.q, k=F.k, v=F.v, a=F.a, o=F.o)]
+        sets.append({n: torch.empty_like(sets[0][n]) for n in ("q", "k", "v", "a", "o")})
+        s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
+        s_comp = F.stream
 
-        def e2e_step():
-            F.q.copy_(hq, non_blocking=True)
-            F.k.copy_(hk, non_blocking=True)
-            F.v.copy_(hv, non_blocking=True)
-            F.a.copy_(ha, non_blocking=True)
-            F.step()
-            ho.copy_(F.o, non_blocking=True)
+        def e2e_run(k_steps):
+            up = [torch.cuda.Event() for _ in range(k_steps)]
+            done = [torch.cuda.Event() for _ in range(k_steps)]
+            down = [torch.cuda.Event() for _ in range(k_steps)]
+            for i in range(k_steps):
+                bufs = sets[i % 2]
+                with torch.cuda.stream(s_up):
+                    if i >= 2:
+                        s_up.wait_event(done[i - 2])  # the set's previous compute has read it
+                    for n, h in (("q", hq), ("k", hk), ("v", hv), ("a", ha)):
+                        bufs[n].copy_(h, non_blocking=True)
+                    up[i].record(s_up)
+                s_comp.wait_event(up[i])
+                if i >= 2:
+                    s_comp.wait_event(down[i - 2])  # the set's previous output has left
+                F.q, F.k, F.v, F.a, F.o = (bufs[n] for n in ("q", "k", "v", "a", "o"))
+                F.step()
+                done[i].record(s_comp)
+                with torch.cuda.stream(s_down):
+                    s_down.wait_event(done[i])
+                    ho[i % 2].copy_(bufs["o"], non_blocking=True)
+                    down[i].record(s_down)
+            return down[-1]
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         k_e2e = max(3, min(args.steps, 10))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(F.stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        e1.record(F.stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_up)
+        last = e2e_run(k_e2e)
+        s_down.wait_event(last)
+        e1.record(s_down)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / k_e2e
         ems = max_over_ranks([ems], dist if world > 1 else None, dev)[0]
+        F.q, F.k, F.v, F.a, F.o = (sets[0][n] for n in ("q", "k", "v", "a", "o"))
         e2e = {"value": job_throughput(world, B * N, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e}
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e,
+               "pipelining": "uploads, compute and downloads of consecutive steps overlap on "
+                             "three streams (two device input/output sets)"}
 
     if rank == 0:
         roof, kernels = forward_line(w, args.workload, ms, ms_k, F.index_bytes(), peaks)

@@ -20,6 +20,8 @@ PACK3D_F32 = 0
 PACK3D_BF16 = 1
 PACK3D_EXCLUDE_NEAR = 1
 PACK3D_K_ROTATED = 2
+PACK3D_ROPE_TOKEN = 0
+PACK3D_ROPE_CENTRE = 1
 
 STATUS_NAMES = {0: "PACK3D_OK", 1: "PACK3D_ERR_INVALID_ARG", 2: "PACK3D_ERR_UNSUPPORTED",
                 3: "PACK3D_ERR_DUP_COORD", 4: "PACK3D_ERR_COORD_RANGE", 5: "PACK3D_ERR_ALIGN",
@@ -36,7 +38,9 @@ class Pack3DError(RuntimeError):
 class pack3d_geom(ctypes.Structure):
     _fields_ = [("gz", ctypes.c_int32), ("gy", ctypes.c_int32), ("gx", ctypes.c_int32),
                 ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("rope_base", ctypes.c_float)]
+                ("head_dim", ctypes.c_int32), ("rope_base", ctypes.c_float),
+                ("pz", ctypes.c_int32), ("py", ctypes.c_int32), ("px", ctypes.c_int32),
+                ("summary_rope", ctypes.c_int32), ("spacing", ctypes.c_float * 3)]
 
 
 _P = ctypes.c_void_p
@@ -44,10 +48,14 @@ _P = ctypes.c_void_p
 
 class pack3d_index(ctypes.Structure):
     _fields_ = [("geom", pack3d_geom), ("n", ctypes.c_int64), ("m", ctypes.c_int64),
-                ("block_volume", ctypes.c_int32), ("rope_pairs", ctypes.c_int32),
-                ("rope_rows", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_blocks", ctypes.c_int64), ("block_volume", ctypes.c_int32),
+                ("rope_pairs", ctypes.c_int32), ("rope_rows", ctypes.c_int32),
+                ("group_volume", ctypes.c_int32), ("sum_ext", ctypes.c_int32 * 3),
+                ("sum_grid", ctypes.c_int32 * 3), ("n_empty", ctypes.c_int32),
+                ("reserved", ctypes.c_int32),
                 ("coord", _P), ("inv", _P), ("nbr", _P), ("block_of", _P), ("slot_of", _P),
-                ("members", _P), ("count", _P), ("rope", _P), ("status", _P)]
+                ("members", _P), ("count", _P), ("sum_of", _P), ("groups", _P),
+                ("count2", _P), ("empty", _P), ("rope", _P), ("rope_c", _P), ("status", _P)]
 
 
 _lib = None
@@ -74,24 +82,24 @@ def lib():
         L.pack3d_summarize.argtypes = [ip, _P, _P, st, st, st, _P, _P, _P]
         L.pack3d_attn_fwd.restype = st
         L.pack3d_attn_local.restype = st
-        L.pack3d_attn_local.argtypes = [ip, _P, _P, _P, st, st, st, f32, u32, _P, _P, _P]
+        L.pack3d_attn_local.argtypes = [ip, _P, _P, _P, st, st, st, st, f32, u32, _P, _P, _P]
         L.pack3d_attn_global.restype = st
-        L.pack3d_attn_global.argtypes = [ip, _P, _P, _P, _P, _P, st, st, st, f32, u32, _P, _P,
-                                         _P, _P]
+        L.pack3d_attn_global.argtypes = [ip, _P, _P, _P, _P, _P, st, st, st, st, f32, u32, _P,
+                                         _P, _P, _P]
         L.pack3d_summarize_rotated.restype = st
         L.pack3d_summarize_rotated.argtypes = [ip, _P, _P, st, st, st, _P, _P, _P, _P]
-        L.pack3d_attn_fwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, st, st, st, f32, u32, _P, _P,
-                                      _P, _P, _P, _P]
+        L.pack3d_attn_fwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, st, st, st, st, f32, u32, _P,
+                                      _P, _P, _P, _P, _P]
         L.pack3d_summary_bytes.restype = sz
         L.pack3d_summary_bytes.argtypes = [ip, st, st, st]
         L.pack3d_bwd_workspace_bytes.restype = sz
-        L.pack3d_bwd_workspace_bytes.argtypes = [ip, st, st, st]
+        L.pack3d_bwd_workspace_bytes.argtypes = [ip, st, st, st, st]
         L.pack3d_attn_bwd.restype = st
         L.pack3d_attn_bwd.argtypes = [ip, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, st, st, st,
-                                      f32, u32, _P, _P, _P, _P, _P, sz, _P]
+                                      st, f32, u32, _P, _P, _P, _P, _P, sz, _P]
         L.pack3d_attn_bwd_noalloc.restype = st
         L.pack3d_attn_bwd_noalloc.argtypes = [ip, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, st,
-                                              st, st, f32, u32, _P, _P, _P, _P, _P]
+                                              st, st, st, f32, u32, _P, _P, _P, _P, _P]
         L.pack3d_device_status.restype = st
         L.pack3d_device_status.argtypes = [ip, _P]
         L.pack3d_last_launch_count.restype = ctypes.c_int
@@ -153,15 +161,29 @@ class Index:
         return self.buf[off:off + 4 * count].view(torch.int32).view(*shape)
 
     def rope_table(self):
+        """[3 axes, rope_rows, pairs, 2] (cos, sin) of the per-axis RoPE angles."""
         base = self.buf.data_ptr()
         off = self.struct.rope - base
         rows, pairs = int(self.struct.rope_rows), int(self.struct.rope_pairs)
-        return self.buf[off:off + 8 * rows * pairs].view(torch.float32).view(rows, pairs, 2)
+        return self.buf[off:off + 24 * rows * pairs].view(torch.float32).view(3, rows, pairs, 2)
+
+    def centre_table(self):
+        """[M, d/2, 2] (cos, sin) of the summary-centre angles."""
+        base = self.buf.data_ptr()
+        off = self.struct.rope_c - base
+        m, half = self.m, int(self.struct.geom.head_dim) // 2
+        return self.buf[off:off + 8 * m * half].view(torch.float32).view(m, half, 2)
 
 
-def make_geom(grid, block, head_dim, rope_base=10000.0):
+def make_geom(grid, block, head_dim, rope_base=10000.0, pool2=(1, 1, 1), summary_rope="token",
+              spacing=(1.0, 1.0, 1.0)):
+    """pool2: second pooling stage (groups of blocks); summary_rope: "token" or "centre";
+    spacing: per-axis scale of the RoPE coordinate."""
+    sr = {"token": PACK3D_ROPE_TOKEN, "centre": PACK3D_ROPE_CENTRE}[summary_rope]
     return pack3d_geom(int(grid[0]), int(grid[1]), int(grid[2]), int(block[0]), int(block[1]),
-                       int(block[2]), int(head_dim), float(rope_base))
+                       int(block[2]), int(head_dim), float(rope_base), int(pool2[0]),
+                       int(pool2[1]), int(pool2[2]), sr,
+                       (ctypes.c_float * 3)(*[float(x) for x in spacing]))
 
 
 def pack3d_index_bytes(geom, n):
@@ -263,9 +285,10 @@ def pack3d_attn_fwd(index, q, k, v, gate, ksum, vsum, *, scale=None, exclude_nea
         o_glob = torch.empty_like(q) if o_glob is None else o_glob
     flags = (PACK3D_EXCLUDE_NEAR if exclude_near else 0) | (PACK3D_K_ROTATED if k_rotated else 0)
     _check(lib().pack3d_attn_fwd(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
-                                 _ptr(gate), _ptr(ksum), _ptr(vsum), _dtype_code(q), B, H, scale,
-                                 flags, _ptr(o), _ptr(lse_loc), _ptr(lse_glob), _ptr(o_loc),
-                                 _ptr(o_glob), _stream(stream)), "pack3d_attn_fwd")
+                                 _ptr(gate), _ptr(ksum), _ptr(vsum), _dtype_code(q), B, H,
+                                 k.shape[1], scale, flags, _ptr(o), _ptr(lse_loc),
+                                 _ptr(lse_glob), _ptr(o_loc), _ptr(o_glob), _stream(stream)),
+           "pack3d_attn_fwd")
     return dict(o=o, lse_loc=lse_loc, lse_glob=lse_glob, o_loc=o_loc, o_glob=o_glob)
 
 
@@ -279,14 +302,15 @@ def pack3d_attn_local(index, q, k, v, *, scale=None, k_rotated=False, o_loc=None
         o_loc = torch.empty_like(q)
     flags = PACK3D_K_ROTATED if k_rotated else 0
     _check(lib().pack3d_attn_local(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
-                                   _dtype_code(q), B, H, scale, flags, _ptr(o_loc),
+                                   _dtype_code(q), B, H, k.shape[1], scale, flags, _ptr(o_loc),
                                    _ptr(lse_loc), _stream(stream)), "pack3d_attn_local")
     return o_loc, lse_loc
 
 
 def pack3d_attn_global(index, q, gate, ksum, vsum, o_loc, *, scale=None, exclude_near=False,
                        o=None, lse_glob=None, o_glob=None, stream=None):
-    """Global branch + mixer over a given o_loc (o may be o_loc itself): returns o."""
+    """Global branch + mixer over a given o_loc (o may be o_loc itself): returns o. The
+    summaries' head count (ksum.shape[1]) is the KV head count."""
     _need_cuda(q, gate, ksum, vsum, o_loc)
     B, H, N, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -294,15 +318,16 @@ def pack3d_attn_global(index, q, gate, ksum, vsum, o_loc, *, scale=None, exclude
         o = torch.empty_like(q)
     flags = PACK3D_EXCLUDE_NEAR if exclude_near else 0
     _check(lib().pack3d_attn_global(ctypes.byref(index.struct), _ptr(q), _ptr(gate), _ptr(ksum),
-                                    _ptr(vsum), _ptr(o_loc), _dtype_code(q), B, H, scale, flags,
-                                    _ptr(o), _ptr(lse_glob), _ptr(o_glob), _stream(stream)),
-           "pack3d_attn_global")
+                                    _ptr(vsum), _ptr(o_loc), _dtype_code(q), B, H, ksum.shape[1],
+                                    scale, flags, _ptr(o), _ptr(lse_glob), _ptr(o_glob),
+                                    _stream(stream)), "pack3d_attn_global")
     return o
 
 
-def pack3d_bwd_workspace_bytes(index, dtype_code, batch, heads):
+def pack3d_bwd_workspace_bytes(index, dtype_code, batch, heads, kv_heads=0):
     st = index.struct if isinstance(index, Index) else index
-    return int(lib().pack3d_bwd_workspace_bytes(ctypes.byref(st), dtype_code, batch, heads))
+    return int(lib().pack3d_bwd_workspace_bytes(ctypes.byref(st), dtype_code, batch, heads,
+                                                kv_heads))
 
 
 def pack3d_attn_bwd(index, q, k, v, gate, ksum, vsum, saved, dO, *, scale=None,
@@ -312,7 +337,7 @@ def pack3d_attn_bwd(index, q, k, v, gate, ksum, vsum, saved, dO, *, scale=None,
     B, H, N, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     code = _dtype_code(q)
-    nbytes = pack3d_bwd_workspace_bytes(index, code, B, H)
+    nbytes = pack3d_bwd_workspace_bytes(index, code, B, H, k.shape[1])
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -321,9 +346,10 @@ def pack3d_attn_bwd(index, q, k, v, gate, ksum, vsum, saved, dO, *, scale=None,
     _check(lib().pack3d_attn_bwd(ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(gate), _ptr(ksum), _ptr(vsum), _ptr(saved["o_loc"]),
                                  _ptr(saved["o_glob"]), _ptr(saved["lse_loc"]),
-                                 _ptr(saved["lse_glob"]), _ptr(dO), code, B, H, scale, flags,
-                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(workspace),
-                                 workspace.numel(), _stream(stream)), "pack3d_attn_bwd")
+                                 _ptr(saved["lse_glob"]), _ptr(dO), code, B, H, k.shape[1],
+                                 scale, flags, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+           "pack3d_attn_bwd")
     return dict(dq=dq, dk=dk, dv=dv, dgate=dgate)
 
 
@@ -340,8 +366,8 @@ def pack3d_attn_bwd_noalloc(index, q, k, v, gate, ksum, vsum, saved, dO, *, scal
                                          _ptr(gate), _ptr(ksum), _ptr(vsum), _ptr(saved["o_loc"]),
                                          _ptr(saved["o_glob"]), _ptr(saved["lse_loc"]),
                                          _ptr(saved["lse_glob"]), _ptr(dO), _dtype_code(q), B, H,
-                                         scale, flags, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate),
-                                         _stream(stream)), "pack3d_attn_bwd_noalloc")
+                                         k.shape[1], scale, flags, _ptr(dq), _ptr(dk), _ptr(dv),
+                                         _ptr(dgate), _stream(stream)), "pack3d_attn_bwd_noalloc")
     return dict(dq=dq, dk=dk, dv=dv, dgate=dgate)
 
 

@@ -11,10 +11,10 @@
 // Backward (paper summary §3.4), one warp per row, lanes over head dims:
 //   k_bwd_prep    rotated q, k; dgate; D_loc = <g dO, o_loc>, D_glob = <(1-g) dO, o_glob>.
 //   k_bwd_dsum    dK_sum[m] = sum_i dS_im q~_i and dV_sum[m] = sum_i P_im (1-g_i) dO_i.
-//   k_bwd_dq      dq = R(c)^T (sum_j dS_ij k~_j + sum_m dS_im K_sum[m]); 8 lanes per row.
+//   k_bwd_dq      dq = R(c)^T (sum_j dS_ij k~_j + sum_m dS_im K_sum[m]); 4 lanes per row.
 //   k_bwd_dkv     dk, dv gathered over the key's own neighbourhood (the 3x3x3 relation is
 //                 symmetric, so no scatter/atomics) plus 1/|S| of its block's summary grads;
-//                 8 lanes per row.
+//                 4 lanes per row.
 // On the bf16 tensor-core path the global branch's summary gradients and its part of dq come
 // from the kernels of bwd_tc.cu instead of k_bwd_dsum and the summary loop of k_bwd_dq.
 // Every reduction order depends on coordinates (offset order, canonical slots, summary ids),
@@ -62,7 +62,7 @@ __device__ __forceinline__ void rotate_row(const pack3d_index& ix, const Coord& 
 #pragma unroll
   for (int e = 0; e < D; e += 2) {
     const int axis = e / DA, p = (e % DA) / 2;
-    const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+    const float2 cs = rope_cs(ix.rope, ix.rope_rows, ix.rope_pairs, axis, coord_axis(c, axis), p);
     const float sn = sign * cs.y;
     const float x0 = x[e], x1 = x[e + 1];
     x[e] = x0 * cs.x - x1 * sn;
@@ -75,12 +75,13 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) k_local_fwd(pack3d_index ix, const T* __restrict__ q,
                                                    const T* __restrict__ k,
                                                    const T* __restrict__ v, float scale,
-                                                   T* __restrict__ o_loc,
+                                                   int kv_group, T* __restrict__ o_loc,
                                                    float* __restrict__ lse_loc) {
   const int64_t bh = blockIdx.y;
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= ix.n) return;
   const int64_t rowbase = bh * ix.n;
+  const int64_t kvbase = kv_of(bh, kv_group) * ix.n;  // keys and values of the KV head
   const Coord ci = decode(ix.coord[i]);
   float qr[D];
   load_row<T, D>(q + (rowbase + i) * D, qr);
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(128) k_local_fwd(pack3d_index ix, const T* __r
     s[o] = -INFINITY;
     if (j < 0) continue;
     float kr[D];
-    load_row<T, D>(k + (rowbase + j) * D, kr);
+    load_row<T, D>(k + (kvbase + j) * D, kr);
     rotate_row<D>(ix, decode(ix.coord[j]), kr, 1.f);
     float dot = 0.f;
 #pragma unroll
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(128) k_local_fwd(pack3d_index ix, const T* __r
     const float p = exp2f(s[o] - mx);
     l += p;
     float vr[D];
-    load_row<T, D>(v + (rowbase + j) * D, vr);
+    load_row<T, D>(v + (kvbase + j) * D, vr);
 #pragma unroll
     for (int e = 0; e < D; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
   }
@@ -130,7 +131,8 @@ template <typename T, int D, int CH>
 __global__ void __launch_bounds__(128) k_global_fwd(
     pack3d_index ix, const T* __restrict__ q, const T* __restrict__ ksum,
     const T* __restrict__ vsum, const T* __restrict__ gate, const T* o_loc_in, float scale,
-    int exclude_near, T* o, float* __restrict__ lse_glob, T* __restrict__ o_glob_out) {
+    int exclude_near, int kv_group, T* o, float* __restrict__ lse_glob,
+    T* __restrict__ o_glob_out) {
   __shared__ float sk[CH][D];
   __shared__ float sv[CH][D];
   const int64_t bh = blockIdx.y;
@@ -156,13 +158,14 @@ __global__ void __launch_bounds__(128) k_global_fwd(
     const int cnt = min(CH, M - m0);
     __syncthreads();
     for (int t = threadIdx.x; t < cnt * D; t += blockDim.x) {
-      const int64_t off = sum_index(bh, m0 + t / D, t % D, D, MT);
+      const int64_t off = sum_index(kv_of(bh, kv_group), m0 + t / D, t % D, D, MT);
       sk[t / D][t % D] = to_f(ksum[off]);
       sv[t / D][t % D] = to_f(vsum[off]);
     }
     __syncthreads();
     if (!live) continue;
     for (int mm = 0; mm < cnt; ++mm) {
+      if (summary_empty(ix, m0 + mm)) continue;  // no member: in no softmax
       if (exclude_near && block_is_near(ix, m0 + mm, ci)) continue;
       float dot = 0.f;
 #pragma unroll
@@ -261,7 +264,8 @@ __device__ __forceinline__ void wr_rotate(const pack3d_index& ix, const Coord& c
     const float partner = __shfl_xor_sync(0xffffffffu, r.x[t], 1);
     if (e < D) {
       const int axis = e / DA, p = (e % DA) / 2;
-      const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+      const float2 cs =
+          rope_cs(ix.rope, ix.rope_rows, ix.rope_pairs, axis, coord_axis(c, axis), p);
       const float sn = sign * cs.y;
       // even e: x0' = x0 c - x1 s ; odd e: x1' = x0 s + x1 c
       r.x[t] = (e & 1) ? fmaf(partner, sn, r.x[t] * cs.x) : fmaf(-partner, sn, r.x[t] * cs.x);
@@ -269,49 +273,79 @@ __device__ __forceinline__ void wr_rotate(const pack3d_index& ix, const Coord& c
   }
 }
 
-// Group layout for the neighbour loops of the backward: 8 lanes per row, 4 rows per warp;
-// lane g of a group owns the KD = d/8 consecutive dims [g KD, g KD + KD). Dot products reduce
-// over the 8 lanes in 3 shuffle steps, and every rotation pair (2p, 2p+1) stays in one lane.
+// Group layout for the neighbour loops of the backward: kGL = 4 lanes per row, 8 rows per
+// warp; lane g of a group owns the KD = d/4 consecutive dims [g KD, g KD + KD), read and
+// written as 16-byte vectors (8-byte ones when a lane's share is 24 bytes). Dot products reduce
+// over the 4 lanes in 2 shuffle steps, and every rotation pair (2p, 2p+1) stays in one lane.
+constexpr int kGL = 4;
 template <int D> struct GRow {
-  static constexpr int KD = D / 8;
+  static constexpr int KD = D / kGL;
   static_assert(KD % 2 == 0, "a lane must own whole rotation pairs");
   float x[KD];
 };
-template <typename T> struct Pair2;
-template <> struct Pair2<float> {
-  __device__ static float2 get(const float* p, int k) { return reinterpret_cast<const float2*>(p)[k]; }
-  __device__ static void put(float* p, int k, float a, float b) {
-    reinterpret_cast<float2*>(p)[k] = make_float2(a, b);
-  }
+// Bytes per vector access of a lane's KD elements of type T: the largest of 16, 8, 4 dividing
+// the lane's share (the share starts on a multiple of it, as rows are 16-byte aligned).
+template <typename T, int KD> constexpr int gr_chunk() {
+  return (KD * (int)sizeof(T)) % 16 == 0 ? 16 : ((KD * (int)sizeof(T)) % 8 == 0 ? 8 : 4);
+}
+template <typename T> struct Unpack;
+template <> struct Unpack<float> {
+  __device__ __forceinline__ static void to_f(uint32_t w, float* x, int& n) { x[n++] = __uint_as_float(w); }
+  __device__ __forceinline__ static uint32_t from_f(const float* x, int& n) { return __float_as_uint(x[n++]); }
 };
-template <> struct Pair2<__nv_bfloat16> {
-  __device__ static float2 get(const __nv_bfloat16* p, int k) {
-    return __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(p)[k]);
+template <> struct Unpack<__nv_bfloat16> {
+  __device__ __forceinline__ static void to_f(uint32_t w, float* x, int& n) {
+    x[n++] = __uint_as_float(w << 16);
+    x[n++] = __uint_as_float(w & 0xffff0000u);
   }
-  __device__ static void put(__nv_bfloat16* p, int k, float a, float b) {
-    reinterpret_cast<__nv_bfloat162*>(p)[k] = __floats2bfloat162_rn(a, b);
+  __device__ __forceinline__ static uint32_t from_f(const float* x, int& n) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x[n], x[n + 1]);
+    n += 2;
+    return *reinterpret_cast<const uint32_t*>(&h);
   }
 };
 template <typename T, int D>
 __device__ __forceinline__ void gr_load(const T* __restrict__ row, GRow<D>& r, int g) {
-  const T* p = row + g * GRow<D>::KD;
+  constexpr int KD = GRow<D>::KD, CH = gr_chunk<T, KD>(), WORDS = CH / 4;
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(row + g * KD);
+  int n = 0;
 #pragma unroll
-  for (int k = 0; k < GRow<D>::KD / 2; ++k) {
-    const float2 v = Pair2<T>::get(p, k);
-    r.x[2 * k] = v.x;
-    r.x[2 * k + 1] = v.y;
+  for (int c = 0; c < KD * (int)sizeof(T) / CH; ++c) {
+    uint32_t w[4];
+    if (CH == 16) {
+      const uint4 t = __ldg(reinterpret_cast<const uint4*>(p) + c);
+      w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    } else if (CH == 8) {
+      const uint2 t = __ldg(reinterpret_cast<const uint2*>(p) + c);
+      w[0] = t.x; w[1] = t.y;
+    } else {
+      w[0] = __ldg(p + c);
+    }
+#pragma unroll
+    for (int k = 0; k < WORDS; ++k) Unpack<T>::to_f(w[k], r.x, n);
   }
 }
 template <typename T, int D>
 __device__ __forceinline__ void gr_store(T* row, const GRow<D>& r, int g) {
-  T* p = row + g * GRow<D>::KD;
+  constexpr int KD = GRow<D>::KD, CH = gr_chunk<T, KD>(), WORDS = CH / 4;
+  uint32_t* p = reinterpret_cast<uint32_t*>(row + g * KD);
+  int n = 0;
 #pragma unroll
-  for (int k = 0; k < GRow<D>::KD / 2; ++k) Pair2<T>::put(p, k, r.x[2 * k], r.x[2 * k + 1]);
+  for (int c = 0; c < KD * (int)sizeof(T) / CH; ++c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < WORDS; ++k) w[k] = Unpack<T>::from_f(r.x, n);
+    if (CH == 16)
+      reinterpret_cast<uint4*>(p)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    else if (CH == 8)
+      reinterpret_cast<uint2*>(p)[c] = make_uint2(w[0], w[1]);
+    else
+      p[c] = w[0];
+  }
 }
 __device__ __forceinline__ float group_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);
   x += __shfl_xor_sync(0xffffffffu, x, 2);
-  x += __shfl_xor_sync(0xffffffffu, x, 4);
   return x;
 }
 template <int D>
@@ -330,7 +364,7 @@ __device__ __forceinline__ void gr_rotate(const pack3d_index& ix, const Coord& c
   for (int k = 0; k < GRow<D>::KD; k += 2) {
     const int e = g * GRow<D>::KD + k;
     const int axis = e / DA, p = (e % DA) / 2;
-    const float2 cs = rope_cs(ix.rope, ix.rope_pairs, coord_axis(c, axis), p);
+    const float2 cs = rope_cs(ix.rope, ix.rope_rows, ix.rope_pairs, axis, coord_axis(c, axis), p);
     const float sn = sign * cs.y, x0 = r.x[k], x1 = r.x[k + 1];
     r.x[k] = x0 * cs.x - x1 * sn;
     r.x[k + 1] = x0 * sn + x1 * cs.x;
@@ -344,16 +378,18 @@ __global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __re
                                                   const T* __restrict__ o_loc,
                                                   const T* __restrict__ o_glob,
                                                   const T* __restrict__ dO, int64_t rows,
-                                                  BwdWork w, T* __restrict__ dgate) {
+                                                  int kv_group, BwdWork w,
+                                                  T* __restrict__ dgate) {
   const int lane = threadIdx.x & 31;
   const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int64_t i = row % ix.n;
+  const int64_t kvrow = kv_of(row / ix.n, kv_group) * ix.n + i;  // the key of the KV head
   const Coord c = decode(ix.coord[i]);
   WarpRow<D> a, b, d;
   wr_load<T, D>(q + row * D, a, lane);
   wr_rotate<D>(ix, c, a, lane, 1.f);
-  wr_load<T, D>(k + row * D, b, lane);
+  wr_load<T, D>(k + kvrow * D, b, lane);
   wr_rotate<D>(ix, c, b, lane, 1.f);
   T* qr = static_cast<T*>(w.qr);
   T* kr = static_cast<T*>(w.kr);
@@ -392,7 +428,7 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
                                                   const T* __restrict__ dO,
                                                   const float* __restrict__ lse_glob,
                                                   float scale, int exclude_near, int64_t bh_count,
-                                                  BwdWork w) {
+                                                  int kv_group, BwdWork w) {
   const int lane = threadIdx.x & 31;
   const int64_t task = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t M = ix.m;
@@ -400,8 +436,8 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
   const int64_t bh = task / M;
   const int m = (int)(task % M);
   WarpRow<D> km, vm, ak, av, x, d;
-  wr_load_sum<T, D>(ksum, bh, m, sum_tiles(M), km, lane);
-  wr_load_sum<T, D>(vsum, bh, m, sum_tiles(M), vm, lane);
+  wr_load_sum<T, D>(ksum, kv_of(bh, kv_group), m, sum_tiles(M), km, lane);
+  wr_load_sum<T, D>(vsum, kv_of(bh, kv_group), m, sum_tiles(M), vm, lane);
 #pragma unroll
   for (int t = 0; t < WarpRow<D>::KT; ++t) ak.x[t] = av.x[t] = 0.f;
   for (int64_t i = 0; i < ix.n; ++i) {
@@ -432,7 +468,7 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
   }
 }
 
-// dq = R(c)^T (sum_j dS_ij k~_j + global part); 8 lanes per query row.
+// dq = R(c)^T (sum_j dS_ij k~_j + global part); kGL lanes per query row.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __restrict__ v,
                                                 const T* __restrict__ ksum,
@@ -441,14 +477,14 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
                                                 const T* __restrict__ dO,
                                                 const float* __restrict__ lse_loc,
                                                 const float* __restrict__ lse_glob, float scale,
-                                                int exclude_near, int64_t rows, BwdWork w,
-                                                T* __restrict__ dq) {
-  const int g = threadIdx.x & 7;
-  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x >> 3) + (threadIdx.x >> 3);
+                                                int exclude_near, int64_t rows, int kv_group,
+                                                BwdWork w, T* __restrict__ dq) {
+  const int g = threadIdx.x & (kGL - 1);
+  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x / kGL) + threadIdx.x / kGL;
   const bool active = row0 < rows;  // inactive groups follow along on row 0 and store nothing
   const int64_t row = active ? row0 : 0;
   const int64_t bh = row / ix.n, i = row % ix.n;
-  const int64_t rowbase = bh * ix.n;
+  const int64_t rowbase = bh * ix.n, kvbase = kv_of(bh, kv_group) * ix.n;
   const Coord c = decode(ix.coord[i]);
   const float gt = 1.f / (1.f + expf(-to_f(gate[row])));
   const T* qr = static_cast<const T*>(w.qr);
@@ -464,7 +500,7 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
     const int j = ix.nbr[i * kNbr + o];
     const int64_t rj = rowbase + (j >= 0 ? j : 0);
     gr_load<T, D>(kr + rj * D, x, g);
-    gr_load<T, D>(v + rj * D, y, g);
+    gr_load<T, D>(v + (kvbase + (j >= 0 ? j : 0)) * D, y, g);
     const float sd = gr_dot<D>(q, x), dp = gr_dot<D>(d, y);
     const float p = j >= 0 ? expf(sd * scale - ll) : 0.f;
     const float ds = p * (gt * dp - Dl) * scale;
@@ -482,12 +518,13 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
       const int M = (int)ix.m;
       const int64_t mt = sum_tiles(M);
       for (int m = 0; m < M; ++m) {
+        if (summary_empty(ix, m)) continue;
         if (exclude_near && block_is_near(ix, m, c)) continue;
 #pragma unroll
         for (int k = 0; k < GRow<D>::KD; ++k) {
           const int e = g * GRow<D>::KD + k;
-          x.x[k] = to_f(ksum[sum_index(bh, m, e, D, mt)]);
-          y.x[k] = to_f(vsum[sum_index(bh, m, e, D, mt)]);
+          x.x[k] = to_f(ksum[sum_index(kv_of(bh, kv_group), m, e, D, mt)]);
+          y.x[k] = to_f(vsum[sum_index(kv_of(bh, kv_group), m, e, D, mt)]);
         }
         const float p = expf(gr_dot<D>(q, x) * scale - lg);
         const float ds = p * ((1.f - gt) * gr_dot<D>(d, y) - Dg) * scale;
@@ -501,16 +538,20 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
 }
 
 // dk, dv of key j: gathered over its own neighbourhood (the 3x3x3 relation is symmetric, so
-// no scatter/atomics) plus 1/|S| of its block's summary gradients; 8 lanes per key row.
+// no scatter/atomics) plus its weight in its summary's mean (1 / (members present in its block
+// x non-empty blocks in its summary's group)) times the summary gradients; kGL lanes per
+// key row. With summary-centre RoPE the summary's key gradient first goes back through the
+// summary's rotation R(centre)^T and is added after the local part's inverse rotation. With
+// GQA each query head's dk, dv go to float32 partials that k_bwd_gqa_reduce sums.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __restrict__ v,
                                                  const T* __restrict__ gate,
                                                  const T* __restrict__ dO,
                                                  const float* __restrict__ lse_loc, float scale,
-                                                 int64_t rows, BwdWork w, T* __restrict__ dk,
-                                                 T* __restrict__ dv) {
-  const int g = threadIdx.x & 7;
-  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x >> 3) + (threadIdx.x >> 3);
+                                                 int64_t rows, int kv_group, BwdWork w,
+                                                 T* __restrict__ dk, T* __restrict__ dv) {
+  const int g = threadIdx.x & (kGL - 1);
+  const int64_t row0 = blockIdx.x * (int64_t)(blockDim.x / kGL) + threadIdx.x / kGL;
   const bool active = row0 < rows;
   const int64_t row = active ? row0 : 0;
   const int64_t bh = row / ix.n, j = row % ix.n;
@@ -520,7 +561,7 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
   const T* kr = static_cast<const T*>(w.kr);
   GRow<D> kj, vj, ak, av, x, d;
   gr_load<T, D>(kr + row * D, kj, g);
-  gr_load<T, D>(v + row * D, vj, g);
+  gr_load<T, D>(v + (kv_of(bh, kv_group) * ix.n + j) * D, vj, g);
 #pragma unroll
   for (int k = 0; k < GRow<D>::KD; ++k) ak.x[k] = av.x[k] = 0.f;
   for (int o = 0; o < kNbr; ++o) {
@@ -538,17 +579,17 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
       av.x[k] = fmaf(p * gt, d.x[k], av.x[k]);
     }
   }
-  // un-pool: 1/|S| of the block summary's gradient (per-query-range partials summed in range
-  // order)
-  const int b = ix.block_of[j];
-  const float inv = 1.f / (float)ix.count[b];
+  // un-pool: the token's weight in its summary's (two-stage) mean times the summary's
+  // gradient (per-query-range partials summed in range order)
+  const int t = ix.sum_of[j];
+  const float wt = 1.f / ((float)ix.count[ix.block_of[j]] * (float)ix.count2[t]);
   const int64_t part = (int64_t)(rows / ix.n) * ix.m * D;
   GRow<D> sk, sv;
 #pragma unroll
   for (int k = 0; k < GRow<D>::KD; ++k) sk.x[k] = sv.x[k] = 0.f;
   for (int sp = 0; sp < w.nsplit; ++sp) {
-    gr_load<float, D>(w.dks + sp * part + (bh * ix.m + b) * D, x, g);
-    gr_load<float, D>(w.dvs + sp * part + (bh * ix.m + b) * D, d, g);
+    gr_load<float, D>(w.dks + sp * part + (bh * ix.m + t) * D, x, g);
+    gr_load<float, D>(w.dvs + sp * part + (bh * ix.m + t) * D, d, g);
 #pragma unroll
     for (int k = 0; k < GRow<D>::KD; ++k) {
       sk.x[k] += x.x[k];
@@ -556,33 +597,71 @@ __global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __res
     }
   }
 #pragma unroll
-  for (int k = 0; k < GRow<D>::KD; ++k) {
-    ak.x[k] = fmaf(sk.x[k], inv, ak.x[k]);
-    av.x[k] = fmaf(sv.x[k], inv, av.x[k]);
+  for (int k = 0; k < GRow<D>::KD; ++k) av.x[k] = fmaf(sv.x[k], wt, av.x[k]);
+  if (ix.geom.summary_rope == PACK3D_ROPE_CENTRE) {
+    gr_rotate<D>(ix, c, ak, g, -1.f);
+    // R(centre_t)^T of the summary's key gradient, pair e/2 of dims (e, e+1)
+    const float2* rc = reinterpret_cast<const float2*>(ix.rope_c) + (int64_t)t * (D / 2);
+#pragma unroll
+    for (int k = 0; k < GRow<D>::KD; k += 2) {
+      const float2 cs = rc[(g * GRow<D>::KD + k) / 2];
+      const float x0 = sk.x[k], x1 = sk.x[k + 1];
+      ak.x[k] = fmaf(x0 * cs.x + x1 * cs.y, wt, ak.x[k]);
+      ak.x[k + 1] = fmaf(x1 * cs.x - x0 * cs.y, wt, ak.x[k + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < GRow<D>::KD; ++k) ak.x[k] = fmaf(sk.x[k], wt, ak.x[k]);
+    gr_rotate<D>(ix, c, ak, g, -1.f);
   }
-  gr_rotate<D>(ix, c, ak, g, -1.f);
   if (active) {
-    gr_store<T, D>(dk + row * D, ak, g);
-    gr_store<T, D>(dv + row * D, av, g);
+    if (w.dkp) {
+      gr_store<float, D>(w.dkp + row * D, ak, g);
+      gr_store<float, D>(w.dvp + row * D, av, g);
+    } else {
+      gr_store<T, D>(dk + row * D, ak, g);
+      gr_store<T, D>(dv + row * D, av, g);
+    }
   }
+}
+
+// GQA: dk, dv of a KV head = the sum, in head order, of its query heads' float32 partials.
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_gqa_reduce(const float* __restrict__ dkp,
+                                                        const float* __restrict__ dvp,
+                                                        int64_t kv_elems, int64_t per_head,
+                                                        int kv_group, T* __restrict__ dk,
+                                                        T* __restrict__ dv) {
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= kv_elems) return;
+  const int64_t bhk = e / per_head, off = e % per_head;
+  float sk = 0.f, sv = 0.f;
+  for (int gq = 0; gq < kv_group; ++gq) {
+    const int64_t src = (bhk * kv_group + gq) * per_head + off;
+    sk += dkp[src];
+    sv += dvp[src];
+  }
+  dk[e] = from_f<T>(sk);
+  dv[e] = from_f<T>(sv);
 }
 
 // ------------------------------------------------------------------------------ launchers
-size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, int dtype, bool tc) {
-  return bwd_workspace_bytes_for(ix, bh, dtype == PACK3D_BF16 ? 2 : 4, tc);
+size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, int dtype, bool tc,
+                           int kv_group) {
+  return bwd_workspace_bytes_for(ix, bh, dtype == PACK3D_BF16 ? 2 : 4, tc, kv_group);
 }
 
 cudaError_t bwd_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* ksum,
-                            const void* vsum, const float* lse_glob, int64_t bh, float scale,
-                            int excl, cudaStream_t s);
+                            const void* vsum, const float* lse_glob, int64_t bh, int kv_group,
+                            float scale, int excl, cudaStream_t s);
 
 template <typename T, int D>
 cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
                      const void* gate, const void* ksum, const void* vsum, const void* o_loc,
                      const void* o_glob, const float* lse_loc, const float* lse_glob,
-                     const void* dO, int64_t bh, float scale, int excl, void* dq, void* dk,
-                     void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
-  const BwdWork w = bwd_carve(ix, bh, ws, sizeof(T), tc);
+                     const void* dO, int64_t bh, int kv_group, float scale, int excl, void* dq,
+                     void* dk, void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
+  const BwdWork w = bwd_carve(ix, bh, ws, sizeof(T), tc, kv_group);
   const int64_t rows = bh * ix.n;
   const unsigned rb = (unsigned)((rows + 3) / 4);
   const unsigned mb = (unsigned)((bh * ix.m + 3) / 4);
@@ -592,41 +671,49 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
   const T* tg = static_cast<const T*>(gate);
   const T* tdo = static_cast<const T*>(dO);
   k_bwd_prep<T, D><<<rb, 128, 0, s>>>(ix, tq, tk, tg, static_cast<const T*>(o_loc),
-                                       static_cast<const T*>(o_glob), tdo, rows, w,
+                                       static_cast<const T*>(o_glob), tdo, rows, kv_group, w,
                                        static_cast<T*>(dgate));
   count_launch();
   if (tc) {
     // the global branch's summary gradients and its part of dq on tensor cores
-    const cudaError_t e = bwd_tc_dispatch(ix, w, ksum, vsum, lse_glob, bh, scale, excl, s);
+    const cudaError_t e =
+        bwd_tc_dispatch(ix, w, ksum, vsum, lse_glob, bh, kv_group, scale, excl, s);
     if (e != cudaSuccess) return e;
   } else {
     k_bwd_dsum<T, D><<<mb, 128, 0, s>>>(ix, static_cast<const T*>(ksum),
                                          static_cast<const T*>(vsum), tg, tdo, lse_glob, scale,
-                                         excl, bh, w);
+                                         excl, bh, kv_group, w);
     count_launch();
   }
-  const unsigned gb = (unsigned)((rows + 15) / 16);  // 16 rows (8 lanes each) per block
+  const unsigned gb = (unsigned)((rows + 128 / kGL - 1) / (128 / kGL));  // kGL lanes per row
   k_bwd_dq<T, D><<<gb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
                                      static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
-                                     scale, excl, rows, w, static_cast<T*>(dq));
-  k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, w,
+                                     scale, excl, rows, kv_group, w, static_cast<T*>(dq));
+  k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, kv_group, w,
                                       static_cast<T*>(dk), static_cast<T*>(dv));
   count_launch(2);
+  if (kv_group > 1) {
+    const int64_t kv_elems = rows / kv_group * D;
+    k_bwd_gqa_reduce<T><<<(unsigned)((kv_elems + 255) / 256), 256, 0, s>>>(
+        w.dkp, w.dvp, kv_elems, ix.n * (int64_t)D, kv_group, static_cast<T*>(dk),
+        static_cast<T*>(dv));
+    count_launch();
+  }
   return cudaGetLastError();
 }
 
 // Global branch + mixer only, over a given local output (which `o` may alias).
 cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                  const void* ksum, const void* vsum, const void* o_loc,
-                                 int dtype, int64_t bh, float scale, int excl, void* o,
-                                 float* lse_glob, void* o_glob, cudaStream_t s) {
+                                 int dtype, int64_t bh, int kv_group, float scale, int excl,
+                                 void* o, float* lse_glob, void* o_glob, cudaStream_t s) {
   const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
   const int d = ix.geom.head_dim;
 #define P3D_GLB(T, D)                                                                          \
   k_global_fwd<T, D, 32><<<grid, 128, 0, s>>>(                                                 \
       ix, static_cast<const T*>(q), static_cast<const T*>(ksum), static_cast<const T*>(vsum), \
-      static_cast<const T*>(gate), static_cast<const T*>(o_loc), scale, excl, static_cast<T*>(o), \
-      lse_glob, static_cast<T*>(o_glob))
+      static_cast<const T*>(gate), static_cast<const T*>(o_loc), scale, excl, kv_group,       \
+      static_cast<T*>(o), lse_glob, static_cast<T*>(o_glob))
   if (dtype == PACK3D_BF16) {
     if (d == 96) P3D_GLB(__nv_bfloat16, 96); else P3D_GLB(__nv_bfloat16, 48);
   } else {
@@ -638,14 +725,14 @@ cudaError_t global_simt_dispatch(const pack3d_index& ix, const void* q, const vo
 }
 
 cudaError_t local_simt_dispatch(const pack3d_index& ix, const void* q, const void* k,
-                                const void* v, int dtype, int64_t bh, float scale, void* o_loc,
-                                float* lse_loc, cudaStream_t s) {
+                                const void* v, int dtype, int64_t bh, int kv_group, float scale,
+                                void* o_loc, float* lse_loc, cudaStream_t s) {
   const dim3 grid((unsigned)((ix.n + 127) / 128), (unsigned)bh);
   const int d = ix.geom.head_dim;
 #define P3D_LOC(T, D)                                                                         \
   k_local_fwd<T, D><<<grid, 128, 0, s>>>(ix, static_cast<const T*>(q), static_cast<const T*>(k), \
-                                          static_cast<const T*>(v), scale, static_cast<T*>(o_loc), \
-                                          lse_loc)
+                                          static_cast<const T*>(v), scale, kv_group,           \
+                                          static_cast<T*>(o_loc), lse_loc)
   if (dtype == PACK3D_BF16) {
     if (d == 96) P3D_LOC(__nv_bfloat16, 96); else P3D_LOC(__nv_bfloat16, 48);
   } else {
@@ -660,12 +747,13 @@ cudaError_t bwd_simt_dispatch(const pack3d_index& ix, const void* q, const void*
                               const void* v, const void* gate, const void* ksum,
                               const void* vsum, const void* o_loc, const void* o_glob,
                               const float* lse_loc, const float* lse_glob, const void* dO,
-                              int dtype, int64_t bh, float scale, int excl, void* dq, void* dk,
-                              void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
+                              int dtype, int64_t bh, int kv_group, float scale, int excl,
+                              void* dq, void* dk, void* dv, void* dgate, void* ws, bool tc,
+                              cudaStream_t s) {
   const int d = ix.geom.head_dim;
 #define P3D_BWD(T, D)                                                                         \
-  bwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc, lse_glob, dO, bh, scale, \
-                 excl, dq, dk, dv, dgate, ws, tc, s)
+  bwd_simt<T, D>(ix, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc, lse_glob, dO, bh,      \
+                 kv_group, scale, excl, dq, dk, dv, dgate, ws, tc, s)
   if (dtype == PACK3D_BF16) return d == 96 ? P3D_BWD(__nv_bfloat16, 96) : P3D_BWD(__nv_bfloat16, 48);
   return d == 96 ? P3D_BWD(float, 96) : P3D_BWD(float, 48);
 #undef P3D_BWD

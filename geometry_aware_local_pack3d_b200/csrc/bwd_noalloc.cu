@@ -22,6 +22,7 @@
 
 namespace p3d {
 pack3d_status check_common(const pack3d_index* idx, int dtype, int batch, int heads);
+pack3d_status kv_group_of(int heads, int kv_heads, int* group);
 }
 
 namespace {
@@ -53,18 +54,22 @@ extern "C" pack3d_status pack3d_attn_bwd_noalloc(
     const pack3d_index* idx, const void* q, const void* k, const void* v, const void* gate,
     const void* ksum, const void* vsum, const void* o_loc, const void* o_glob,
     const float* lse_loc, const float* lse_glob, const void* dO, int dtype, int batch, int heads,
-    float scale, uint32_t flags, void* dq, void* dk, void* dv, void* dgate, void* stream) {
+    int kv_heads, float scale, uint32_t flags, void* dq, void* dk, void* dv, void* dgate,
+    void* stream) {
   // a rejected call launches nothing: the launch count reads 0 afterwards, and argument errors
   // are the ones pack3d_attn_bwd reports for the same arguments
   p3d::reset_launches();
   const pack3d_status common = p3d::check_common(idx, dtype, batch, heads);
   if (common != PACK3D_OK) return common;
-  const size_t need = pack3d_bwd_workspace_bytes(idx, dtype, batch, heads);
+  int group = 1;
+  const pack3d_status kv = p3d::kv_group_of(heads, kv_heads, &group);
+  if (kv != PACK3D_OK) return kv;
+  const size_t need = pack3d_bwd_workspace_bytes(idx, dtype, batch, heads, kv_heads);
   if (need > kScratchBytes) return PACK3D_ERR_WORKSPACE;  // problem too large for the buffer
   void* ws = nullptr;
   const pack3d_status st = scratch_address(&ws);
   if (st != PACK3D_OK) return st;
   return pack3d_attn_bwd(idx, q, k, v, gate, ksum, vsum, o_loc, o_glob, lse_loc, lse_glob, dO,
-                         dtype, batch, heads, scale, flags, dq, dk, dv, dgate, ws, kScratchBytes,
-                         stream);
+                         dtype, batch, heads, kv_heads, scale, flags, dq, dk, dv, dgate, ws,
+                         kScratchBytes, stream);
 }

@@ -56,24 +56,9 @@ struct Params {
   int64_t units, units_per_bh;  // dq: 128-query tiles
   int n_chunks;                 // dq: 64-summary chunks per (batch, head)
   int m_tiles, q_tiles, q_per_split;  // dsum: 128-summary tiles, 64-query tiles
+  int kv_group;                       // query heads per KV head (summaries per KV head)
   long long wait_budget;              // SM cycles of each bounded wait
 };
-
-// summaries of block coordinates [z0, z1] x [y0, y1] x [x0, x1] are excluded for a query at
-// c (the blocks meeting the cube [c - 1, c + 1]^3); empty ranges when exclusion is off
-struct ExclBox {
-  int z0, z1, y0, y1, x0, x1;
-};
-__device__ __forceinline__ ExclBox excl_box(const pack3d_index& ix, int32_t code, bool on) {
-  ExclBox e{0, -1, 0, -1, 0, -1};
-  if (!on) return e;
-  const Coord c = decode(code);
-  const pack3d_geom& g = ix.geom;
-  e.z0 = max(c.z - 1, 0) / g.bz; e.z1 = min(c.z + 1, g.gz - 1) / g.bz;
-  e.y0 = max(c.y - 1, 0) / g.by; e.y1 = min(c.y + 1, g.gy - 1) / g.by;
-  e.x0 = max(c.x - 1, 0) / g.bx; e.x1 = min(c.x + 1, g.gx - 1) / g.bx;
-  return e;
-}
 }  // namespace btc
 
 // ============================================================================= dq~ (global)
@@ -136,7 +121,7 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
 
   if (warp < 4) {
     // ------------------------------------------------------------ elementwise + epilogue
-    const int nby = P.ix.geom.gy / P.ix.geom.by, nbx = P.ix.geom.gx / P.ix.geom.bx;
+    const int nby = P.ix.sum_grid[1], nbx = P.ix.sum_grid[2];
     uint32_t gc = 0;
     int pc = 0;
     bool ok = true;
@@ -154,8 +139,8 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
       const float Dg = valid ? P.Dg[grow] : 0.f;
       const bool live = lse != -INFINITY;  // every summary excluded: no global gradient
       const float nl = live ? -lse * kLog2e : 0.f;
-      const btc::ExclBox ex = btc::excl_box(P.ix, valid ? P.ix.coord[row] : 0,
-                                           P.exclude_near != 0 && valid);
+      const ExclBox ex = excl_box(P.ix, decode(valid ? P.ix.coord[row] : 0),
+                                  P.exclude_near != 0 && valid);
       for (int j = 0; j < NC; ++j, ++gc) {
         if (!__all_sync(0xffffffffu, ab.wait(&bars[B_SFULL], gc & 1))) { ok = false; break; }
         tc::tc_fence_after();
@@ -261,7 +246,7 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
           if (kv >= (uint32_t)S::kStages &&
               !ab.wait(&bars[B_KVEMPTY + st], ((kv / S::kStages) - 1) & 1)) { ok = false; break; }
           tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kCTile);
-          const int64_t tile = (bh * MT + j) * (int64_t)(btc::kChunk * D);
+          const int64_t tile = (kv_of(bh, P.kv_group) * MT + j) * (int64_t)(btc::kChunk * D);
           tc::bulk_g2s(smem + S::kK + st * S::kCTile, P.ksum + tile, S::kCTile,
                        &bars[B_KVFULL + st]);
           tc::bulk_g2s(smem + S::kV + st * S::kCTile, P.vsum + tile, S::kCTile,
@@ -415,9 +400,8 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
     const int rin = warp * 32 + lane;           // summary row of the tile
     const int m = mt * btc::kRows + rin;        // summary id
     const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
-    const pack3d_geom& g = P.ix.geom;
-    const int nby = g.gy / g.by, nbx = g.gx / g.bx;
-    const int bz = m / (nby * nbx), byy = (m / nbx) % nby, bxx = m % nbx;  // block coords
+    const int nby = P.ix.sum_grid[1], nbx = P.ix.sum_grid[2];
+    const int bz = m / (nby * nbx), byy = (m / nbx) % nby, bxx = m % nbx;  // summary coords
     const bool excl = P.exclude_near != 0;
     const float2* rowf = reinterpret_cast<const float2*>(smem + S::kRowF);
     const int* rowx = reinterpret_cast<const int*>(smem + S::kRowX);
@@ -515,7 +499,8 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
       tc::PieceOrder<KC>::at(i, r, kc);
       const int m = mt * btc::kRows + r;
       const bool ok = m < MT * 64;
-      const int64_t src = ((bh * MT + (ok ? m / 64 : 0)) * (D / 8) + kc) * 512 + (ok ? m % 64 : 0) * 8;
+      const int64_t src = ((kv_of(bh, P.kv_group) * MT + (ok ? m / 64 : 0)) * (D / 8) + kc) * 512 +
+                          (ok ? m % 64 : 0) * 8;
       const int off = kc * 2048 + (r >> 3) * 128 + (r & 7) * 16;
       tc::cp_async16(smem + S::kK + off, P.ksum + src, ok);
       tc::cp_async16(smem + S::kV + off, P.vsum + src, ok);
@@ -541,11 +526,11 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
       if (ptid < btc::kChunk) {
         const int64_t row = row0 + ptid;
         float2 rf = make_float2(-INFINITY, 0.f);
-        btc::ExclBox ex{0, -1, 0, -1, 0, -1};
+        ExclBox ex{0, -1, 0, -1, 0, -1};
         if (row < N) {
           const float lse = P.lse[bh * N + row];
           rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY, P.Dg[bh * N + row]);
-          ex = btc::excl_box(P.ix, P.ix.coord[row], P.exclude_near != 0);
+          ex = excl_box(P.ix, decode(P.ix.coord[row]), P.exclude_near != 0);
         }
         reinterpret_cast<float2*>(smem + S::kRowF)[st * btc::kChunk + ptid] = rf;
         int* x = reinterpret_cast<int*>(smem + S::kRowX) + (st * btc::kChunk + ptid) * 6;
@@ -630,8 +615,8 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
 // ------------------------------------------------------------------------------ host side
 template <int D>
 cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* ksum,
-                          const void* vsum, const float* lse_glob, int64_t bh, float scale,
-                          int excl, cudaStream_t s) {
+                          const void* vsum, const float* lse_glob, int64_t bh, int kv_group,
+                          float scale, int excl, cudaStream_t s) {
   static std::atomic<uint64_t> attr_dq{0}, attr_dsum{0};
   if (smem_attr_once(reinterpret_cast<const void*>(k_bwd_dq_tc<D>), bdq::Smem<D>::kBytes,
                      attr_dq) != cudaSuccess ||
@@ -650,6 +635,7 @@ cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* 
   p.scale_log2 = scale * kLog2e;
   p.exclude_near = excl;
   p.wait_budget = wait_budget_cycles();
+  p.kv_group = kv_group;
   p.bh_count = bh;
   // summary gradients: (batch*head) x 128-summary tiles x query ranges
   p.m_tiles = (int)((ix.m + btc::kRows - 1) / btc::kRows);
@@ -674,11 +660,11 @@ cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* 
 }
 
 cudaError_t bwd_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* ksum,
-                            const void* vsum, const float* lse_glob, int64_t bh, float scale,
-                            int excl, cudaStream_t s) {
+                            const void* vsum, const float* lse_glob, int64_t bh, int kv_group,
+                            float scale, int excl, cudaStream_t s) {
   if (ix.geom.head_dim == 96)
-    return launch_bwd_tc<96>(ix, w, ksum, vsum, lse_glob, bh, scale, excl, s);
-  return launch_bwd_tc<48>(ix, w, ksum, vsum, lse_glob, bh, scale, excl, s);
+    return launch_bwd_tc<96>(ix, w, ksum, vsum, lse_glob, bh, kv_group, scale, excl, s);
+  return launch_bwd_tc<48>(ix, w, ksum, vsum, lse_glob, bh, kv_group, scale, excl, s);
 }
 
 }  // namespace p3d

@@ -25,22 +25,30 @@ struct BwdWork {
   __nv_bfloat16* qtb;   // [BH, N, d]  rotated q, bf16 (the qr array itself)
   __nv_bfloat16* dogb;  // [BH, N, d]  (1 - g) dO, bf16
   float* dqg;           // [BH, N, d]  global branch's part of dq~ (rotated space)
+  // GQA only (null with one query head per KV head): each query head's dk, dv in float32,
+  // summed over the query heads of a KV head by k_bwd_gqa_reduce
+  float* dkp;           // [BH, N, d]
+  float* dvp;           // [BH, N, d]
 };
 
 inline size_t bwd_align(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Bytes of workspace for I/O elements of `el` bytes; `tc` (bf16 only) adds the tensor-core
-// path's arrays.
-inline size_t bwd_workspace_bytes_for(const pack3d_index& ix, int64_t bh, size_t el, bool tc) {
+// path's arrays; `kv_group` > 1 (GQA) adds the per-query-head key gradients. `bh` counts query
+// heads.
+inline size_t bwd_workspace_bytes_for(const pack3d_index& ix, int64_t bh, size_t el, bool tc,
+                                      int kv_group) {
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
   const int ns = tc ? kDsumSplit : 1;
   size_t b = 2 * bwd_align(el * rows * D) + 2 * bwd_align(sizeof(float) * rows) +
              2 * bwd_align(sizeof(float) * ns * sums * D);
   if (tc) b += bwd_align(sizeof(__nv_bfloat16) * rows * D) + bwd_align(sizeof(float) * rows * D);
+  if (kv_group > 1) b += 2 * bwd_align(sizeof(float) * rows * D);
   return b;
 }
 
-inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, size_t el, bool tc) {
+inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, size_t el, bool tc,
+                         int kv_group) {
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
   char* p = static_cast<char*>(ws);
   BwdWork w;
@@ -53,10 +61,15 @@ inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, size_t el
   w.dvs = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * w.nsplit * sums * D);
   w.qtb = w.dogb = nullptr;
   w.dqg = nullptr;
+  w.dkp = w.dvp = nullptr;
   if (tc) {  // bf16 I/O: qr already holds the rotated q in bf16
     w.qtb = static_cast<__nv_bfloat16*>(w.qr);
     w.dogb = reinterpret_cast<__nv_bfloat16*>(p); p += bwd_align(sizeof(__nv_bfloat16) * rows * D);
-    w.dqg = reinterpret_cast<float*>(p);
+    w.dqg = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows * D);
+  }
+  if (kv_group > 1) {
+    w.dkp = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows * D);
+    w.dvp = reinterpret_cast<float*>(p);
   }
   return w;
 }

@@ -39,19 +39,51 @@ __device__ __forceinline__ void set_status(int32_t* status, int code) {
   if (status) atomicCAS(status + kStatusFirstError, 0, code);
 }
 
-// (cos, sin) of coordinate value `cv` for rotation pair p of an axis third.
-__device__ __forceinline__ float2 rope_cs(const float* rope, int pairs, int cv, int p) {
-  return reinterpret_cast<const float2*>(rope)[cv * pairs + p];
+// (cos, sin) of coordinate value `cv` on axis `a` for rotation pair p of that axis third;
+// the table is [3 axes][rows][pairs] (each axis carries its own coordinate scale).
+__device__ __forceinline__ int rope_slot(int rows, int pairs, int a, int cv, int p) {
+  return (a * rows + cv) * pairs + p;
+}
+__device__ __forceinline__ float2 rope_cs(const float* rope, int rows, int pairs, int a, int cv,
+                                          int p) {
+  return reinterpret_cast<const float2*>(rope)[rope_slot(rows, pairs, a, cv, p)];
 }
 
-// Is summary `m` (block box) within Chebyshev distance 1 of coordinate c?
+// Is summary `m`'s box within Chebyshev distance 1 of coordinate c? The box of summary
+// (mz, my, mx) spans [m_a * ext_a, m_a * ext_a + ext_a - 1] per axis (its part outside the grid
+// cannot change the answer: the cube around a token reaches at most one site past the grid).
 __device__ __forceinline__ bool block_is_near(const pack3d_index& ix, int m, const Coord& c) {
-  const int nbx = ix.geom.gx / ix.geom.bx, nby = ix.geom.gy / ix.geom.by;
-  const int mx = m % nbx, my = (m / nbx) % nby, mz = m / (nbx * nby);
-  const int lz = mz * ix.geom.bz, ly = my * ix.geom.by, lx = mx * ix.geom.bx;
-  return lz <= c.z + 1 && lz + ix.geom.bz - 1 >= c.z - 1 && ly <= c.y + 1 &&
-         ly + ix.geom.by - 1 >= c.y - 1 && lx <= c.x + 1 && lx + ix.geom.bx - 1 >= c.x - 1;
+  const int ngx = ix.sum_grid[2], ngy = ix.sum_grid[1];
+  const int mx = m % ngx, my = (m / ngx) % ngy, mz = m / (ngx * ngy);
+  const int ez = ix.sum_ext[0], ey = ix.sum_ext[1], ex = ix.sum_ext[2];
+  const int lz = mz * ez, ly = my * ey, lx = mx * ex;
+  return lz <= c.z + 1 && lz + ez - 1 >= c.z - 1 && ly <= c.y + 1 && ly + ey - 1 >= c.y - 1 &&
+         lx <= c.x + 1 && lx + ex - 1 >= c.x - 1;
 }
+
+// A summary with no member present takes part in no softmax.
+__device__ __forceinline__ bool summary_empty(const pack3d_index& ix, int m) {
+  return (ix.empty[m >> 5] >> (m & 31)) & 1u;
+}
+
+// Summary-grid coordinates of the summaries whose box meets the cube [c-1, c+1]^3 (clipped to
+// the grid): [z0, z1] x [y0, y1] x [x0, x1]; empty ranges when `on` is false.
+struct ExclBox {
+  int z0, z1, y0, y1, x0, x1;
+};
+__device__ __forceinline__ ExclBox excl_box(const pack3d_index& ix, const Coord& c, bool on) {
+  ExclBox e{0, -1, 0, -1, 0, -1};
+  if (!on) return e;
+  const pack3d_geom& g = ix.geom;
+  e.z0 = max(c.z - 1, 0) / ix.sum_ext[0]; e.z1 = min(c.z + 1, g.gz - 1) / ix.sum_ext[0];
+  e.y0 = max(c.y - 1, 0) / ix.sum_ext[1]; e.y1 = min(c.y + 1, g.gy - 1) / ix.sum_ext[1];
+  e.x0 = max(c.x - 1, 0) / ix.sum_ext[2]; e.x1 = min(c.x + 1, g.gx - 1) / ix.sum_ext[2];
+  return e;
+}
+
+// GQA: query head bh = b * H + h reads the keys, values and summaries of KV head
+// b * H_kv + h / G = bh / G, G = H / H_kv query heads per KV head.
+__host__ __device__ __forceinline__ int64_t kv_of(int64_t bh, int group) { return bh / group; }
 
 __device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + __expf(-a)); }
 

@@ -46,7 +46,7 @@ constexpr int kThreads = 480;
 constexpr int kProd = 128;        // query producer threads
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kRopeSmemBytes = 16384;
+constexpr int kRopeSmemBytes = 24576;  // [3 axes][64 coordinates][16 pairs] (cos, sin)
 #ifndef P3D_POLY_EVERY
 #define P3D_POLY_EVERY 0
 #endif
@@ -101,6 +101,8 @@ struct Params {
   int units_per_bh;
   int n_chunks;
   int rope_in_smem;
+  int kv_group;                // query heads per KV head (summaries are per KV head)
+  int has_empty;               // some summary has no member (masked in every row)
   long long wait_budget;       // SM cycles of each bounded wait
 };
 
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
   }
   // the rotation table in shared memory when it fits (read by the query producer)
   if (P.rope_in_smem) {
-    const int n = P.ix.rope_rows * P.ix.rope_pairs * 2;
+    const int n = 3 * P.ix.rope_rows * P.ix.rope_pairs * 2;
     float* dst = reinterpret_cast<float*>(smem + S::kRope);
     for (int i = tid; i < n; i += blockDim.x) dst[i] = P.ix.rope[i];
   }
@@ -168,22 +170,17 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     const int t = warp >> 2;
     const int rin = (warp & 3) * 32 + lane;
     const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
-    const int nby = P.ix.geom.gy / P.ix.geom.by, nbx = P.ix.geom.gx / P.ix.geom.bx;
+    const int nby = P.ix.sum_grid[1], nbx = P.ix.sum_grid[2];
     int pc = 0;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int64_t bh = u / P.units_per_bh;
       const int64_t row = (u % P.units_per_bh) * (kRows * kTiles) + t * kRows + rin;
       const bool valid = row < N;
-      // summaries excluded for this row: blocks meeting the cube [c-1, c+1]^3, kept as block
-      // coordinate ranges [z0,z1] x [y0,y1] x [x0,x1] (empty when exclusion is off)
-      int z0 = 0, z1 = -1, y0 = 0, y1 = -1, x0 = 0, x1 = -1;
-      if (P.exclude_near && valid) {
-        const Coord c = decode(P.ix.coord[row]);
-        const pack3d_geom& g = P.ix.geom;
-        z0 = max(c.z - 1, 0) / g.bz; z1 = min(c.z + 1, g.gz - 1) / g.bz;
-        y0 = max(c.y - 1, 0) / g.by; y1 = min(c.y + 1, g.gy - 1) / g.by;
-        x0 = max(c.x - 1, 0) / g.bx; x1 = min(c.x + 1, g.gx - 1) / g.bx;
-      }
+      // summaries excluded for this row: those whose box meets the cube [c-1, c+1]^3, kept as
+      // summary-grid ranges [z0,z1] x [y0,y1] x [x0,x1] (empty when exclusion is off)
+      const ExclBox xb = excl_box(P.ix, valid ? decode(P.ix.coord[row]) : Coord{0, 0, 0},
+                                  P.exclude_near && valid);
+      const int z0 = xb.z0, z1 = xb.z1, y0 = xb.y0, y1 = xb.y1, x0 = xb.x0, x1 = xb.x1;
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < NC; ++j) {
@@ -198,8 +195,13 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         tc::tc_fence_after();
         const int m0 = j * kChunk;
         const int ncol = min(kChunk, M - m0);
+        // summaries with no member are out of every row's softmax
         uint32_t xm[2] = {0u, 0u};
-        bool any_x = false;
+        if (P.has_empty) {
+          xm[0] = P.ix.empty[2 * j];
+          xm[1] = (m0 + 32 < M) ? P.ix.empty[2 * j + 1] : 0u;
+        }
+        bool any_x = (xm[0] | xm[1]) != 0u;
         for (int mz = z0; mz <= z1; ++mz)
           for (int my = y0; my <= y1; ++my)
             for (int mx = x0; mx <= x1; ++mx) {
@@ -436,7 +438,8 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         const int axis = (kc * 8) / DA, p0 = ((kc * 8) % DA) / 2;
         const int cv = coord_axis(cc, axis);
         // (cos, sin) of the 4 pairs of this piece: 32 contiguous bytes of the table
-        const float4* cs4 = reinterpret_cast<const float4*>(rope + 2 * (cv * P.ix.rope_pairs + p0));
+        const float4* cs4 = reinterpret_cast<const float4*>(
+            rope + 2 * rope_slot(P.ix.rope_rows, P.ix.rope_pairs, axis, cv, p0));
         const float4 ca = cs4[0], cb = cs4[1];
         const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
         const uint32_t xin[4] = {x.x, x.y, x.z, x.w};
@@ -566,14 +569,14 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       const int64_t MT = sum_tiles(M);
       uint32_t kv_it = 0;
       for (int64_t u = blockIdx.x; u < P.units && !*abort_flag; u += gridDim.x) {
-        const int64_t bh = u / P.units_per_bh;
+        const int64_t bhk = kv_of(u / P.units_per_bh, P.kv_group);  // summaries of the KV head
         bool ok = true;
         for (int j = 0; j < NC; ++j, ++kv_it) {
           const int st = kv_it % kStages;
           if (kv_it >= (uint32_t)kStages &&
               !ab.wait(&bars[B_KVEMPTY + st], ((kv_it / kStages) - 1) & 1)) { ok = false; break; }
           tc::mbar_expect_tx(&bars[B_KVFULL + st], 2u * S::kCTile);
-          const int64_t tile = (bh * MT + j) * (int64_t)(kChunk * D);  // element offset
+          const int64_t tile = (bhk * MT + j) * (int64_t)(kChunk * D);  // element offset
           tc::bulk_g2s(smem + S::kK + st * S::kCTile, P.ksum + tile, S::kCTile,
                        &bars[B_KVFULL + st]);
           tc::bulk_g2s(smem + S::kV + st * S::kCTile, P.vsum + tile, S::kCTile,
@@ -600,8 +603,8 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
 template <int D>
 cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* gate,
                              const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
-                             float scale, int excl, void* o, float* lse_glob, void* o_glob,
-                             cudaStream_t s) {
+                             int kv_group, float scale, int excl, void* o, float* lse_glob,
+                             void* o_glob, cudaStream_t s) {
   using namespace gtc;
   static std::atomic<uint64_t> attr_done{0};
   if (smem_attr_once(reinterpret_cast<const void*>(k_global_tc<D>), Smem<D>::kBytes, attr_done) !=
@@ -623,7 +626,9 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   p.units_per_bh = (int)((ix.n + kRows * kTiles - 1) / (kRows * kTiles));
   p.units = bh * p.units_per_bh;
   p.n_chunks = (int)((ix.m + kChunk - 1) / kChunk);
-  p.rope_in_smem = (int64_t)ix.rope_rows * ix.rope_pairs * 8 <= kRopeSmemBytes ? 1 : 0;
+  p.rope_in_smem = 3LL * ix.rope_rows * ix.rope_pairs * 8 <= kRopeSmemBytes ? 1 : 0;
+  p.kv_group = kv_group;
+  p.has_empty = ix.n_empty > 0 ? 1 : 0;
   const int grid = (int)(p.units < sm_count() ? p.units : sm_count());
   k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(p);
   count_launch();
@@ -632,13 +637,13 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
 
 cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void* gate,
                                const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
-                               float scale, int excl, void* o, float* lse_glob, void* o_glob,
-                               cudaStream_t s) {
+                               int kv_group, float scale, int excl, void* o, float* lse_glob,
+                               void* o_glob, cudaStream_t s) {
   if (ix.geom.head_dim == 96)
-    return launch_global_tc<96>(ix, q, gate, ksum, vsum, o_loc, bh, scale, excl, o, lse_glob,
-                                o_glob, s);
-  return launch_global_tc<48>(ix, q, gate, ksum, vsum, o_loc, bh, scale, excl, o, lse_glob,
-                              o_glob, s);
+    return launch_global_tc<96>(ix, q, gate, ksum, vsum, o_loc, bh, kv_group, scale, excl, o,
+                                lse_glob, o_glob, s);
+  return launch_global_tc<48>(ix, q, gate, ksum, vsum, o_loc, bh, kv_group, scale, excl, o,
+                              lse_glob, o_glob, s);
 }
 
 }  // namespace p3d

@@ -1,43 +1,46 @@
-// Local branch of PACK3D attention, row-gather form (bf16 I/O, head_dim 48 or 96), for keys
-// that were rotated once up front (pack3d_summarize_rotated).
+// Local branch of PACK3D attention on tcgen05 tensor cores (bf16 I/O, head_dim 48 or 96), for
+// raw keys (ROT: the producer warps rotate each key row in shared memory once it has landed) or
+// for keys rotated once up front by pack3d_summarize_rotated (gathered as they are).
 //
 // Project page "Geometry Matters in Packed 3D Attention", Chapter 3 Contract 1: each query
 // attends exactly to every token of its 3x3x3 coordinate neighbourhood, found by coordinate,
 // never by adjacency in memory; paper summary §3.5: streamed online softmax, no gathered
 // neighbour tensor in memory.
 //
-// Work unit: one 8x4x8 (z, y, x) brick of one (batch, head), split into two 128-query tiles
-// (x0..x0+3 and x0+4..x0+7); one persistent CTA per SM. The two
-// tiles share one stream of halo z-slices (10 slices of 6x10 = 60 keys), so a key row is
-// fetched once for 256 queries. Units are handed out by a device-wide counter (status word 2
-// of the index; the last CTA to finish puts it back to zero), so SMs that run slower take
-// fewer units. Per unit:
-//   * one 3D TMA box load brings the memory slots of the unit's 10x6x10 halo from the inverse
-//     map (x start rounded down to a 16-byte boundary: box 16x6x10 int32);
-//   * four producer warps fetch, per halo z-slice, the 60 rotated key rows and value rows with
-//     one cp.async per 16-byte piece (rows off the grid are zero-filled) into the no-swizzle
-//     core-matrix layout, four stages deep; each thread's copies arrive on the stage's barrier
-//     by themselves when they land;
+// Work unit: one 4x8x8 (z, y, x) brick of one (batch, head), split into two 128-query tiles
+// (y0..y0+3 and y0+4..y0+7); one persistent CTA per SM. The two tiles share one stream of
+// halo z-slices (6 slices of 10x10 = 100 keys), so a key row is fetched once for 256 queries.
+// Units are handed out by a device-wide counter (status word 2 of the index; the last CTA to
+// finish puts it back to zero), so SMs that run slower take fewer units. Per unit:
+//   * one 3D TMA box load brings the memory slots of the unit's 6x10x10 halo from the inverse
+//     map (x start rounded down to a 16-byte boundary: box 16x10x6 int32);
+//   * four producer warps fetch, per halo z-slice, the 100 key rows and value rows with one
+//     cp.async per 16-byte piece (rows off the grid or at empty sites are zero-filled) into the
+//     no-swizzle core-matrix layout, three stages deep. With rotated keys each thread's copies
+//     arrive on the stage's barrier by themselves when they land; with raw keys each thread
+//     waits for its copies of a slice (the next slice's copies already in flight), rotates its
+//     key pieces in place by the key's coordinate (known from the halo position) and then
+//     arrives;
 //   * the q tiles are double-buffered: softmax warps 0 and 1 of each tile, idle once their
 //     slices of a unit are done, load the next unit's q rows (64 rows each, one row per lane),
 //     rotate them in registers (axial RoPE by the row's coordinates) and store them into the
 //     tile's other q buffer, so the MMAs start a unit as soon as the previous one's last PV
 //     has been issued.
-// Slice key order: x columns 0-3, then 4-5, then 6-9 of the halo (each block y-major), so tile
-// 0's neighbours (halo x 0..5) are slice rows 0..35 and tile 1's (halo x 4..9) rows 24..59:
-// each tile works on a 48-row window (rows 24 t .. 24 t + 47; rows 60..71 are zero padding).
-// Per tile, chunk s = halo z-slice s. Row r = 32 w + 16 dz + 4 y + x holds brick position
-// (2w + dz, y, x), so warp w of a tile needs exactly slices 2w .. 2w+3 and chunk s is owned by
-// warps max(0, (s-2)/2) .. min(3, s/2). Per tile and chunk:
-//   S_s = q~ k~_s^T   (SS MMA 128 x 48, fp32, TMEM buffer s % 2)
-//   owners: 3x3x3 mask, online softmax over the window's first 36 columns (the only ones that
-//   can hold a neighbour of the tile), P = exp2(s - m) as bf16 over the buffer's first 24
-//   columns (P = 0 in window columns 36..47);  O += P_s v_s  (TS MMA, N = d) with the rows
+// Slice key order: halo row hy major, then halo column hx (row 10 hy + hx), so tile t's keys
+// (halo rows 4t .. 4t+5) are slice rows 40t .. 40t+59: each tile works on a 64-row window
+// starting at slice row 40 t (rows 100..103 of a stage are zero padding).
+// Row r = 32 z + 8 y + x of a tile holds brick position (z, 4 t + y, x): warp w is the z-plane
+// w of the brick, so it needs exactly slices w .. w+2, and slice s is owned by warps
+// max(0, s-2) .. min(3, s). Per tile and slice:
+//   S_s = q~ k~_s^T   (SS MMA 128 x 64, fp32, TMEM buffer s % 2)
+//   owners: 3x3x3 mask, online softmax over the window's first 60 columns (the only ones that
+//   can hold a neighbour of the tile), P = exp2(s - m) as bf16 over the buffer's first 32
+//   columns (P = 0 in window columns 60..63);  O += P_s v_s  (TS MMA, N = d) with the rows
 //   of the other warps disabled through the MMA's output-lane mask, so non-owners never touch
-//   chunk s.
-// Each tile has its own MMA warp; QK runs two chunks ahead of PV, so S_{s+2} is ready when the
-// owners finish chunk s + 1. Each softmax warp zeroes its O rows when it starts a unit; its
-// epilogue runs after the PV of its last chunk. Every query sits at the same row and every
+//   slice s.
+// Each tile has its own MMA warp; QK runs two slices ahead of PV, so S_{s+2} is ready when the
+// owners finish slice s + 1. Each softmax warp zeroes its O rows when it starts a unit; its
+// epilogue runs after the PV of its last slice. Every query sits at the same row and every
 // neighbour at the same column whatever the packing, so a coordinate-carrying repack permutes
 // the output bit for bit.
 #include <math.h>
@@ -50,16 +53,17 @@
 namespace p3d {
 
 namespace lg {
-constexpr int BZ = 8, BY = 4, BX = 8;  // unit; two tiles of 8 x 4 x 4
+constexpr int BZ = 4, BY = 8, BX = 8;  // unit; two tiles of 4 x 4 x 8 (z, y, x)
 constexpr int kTiles = 2;
+constexpr int TY = BY / kTiles;        // 4 y-rows per tile
 constexpr int HY = BY + 2, HX = BX + 2;
-constexpr int kChunks = BZ + 2;        // halo z-slices
-constexpr int kSliceKeys = HY * HX;    // 60
-constexpr int kNK = 48;                // tile window (MMA N of QK, K of PV)
-constexpr int kNV = 36;                // window columns that can hold a neighbour
-constexpr int kWin = 24;               // first slice row of tile 1's window
-constexpr int kRows = kWin + kNK;      // 72 rows per stage
-constexpr int kStages = 4;
+constexpr int kChunks = BZ + 2;        // 6 halo z-slices
+constexpr int kSliceKeys = HY * HX;    // 100
+constexpr int kNK = 64;                // tile window (MMA N of QK, K of PV)
+constexpr int kNV = (TY + 2) * HX;     // 60 window columns that can hold a neighbour
+constexpr int kWin = TY * HX;          // 40: first slice row of tile 1's window
+constexpr int kRows = kWin + kNK;      // 104 rows per stage
+constexpr int kStages = 3;
 // warps: softmax 0-7 (tile = warp / 4; warps 0, 1, 4, 5 also prepare q tiles), slot boxes 8
 // (warp 9 idle), k/v producers 10-13, MMA 14-15 (tile = warp - 14)
 constexpr int kThreads = 512;
@@ -69,16 +73,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTileCols = 256;  // per tile: S buffers at 0 / 64, O at 128
 constexpr uint32_t kOCol = 128;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kBoxX = 16, kBoxY = 6, kBoxZ = 10;  // slot box: x from x0 - 4
+constexpr int kBoxX = 16, kBoxY = HY, kBoxZ = kChunks;  // slot box: x from x0 - 4
 constexpr int kBoxBytes = kBoxX * kBoxY * kBoxZ * 4;
 constexpr int kBoxPitch = 4096;  // box, then the unit index (int64) at kBoxBytes
 
 __device__ __forceinline__ uint32_t s_col(int b) { return b ? 64u : 0u; }
 
-// slice row of halo position (hy, hx): halo x 0-3, then 4-5, then 6-9, each block y-major
-__host__ __device__ constexpr int slice_row(int hy, int hx) {
-  return hx < 4 ? hy * 4 + hx : (hx < 6 ? 24 + hy * 2 + (hx - 4) : 36 + hy * 4 + (hx - 6));
-}
+// slice row of halo position (hy, hx): halo row major
+__host__ __device__ constexpr int slice_row(int hy, int hx) { return hy * HX + hx; }
 
 // Shared memory. Operands use the no-swizzle core-matrix layout: the 16-byte piece (row r,
 // column chunk c) of a q tile sits at c * kQCol + (r / 8) * 128 + (r % 8) * 16 and that of a
@@ -94,10 +96,12 @@ template <int D> struct Smem {
   static constexpr int kQ = 0;                            // [2 buffers][2 tiles] q tiles
   static constexpr int kK = kQ + 4 * kQBuf;               // [kStages] key chunks
   static constexpr int kV = kK + kStages * kStage;        // [kStages] value chunks
-  static constexpr int kBox = kV + kStages * kStage;      // [2] slot boxes (TMA: 128-aligned)
+  static constexpr int kBox = (kV + kStages * kStage + 127) / 128 * 128;  // [2] slot boxes (TMA)
   static constexpr int kBar = kBox + 2 * kBoxPitch;
   static constexpr int kBytes = kBar + 1024;
   static_assert(kBox % 128 == 0, "box alignment");
+  static_assert(kBoxBytes + 8 <= kBoxPitch, "slot box and unit index");
+  static_assert(kBytes <= 232448, "dynamic shared memory of one CTA");
   __device__ static int q_off(int r, int c) { return c * kQCol + (r >> 3) * 128 + (r & 7) * 16; }
 };
 
@@ -116,7 +120,7 @@ static_assert(8 * B_COUNT + 16 <= 1024, "barrier area");
 struct Params {
   pack3d_index ix;
   const __nv_bfloat16* q;      // [B, H, N, d]
-  const __nv_bfloat16* k_rot;  // rotated keys [B, H, N, d]
+  const __nv_bfloat16* k;      // keys [B, H_kv, N, d]: raw (ROT) or rotated
   const __nv_bfloat16* v;
   __nv_bfloat16* o_loc;
   float* lse_loc;  // optional
@@ -124,6 +128,7 @@ struct Params {
   int nbz, nby, nbx;
   int box_tma;        // slot boxes by TMA (else plain loads)
   int64_t units;      // batch * heads * units per field
+  int kv_group;       // query heads per KV head: k_rot and v rows of KV head bh / kv_group
   long long wait_budget;  // SM cycles of each bounded wait
 };
 
@@ -136,6 +141,13 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t* r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
                : "r"(taddr));
 }
 
@@ -171,13 +183,20 @@ static __device__ unsigned long long g_brick_t[512 * 32];
   } while (0)
 #endif
 
-// first and last softmax warp owning halo slice s
-__device__ __forceinline__ int owner_lo(int s) { return max(0, (s - 2) >> 1); }
-__device__ __forceinline__ int owner_hi(int s) { return min(3, s >> 1); }
+// first and last softmax warp owning halo slice s (warp w needs slices w .. w + 2)
+__device__ __forceinline__ int owner_lo(int s) { return max(0, s - 2); }
+__device__ __forceinline__ int owner_hi(int s) { return min(3, s); }
+// Parity of the wait of warp w on its S / P barrier of slice s (buffer s % 2) in unit ti:
+// per unit the buffer of parity w % 2 serves slices w and w + 2 (two phases), the other
+// buffer slice w + 1 (one phase).
+__host__ __device__ __forceinline__ uint32_t sp_parity(int w, int s, int ti) {
+  const int i = s - w;
+  return (i & 1) ? (uint32_t)(ti & 1) : (uint32_t)((i >> 1) & 1);
+}
 
 }  // namespace lg
 
-template <int D>
+template <int D, bool ROT>
 __global__ void __launch_bounds__(lg::kThreads, 1)
     k_local_tma(const __grid_constant__ CUtensorMap mg, const lg::Params P) {
   using namespace lg;
@@ -234,8 +253,8 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     tc::fence_mbar_init();
   }
   if (warp == W_BOX && lane == 0 && P.box_tma) tc::tma_prefetch_desc(&mg);
-  // rows 60..71 of every k/v stage are never written by the producers: zero them once (tile 1's
-  // MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
+  // rows 100..103 of every k/v stage are never written by the producers: zero them once
+  // (tile 1's MMAs read them; their scores are masked, and P = 0 times a zero v row is 0)
   for (int i = tid; i < kStages * 2 * KC * (kRows - kSliceKeys); i += kThreads) {
     const int row = kSliceKeys + i % (kRows - kSliceKeys), c = (i / (kRows - kSliceKeys)) % KC;
     const int blk = i / ((kRows - kSliceKeys) * KC);  // stage * 2 + tensor
@@ -257,7 +276,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     // 64 w .. 64 w + 63, one row per lane and pass -- loaded, rotated in registers by the row's
     // coordinates (axial RoPE) and stored in the operand layout -- then publishes its share
     // (QFULL: 64 arrivals per tile). Row r of a tile holds brick position
-    // (2 (r / 32) + (r % 32) / 16, (r / 4) % 4, r % 4); rows off the grid are zero.
+    // (r / 32, 4 tile + (r / 8) % 4, r % 8); rows off the grid or at empty sites are zero.
     auto prepare_q = [&](int64_t un, int nb, int qi) {
       int64_t qbh;
       int qz0, qy0, qx0;
@@ -268,8 +287,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
         const int r = 64 * w + 32 * pass + lane;
-        const int rw = r >> 5, rl = r & 31;
-        const int z = 2 * rw + (rl >> 4), y = (rl >> 2) & 3, x = 4 * tile + (rl & 3);
+        const int z = r >> 5, y = TY * tile + ((r >> 3) & 3), x = r & 7;
         const int slot = in_grid(qz0 + z, qy0 + y, qx0 + x)
                              ? qbox[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4]
                              : -1;
@@ -284,7 +302,8 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
           const int cv = axis == 0 ? cz : (axis == 1 ? cy : cx);
           // (cos, sin) of the piece's 4 rotation pairs: 32 contiguous bytes of the table
-          const float4* cs4 = reinterpret_cast<const float4*>(P.ix.rope + 2 * (cv * pairs + p0));
+          const float4* cs4 = reinterpret_cast<const float4*>(
+              P.ix.rope + 2 * rope_slot(P.ix.rope_rows, pairs, axis, cv, p0));
           const float4 ca = __ldg(cs4), cbv = __ldg(cs4 + 1);
           const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
           const uint32_t xin[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
@@ -311,7 +330,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       uint32_t tl = tbase;
       asm volatile("" : "+r"(ln), "+r"(tl));
       tl += ((uint32_t)(w * 32) << 16) + tile * kTileCols;
-      const int dz = ln >> 4, qy = (ln >> 2) & 3, qx = 4 * tile + (ln & 3);
+      const int qy = TY * tile + ((ln >> 3) & 3), qx = ln & 7;  // brick position (w, qy, qx)
       const int bb = ti & 1;
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + bb], (ti >> 1) & 1))) break;
       const int64_t u = unit_of(bb);
@@ -321,22 +340,23 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       int z0, y0, x0;
       origin(u, bh, z0, y0, x0);
       const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
-      const int cz = z0 + 2 * w + dz, cy = y0 + qy, cx = x0 + qx;
+      const int cz = z0 + w, cy = y0 + qy, cx = x0 + qx;
       const bool valid = cz < g.gz && cy < g.gy && cx < g.gx;
-      // neighbour bits of the warp's four slices: bit slice_row(hy, hx) - 24 tile of slice
-      // 2w + i
-      uint64_t nb[4] = {0ull, 0ull, 0ull, 0ull};
+      // neighbour bits of the warp's three slices: bit slice_row(hy, hx) - 40 tile of slice
+      // w + i, i = 1 + dz (empty sites, with slot -1, are no neighbours)
+      uint64_t nb[3] = {0ull, 0ull, 0ull};
       if (valid) {
 #pragma unroll
         for (int o = 0; o < 27; ++o) {
           const int ddz = o / 9 - 1, ddy = (o / 3) % 3 - 1, ddx = o % 3 - 1;
           const int hy = qy + 1 + ddy, hx = qx + 1 + ddx;
-          const int hz = 2 * w + dz + 1 + ddz;  // halo slice
+          const int hz = w + 1 + ddz;  // halo slice
           if (!in_grid(cz + ddz, cy + ddy, cx + ddx)) continue;
           if (box[(hz * kBoxY + hy) * kBoxX + hx + 3] < 0) continue;
           const uint64_t bit = 1ull << (slice_row(hy, hx) - kWin * tile);
-          nb[1 + ddz] |= dz == 0 ? bit : 0ull;  // slice index i = dz + 1 + ddz
-          nb[2 + ddz] |= dz == 1 ? bit : 0ull;
+          nb[0] |= ddz == -1 ? bit : 0ull;
+          nb[1] |= ddz == 0 ? bit : 0ull;
+          nb[2] |= ddz == 1 ? bit : 0ull;
         }
       }
       // this warp's O rows start at zero (the previous unit's epilogue has read them)
@@ -349,22 +369,23 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       uint64_t* pfull = &bars[B_PFULL + (tile * 4 + w) * 2];
       float m_run = -INFINITY, l_run = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int s = 2 * w + i, b = i & 1;
+      for (int i = 0; i < 3; ++i) {
+        const int s = w + i, b = s & 1;
         const uint32_t gs = (uint32_t)ti * kChunks + s;
-        if (!__all_sync(0xffffffffu, ab.wait(&sfull[b], (i >> 1) & 1))) {
+        if (!__all_sync(0xffffffffu, ab.wait(&sfull[b], sp_parity(w, s, ti)))) {
           ok = false;
           break;
         }
         if (ln == 0 && tile == 0) GTR(ti, 110 + w * 20 + i * 4);
         tc::tc_fence_after();
-        // the chunk's first 36 window scores (the rest never hold a neighbour of this tile);
+        // the slice's first 60 window scores (the rest never hold a neighbour of this tile);
         // entries off the 3x3x3 cube become -inf
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         uint32_t r[kNV];
-        tc::tmem_ld16(tl + s_col(b), *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-        tc::tmem_ld16(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-        lg::tmem_ld4(tl + s_col(b) + 32, &r[32]);
+        tc::tmem_ld32(tl + s_col(b), *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tc::tmem_ld16(tl + s_col(b) + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
+        lg::tmem_ld8(tl + s_col(b) + 48, &r[48]);
+        lg::tmem_ld4(tl + s_col(b) + 56, &r[56]);
         tc::tmem_wait_ld();
         const uint64_t win = nb[i];
 #pragma unroll
@@ -420,7 +441,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         }
         l_run += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
         tc::tmem_st16(tl + s_col(b), *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
-        lg::tmem_st8(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[8]>(&p[16]));
+        tc::tmem_st16(tl + s_col(b) + 16, *reinterpret_cast<uint32_t(*)[16]>(&p[16]));
         tc::tmem_wait_st();
         tc::tc_fence_before();
         tc::mbar_arrive(&pfull[b]);
@@ -442,8 +463,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           ow[c0 / 2 + k] =
               tc::pack_bf16(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
       }
-      const int slot =
-          valid ? box[((2 * w + dz + 1) * kBoxY + qy + 1) * kBoxX + qx + 4] : -1;
+      const int slot = valid ? box[((w + 1) * kBoxY + qy + 1) * kBoxX + qx + 4] : -1;
       __syncwarp();
       if (ln == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
       if (ln == 0 && tile == 0) GTR(ti, 190 + w);
@@ -529,10 +549,12 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           set_status(P.ix.status, PACK3D_ERR_TIMEOUT);
   } else if (warp >= W_PROD && warp < W_MMA) {
     // --------------------------------------------------------- k/v rows (128 threads)
-    // Halo slice s of rotated keys and values: 60 rows x d, one cp.async per 16-byte piece in
-    // row-contiguous order (rows off the grid are zero-filled). Each thread's copies arrive on
-    // the stage's barrier by themselves when they land, so the warps run ahead as far as the
-    // free stages allow.
+    // Halo slice s of keys and values: 100 rows x d, one cp.async per 16-byte piece in
+    // row-contiguous order (rows off the grid or at empty sites are zero-filled). Rotated keys:
+    // each thread's copies arrive on the stage's barrier by themselves when they land, so the
+    // warps run ahead as far as the free stages allow. Raw keys (ROT): slice s's copies are
+    // issued, then the thread waits for its copies of slice s - 1, rotates those key pieces in
+    // place and arrives for slice s - 1.
     const int pt = tid - W_PROD * 32;
     volatile int* pflag = abort_flag + 1;  // [2], used alternately
     int nwait = 0;
@@ -560,8 +582,42 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
                              ((uint32_t)c << 24))
                           : 0xffffffffu;
     }
-    const __nv_bfloat16* kg = P.k_rot;
+    const __nv_bfloat16* kg = P.k;
     const __nv_bfloat16* vg = P.v;
+    const int pairs = P.ix.rope_pairs;
+    // rotation of this thread's key pieces of slice s (stage st) in place: the key's
+    // coordinate is its halo position; pieces of rows off the grid stay zero
+    auto rotate_slice = [&](int s, int st, int z0, int y0, int x0) {
+      uint8_t* kd = smem + S::kK + st * S::kStage;
+      const int zc = z0 - 1 + s;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        if (pc[j] == 0xffffffffu) continue;
+        const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf, c = pc[j] >> 24;
+        const int y = y0 - 1 + hy, x = x0 - 1 + hx;
+        if (!in_grid(zc, y, x)) continue;
+        const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
+        const int cv = axis == 0 ? zc : (axis == 1 ? y : x);
+        const float4* cs4 = reinterpret_cast<const float4*>(
+            P.ix.rope + 2 * rope_slot(P.ix.rope_rows, pairs, axis, cv, p0));
+        const float4 ca = __ldg(cs4), cbv = __ldg(cs4 + 1);
+        const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
+        uint4* ptr = reinterpret_cast<uint4*>(kd + ((pc[j] & 0xffffu) << 4));
+        const uint4 xv = *ptr;
+        const uint32_t xin[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t xo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float e0 = __uint_as_float(xin[k] << 16);
+          const float e1 = __uint_as_float(xin[k] & 0xffff0000u);
+          xo[k] = tc::pack_bf16(e0 * cs[2 * k] - e1 * cs[2 * k + 1],
+                                e0 * cs[2 * k + 1] + e1 * cs[2 * k]);
+        }
+        *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+      }
+      tc::fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+      tc::mbar_arrive(&bars[B_KVFULL + st]);
+    };
     int ti = 0;
     uint32_t gs = 0;
     bool ok = true;
@@ -574,7 +630,8 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       int64_t bh;
       int z0, y0, x0;
       origin(u, bh, z0, y0, x0);
-      const int64_t rbase = bh * N;
+      const int64_t rbase = kv_of(bh, P.kv_group) * N;  // key and value rows of the KV head
+      int prev_st = 0;
       for (int s = 0; s < kChunks; ++s, ++gs) {
         const int st = gs % kStages;
         if (gs >= (uint32_t)kStages && !pwait(&bars[B_KVEMPTY + st], ((gs / kStages) - 1) & 1)) {
@@ -598,10 +655,23 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           tc::cp_async16(kd + off, kg + src, slot >= 0);
           tc::cp_async16(vd + off, vg + src, slot >= 0);
         }
-        tc::cp_async_arrive_noinc(&bars[B_KVFULL + st]);
+        if constexpr (ROT) {
+          tc::cp_async_commit();
+          if (s > 0) {
+            tc::cp_async_wait_group<1>();  // this thread's copies of slice s - 1 have landed
+            rotate_slice(s - 1, prev_st, z0, y0, x0);
+          }
+          prev_st = st;
+        } else {
+          tc::cp_async_arrive_noinc(&bars[B_KVFULL + st]);
+        }
         if (pt == 0) GTR(ti, 11 + s * 2);
       }
       if (!ok) break;
+      if constexpr (ROT) {
+        tc::cp_async_wait_group<0>();
+        rotate_slice(kChunks - 1, prev_st, z0, y0, x0);
+      }
       // this warp's reads of the slot box are done
       __syncwarp();
       if ((pt & 31) == 0) tc::mbar_arrive(&bars[B_BOXFREE + bb]);
@@ -618,7 +688,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
     // no-swizzle descriptors: q and k K-major (lbo = column-chunk stride, sbo = 8 rows), v
     // MN-major (lbo = 8 key rows, sbo = column-chunk stride); the tile's window starts at
-    // slice row 24 tile
+    // slice row 40 tile
     const uint64_t qd0 = tc::smem_desc(tc::smem_u32(smem + S::kQ), S::kQCol, 128);
     const uint64_t kd0 =
         tc::smem_desc(tc::smem_u32(smem + S::kK + (kWin * tile / 8) * 128), S::kChunkCol, 128);
@@ -668,7 +738,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       for (int s = 0; s < kChunks && ok; ++s, ++gs) {
         const int st = gs % kStages, b = s & 1;
         const int wlo = owner_lo(s), whi = owner_hi(s);
-        for (int w = wlo; w <= whi && ok; ++w) ok = wwait(&pfull[2 * w + b], ((s - 2 * w) >> 1) & 1);
+        for (int w = wlo; w <= whi && ok; ++w) ok = wwait(&pfull[2 * w + b], sp_parity(w, s, ti));
         if (!ok) break;
         if (lane == 0 && tile == 0) GTR(ti, 60 + s * 4);
         tc::tc_fence_after();
@@ -684,7 +754,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
                               id_pv, 1u, m0, m1, m2, m3);
           tc::tc_commit(&bars[B_KVEMPTY + st]);
           tc::tc_commit(pvall);
-          if ((s & 1) && s >= 3) tc::tc_commit(&bars[B_EPI + tile * 4 + ((s - 3) >> 1)]);
+          if (s >= 2) tc::tc_commit(&bars[B_EPI + tile * 4 + (s - 2)]);  // warp s-2 done
         }
         __syncwarp();
         if (lane == 0 && tile == 0) GTR(ti, 61 + s * 4);
@@ -720,14 +790,14 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* k_rot,
-                             const void* v, int64_t bh, float scale, void* o_loc, float* lse_loc,
+template <int D, bool ROT>
+cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* k, const void* v,
+                             int64_t bh, int kv_group, float scale, void* o_loc, float* lse_loc,
                              cudaStream_t s) {
   using namespace lg;
   static std::atomic<uint64_t> attr_done{0};
-  if (smem_attr_once(reinterpret_cast<const void*>(k_local_tma<D>), Smem<D>::kBytes, attr_done) !=
-      cudaSuccess)
+  if (smem_attr_once(reinterpret_cast<const void*>(k_local_tma<D, ROT>), Smem<D>::kBytes,
+                     attr_done) != cudaSuccess)
     return cudaErrorInvalidValue;
   Params p;
   p.ix = ix;
@@ -735,6 +805,7 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   p.lse_loc = lse_loc;
   p.scale_log2 = scale * kLog2e;
   p.wait_budget = wait_budget_cycles();
+  p.kv_group = kv_group;
   p.nbz = (ix.geom.gz + BZ - 1) / BZ;
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;
@@ -742,7 +813,7 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   if (p.units <= 0) return cudaSuccess;
   if (!ix.status || p.units >= 0x7fffffffLL) return cudaErrorInvalidValue;  // unit counter
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_rot = static_cast<const __nv_bfloat16*>(k_rot);
+  p.k = static_cast<const __nv_bfloat16*>(k);
   p.v = static_cast<const __nv_bfloat16*>(v);
   CUtensorMap mg;
   memset(&mg, 0, sizeof(mg));
@@ -751,17 +822,22 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
                   : 0;
   const int64_t cap = sm_count();
   const unsigned grid = (unsigned)(p.units < cap ? p.units : cap);
-  k_local_tma<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(mg, p);
+  k_local_tma<D, ROT><<<grid, kThreads, Smem<D>::kBytes, s>>>(mg, p);
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void* k_rot,
-                               const void* v, int64_t bh, float scale, void* o_loc,
-                               float* lse_loc, cudaStream_t s) {
+// k_rotated: k holds R(c) k (pack3d_summarize_rotated); otherwise the kernel rotates the keys.
+cudaError_t local_tma_dispatch(const pack3d_index& ix, const void* q, const void* k,
+                               const void* v, int64_t bh, int kv_group, float scale,
+                               bool k_rotated, void* o_loc, float* lse_loc, cudaStream_t s) {
   if (ix.geom.head_dim == 96)
-    return launch_local_tma<96>(ix, q, k_rot, v, bh, scale, o_loc, lse_loc, s);
-  return launch_local_tma<48>(ix, q, k_rot, v, bh, scale, o_loc, lse_loc, s);
+    return k_rotated
+               ? launch_local_tma<96, false>(ix, q, k, v, bh, kv_group, scale, o_loc, lse_loc, s)
+               : launch_local_tma<96, true>(ix, q, k, v, bh, kv_group, scale, o_loc, lse_loc, s);
+  return k_rotated
+             ? launch_local_tma<48, false>(ix, q, k, v, bh, kv_group, scale, o_loc, lse_loc, s)
+             : launch_local_tma<48, true>(ix, q, k, v, bh, kv_group, scale, o_loc, lse_loc, s);
 }
 
 }  // namespace p3d

@@ -16,12 +16,20 @@
  *
  * Conventions shared by every call:
  *   - Tensors are dense, row-major [B, H, N, d] with N in MEMORY order (the packing);
- *     gate logits are [B, H, N]; lse outputs are float32 [B, H, N].
- *   - Summaries (ksum, vsum) hold M = number of blocks summaries per (b, h), block ids raster
- *     over the block grid, in SUMMARY TILES: the summaries of each (b, h) are grouped in tiles
- *     of 64 (the last tile zero-padded); a tile is d/8 columns of 64 summaries x 8 consecutive
- *     elements. Element (b, h, m, e) sits at element offset
- *         (((b*H + h)*T + m/64)*(d/8) + e/8)*512 + (m%64)*8 + e%8,   T = ceil(M/64),
+ *     gate logits are [B, H, N]; lse outputs are float32 [B, H, N]. Keys and values may have
+ *     fewer heads than queries (GQA / MQA: [B, H_kv, N, d], H_kv dividing H; query head h
+ *     uses KV head h / (H / H_kv); project page Ch.3 Contract 2 "summaries per KV head",
+ *     paper summary §D.1); the calls take both head counts (kv_heads 0 means H_kv = H).
+ *   - Validity: a field holds N <= Gz*Gy*Gx tokens at distinct lattice sites; the sites
+ *     without a token are empty (project page Ch.3 Contract 1, "coordinate offsets and
+ *     validity"; Ch.4 Proposition 2). Neighbourhoods skip empty sites. Blocks tile the grid
+ *     from the origin and may stick out of it at the far edges (partial blocks); a summary is
+ *     the mean over its members present, and a summary with none takes part in no softmax.
+ *   - Summaries (ksum, vsum) hold M summaries per (b, h_kv), ids raster over the summary
+ *     grid, in SUMMARY TILES: the summaries of each (b, h_kv) are grouped in tiles of 64 (the
+ *     last tile zero-padded); a tile is d/8 columns of 64 summaries x 8 consecutive
+ *     elements. Element (b, h_kv, m, e) sits at element offset
+ *         (((b*H_kv + h_kv)*T + m/64)*(d/8) + e/8)*512 + (m%64)*8 + e%8,   T = ceil(M/64),
  *     and a buffer takes pack3d_summary_bytes(...) bytes. A tile is exactly the tensor-core
  *     operand layout of a 64-summary chunk, so the forward moves it with one bulk copy.
  *   - dtype: PACK3D_F32 or PACK3D_BF16 for q, k, v, gate, summaries, outputs and gradients.
@@ -33,8 +41,7 @@
  *     that stream unless stated otherwise. Argument errors are returned synchronously before
  *     any launch; a launch failure returns PACK3D_ERR_CUDA.
  *   - d (head_dim) must be 48 or 96 (a multiple of 6 is required by axial RoPE; other values
- *     return PACK3D_ERR_UNSUPPORTED). The grid must be fully populated (N = Gz*Gy*Gx) and
- *     divisible by the block extents.
+ *     return PACK3D_ERR_UNSUPPORTED).
  */
 #ifndef PACK3D_H
 #define PACK3D_H
@@ -68,12 +75,27 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
  * otherwise the call returns UNSUPPORTED. */
 #define PACK3D_K_ROTATED 2u
 
+/* pack3d_geom.summary_rope: where the global branch's keys are rotated. */
+#define PACK3D_ROPE_TOKEN 0   /* each key at its own coordinate, then pooled (exact; Ch.3
+                                 "Rotate first, then pool", paper summary §B.5) */
+#define PACK3D_ROPE_CENTRE 1  /* the unrotated keys pooled, the mean rotated once at the centre
+                                 of the summary's box (the cheaper variant; Ch.3 "One block, two
+                                 ways to summarize it", paper summary §B.7-§B.8) */
+
 /* Geometry of a packed field: grid extents, block (summary) extents, RoPE plan. */
 typedef struct {
   int32_t gz, gy, gx;   /* grid extents, each in [1, 1024] */
-  int32_t bz, by, bx;   /* block extents, each dividing the grid extent */
+  int32_t bz, by, bx;   /* block extents, each in [1, grid extent] */
   int32_t head_dim;     /* d: 48 or 96 */
   float rope_base;      /* RoPE base per axis (10000 on the pages) */
+  int32_t pz, py, px;   /* second pooling stage (note under Figure 1 of the project page): each
+                           summary is the mean of the non-empty block summaries of a
+                           pz x py x px group of the block grid; 0 or 1 on every axis: none.
+                           Each extent in [0, 1024]. */
+  int32_t summary_rope; /* PACK3D_ROPE_TOKEN or PACK3D_ROPE_CENTRE */
+  float spacing[3];     /* RoPE angle of axis a is spacing[a] * c_a * theta_p: a fixed
+                           anisotropic or normalised coordinate map (paper summary §B.2, §B.9);
+                           0 means 1. Neighbourhoods and blocks stay on the integer lattice. */
 } pack3d_geom;
 
 /* Index tables of one packed field (one geometry, one packing). Filled by
@@ -81,25 +103,38 @@ typedef struct {
  * Coordinates are stored packed as (z << 20) | (y << 10) | x. */
 typedef struct {
   pack3d_geom geom;
-  int64_t n;              /* tokens N = Gz*Gy*Gx */
-  int64_t m;              /* summaries M = (Gz/bz)*(Gy/by)*(Gx/bx) */
+  int64_t n;              /* tokens present, N <= Gz*Gy*Gx */
+  int64_t m;              /* summaries M the global branch attends to (second stage, if any) */
+  int64_t n_blocks;       /* first-stage blocks ceil(Gz/bz)*ceil(Gy/by)*ceil(Gx/bx) */
   int32_t block_volume;   /* v = bz*by*bx */
   int32_t rope_pairs;     /* d / 6 rotation pairs per axis */
   int32_t rope_rows;      /* max(Gz, Gy, Gx): coordinates covered by the rotation table */
+  int32_t group_volume;   /* first-stage blocks per summary, pz*py*px (1 without a 2nd stage) */
+  int32_t sum_ext[3];     /* lattice extents (z, y, x) of a summary's box: block * group */
+  int32_t sum_grid[3];    /* summaries per axis, ceil(G / sum_ext); M is their product */
+  int32_t n_empty;        /* summaries with no member present */
   int32_t reserved;
   int32_t* coord;         /* device [N]      packed coordinate of the token at each slot */
-  int32_t* inv;           /* device [Gz*Gy*Gx] memory slot of each raster site (-1: none) */
+  int32_t* inv;           /* device [Gz*Gy*Gx] memory slot of each raster site (-1: empty) */
   int32_t* nbr;           /* device [N, 27]  slot of c + delta_o, o = 9(dz+1)+3(dy+1)+(dx+1);
-                             -1 outside the grid */
-  int32_t* block_of;      /* device [N]      block id of each token */
+                             -1 outside the grid or at an empty site */
+  int32_t* block_of;      /* device [N]      first-stage block id of each token */
   int32_t* slot_of;       /* device [N]      canonical slot inside its block (raster) */
-  int32_t* members;       /* device [M, v]   slot of the member at each canonical slot */
-  int32_t* count;         /* device [M]      members present */
-  float* rope;            /* device [rope_rows, rope_pairs, 2] (cos, sin) of c * theta_p */
+  int32_t* members;       /* device [n_blocks, v] slot of the member at each canonical slot */
+  int32_t* count;         /* device [n_blocks] members present */
+  int32_t* sum_of;        /* device [N]      summary id of each token */
+  int32_t* groups;        /* device [M, group_volume] first-stage block ids of each summary,
+                             raster inside the group; -1 past the block grid */
+  int32_t* count2;        /* device [M]      non-empty first-stage blocks of each summary */
+  uint32_t* empty;        /* device [ceil(M/32)] bit m%32 of word m/32 set: summary m empty */
+  float* rope;            /* device [3, rope_rows, rope_pairs, 2] (cos, sin) of
+                             spacing[a] * c * theta_p for axis a */
+  float* rope_c;          /* device [M, d/2, 2] (cos, sin) of the angles of each summary's box
+                             centre, pair e/2 of dims (e, e+1) (summary-centre RoPE) */
   int32_t* status;        /* device [4]      status words written by kernels: [0] first error;
-                             [2], [3] the work counter of the bf16 rotated-key local kernel
-                             (zero between calls; calls that use one index must therefore be
-                             ordered, e.g. on one stream) */
+                             [1] empty summaries (index build); [2], [3] the work counter of
+                             the bf16 rotated-key local kernel (zero between calls; calls that
+                             use one index must therefore be ordered, e.g. on one stream) */
 } pack3d_index;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -121,18 +156,22 @@ size_t pack3d_index_bytes(const pack3d_geom* g, int64_t n);
  * buf      device buffer of at least pack3d_index_bytes(g, n) bytes, 256-byte aligned; it
  *          holds every table and must outlive `out`'s use.
  * out      host   filled with the table pointers and sizes.
- * Errors: INVALID_ARG, UNSUPPORTED (n != Gz*Gy*Gx, d not 48/96), WORKSPACE, ALIGN, and --
- * after one stream synchronisation at the end of the call -- DUP_COORD or COORD_RANGE
- * detected by the kernels. */
+ * n          tokens present, 1 <= n <= Gz*Gy*Gx (the other sites are empty).
+ * Errors: INVALID_ARG, UNSUPPORTED (d not 48/96), WORKSPACE, ALIGN, and -- after one stream
+ * synchronisation at the end of the call, which also reads the number of empty summaries --
+ * DUP_COORD or COORD_RANGE detected by the kernels. */
 pack3d_status pack3d_build_index(const pack3d_geom* g, const int32_t* coords,
                                  const int64_t* perm, int64_t n, void* buf, size_t buf_bytes,
                                  pack3d_index* out, void* stream);
 
 /* Rotate-then-pool block summaries: ksum[m] = mean over members j of R(c_j) k_j and
  * vsum[m] = mean of v_j, summed in canonical-slot order (project page Ch.3 "Rotate first,
- * then pool"; paper summary §3.2, §B.5).
- * k, v       device [B, H, N, d] dtype;  ksum, vsum device summary tiles, dtype, each of
- *            pack3d_summary_bytes(idx, dtype, B, H) bytes (outputs; the padding is zeroed). */
+ * then pool"; paper summary §3.2, §B.5); with a second stage, the mean of the non-empty block
+ * means of each group, in group order; with PACK3D_ROPE_CENTRE, the unrotated keys are
+ * pooled and the mean is rotated at the centre of the summary's box.
+ * k, v       device [B, H_kv, N, d] dtype (`heads` is H_kv here: summaries are per KV head);
+ * ksum, vsum device summary tiles, dtype, each of pack3d_summary_bytes(idx, dtype, B, H_kv)
+ *            bytes (outputs; the padding and empty summaries are zero). */
 pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const void* v,
                                int dtype, int batch, int heads, void* ksum, void* vsum,
                                void* stream);
@@ -141,14 +180,15 @@ pack3d_status pack3d_summarize(const pack3d_index* idx, const void* k, const voi
  * k_rot[b,h,j] = R(c_j) k[b,h,j] (axial RoPE of each token's coordinate, rounded to dtype).
  * The pages rotate q and k inside attention; doing it for k once here, where every key row is
  * already read, lets the local branch fetch key rows with plain row gathers.
- * k_rot      device [B, H, N, d] dtype (output); must not alias k. */
+ * k_rot      device [B, H_kv, N, d] dtype (output); must not alias k. */
 pack3d_status pack3d_summarize_rotated(const pack3d_index* idx, const void* k, const void* v,
                                        int dtype, int batch, int heads, void* ksum, void* vsum,
                                        void* k_rot, void* stream);
 
 /* PACK3D forward: local branch + global branch over (ksum, vsum) + sigmoid mixer
  * (project page Ch.3 Contracts 1-3; paper summary §3.2, §3.3, §3.5).
- * q, k, v    device [B, H, N, d] dtype;  gate device [B, H, N] dtype (logits a).
+ * q          device [B, H, N, d] dtype;  k, v device [B, H_kv, N, d] dtype (kv_heads = H_kv,
+ *            dividing H; 0 means H);  gate device [B, H, N] dtype (logits a).
  * ksum, vsum device summary tiles from pack3d_summarize of the same k, v.
  * scale      softmax scale tau (both branches); pass 1/sqrt(d) for the usual choice.
  * flags      0, or PACK3D_EXCLUDE_NEAR and/or PACK3D_K_ROTATED (k is then the k_rot of
@@ -161,9 +201,9 @@ pack3d_status pack3d_summarize_rotated(const pack3d_index* idx, const void* k, c
  *            o_glob = 0. */
 pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void* k,
                               const void* v, const void* gate, const void* ksum,
-                              const void* vsum, int dtype, int batch, int heads, float scale,
-                              uint32_t flags, void* o, float* lse_loc, float* lse_glob,
-                              void* o_loc, void* o_glob, void* stream);
+                              const void* vsum, int dtype, int batch, int heads, int kv_heads,
+                              float scale, uint32_t flags, void* o, float* lse_loc,
+                              float* lse_glob, void* o_loc, void* o_glob, void* stream);
 
 /* The two halves of pack3d_attn_fwd as separate calls (same kernels, same results).
  * pack3d_attn_local: the local branch alone (project page Ch.3 Contract 1; paper summary
@@ -175,35 +215,39 @@ pack3d_status pack3d_attn_fwd(const pack3d_index* idx, const void* q, const void
  *   o_glob as in pack3d_attn_fwd. flags: 0 or PACK3D_EXCLUDE_NEAR.
  * Errors as pack3d_attn_fwd. */
 pack3d_status pack3d_attn_local(const pack3d_index* idx, const void* q, const void* k,
-                                const void* v, int dtype, int batch, int heads, float scale,
-                                uint32_t flags, void* o_loc, float* lse_loc, void* stream);
+                                const void* v, int dtype, int batch, int heads, int kv_heads,
+                                float scale, uint32_t flags, void* o_loc, float* lse_loc,
+                                void* stream);
 pack3d_status pack3d_attn_global(const pack3d_index* idx, const void* q, const void* gate,
                                  const void* ksum, const void* vsum, const void* o_loc,
-                                 int dtype, int batch, int heads, float scale, uint32_t flags,
-                                 void* o, float* lse_glob, void* o_glob, void* stream);
+                                 int dtype, int batch, int heads, int kv_heads, float scale,
+                                 uint32_t flags, void* o, float* lse_glob, void* o_glob,
+                                 void* stream);
 
-/* Bytes of one summary buffer (ksum or vsum) for B x H heads in summary tiles. Host-only;
- * 0 if the arguments are invalid. */
+/* Bytes of one summary buffer (ksum or vsum) for B x H_kv heads in summary tiles (pass the
+ * KV head count as `heads`). Host-only; 0 if the arguments are invalid. */
 size_t pack3d_summary_bytes(const pack3d_index* idx, int dtype, int batch, int heads);
 
-/* Bytes of device workspace pack3d_attn_bwd needs. Host-only. */
-size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch, int heads);
+/* Bytes of device workspace pack3d_attn_bwd needs. Host-only; 0 if the arguments are invalid. */
+size_t pack3d_bwd_workspace_bytes(const pack3d_index* idx, int dtype, int batch, int heads,
+                                  int kv_heads);
 
 /* PACK3D backward: gradients of sum(dO * o) through the mixer, both softmax branches, the
  * mean pooling and the axial RoPE (paper summary §3.4: the backward follows the forward's
  * streamed access pattern).
  * Inputs as in pack3d_attn_fwd plus the forward's saved o_loc, o_glob (dtype), lse_loc,
  * lse_glob (float32) and the upstream gradient dO [B, H, N, d] dtype.
- * Outputs dq, dk, dv [B, H, N, d] dtype and dgate [B, H, N] dtype (gradient w.r.t. the gate
- * logit). workspace: device, >= pack3d_bwd_workspace_bytes bytes, 256-byte aligned;
- * contents on entry are ignored. */
+ * Outputs dq [B, H, N, d], dk, dv [B, H_kv, N, d] (a KV head's gradients sum over its query
+ * heads) and dgate [B, H, N], all dtype (dgate: gradient w.r.t. the gate logit).
+ * workspace: device, >= pack3d_bwd_workspace_bytes bytes, 256-byte aligned; contents on entry
+ * are ignored. */
 pack3d_status pack3d_attn_bwd(const pack3d_index* idx, const void* q, const void* k,
                               const void* v, const void* gate, const void* ksum,
                               const void* vsum, const void* o_loc, const void* o_glob,
                               const float* lse_loc, const float* lse_glob, const void* dO,
-                              int dtype, int batch, int heads, float scale, uint32_t flags,
-                              void* dq, void* dk, void* dv, void* dgate, void* workspace,
-                              size_t workspace_bytes, void* stream);
+                              int dtype, int batch, int heads, int kv_heads, float scale,
+                              uint32_t flags, void* dq, void* dk, void* dv, void* dgate,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* Largest backward workspace pack3d_attn_bwd_noalloc can serve from its built-in buffer. */
 #define PACK3D_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -225,8 +269,8 @@ pack3d_status pack3d_attn_bwd_noalloc(const pack3d_index* idx, const void* q, co
                                       const void* vsum, const void* o_loc, const void* o_glob,
                                       const float* lse_loc, const float* lse_glob,
                                       const void* dO, int dtype, int batch, int heads,
-                                      float scale, uint32_t flags, void* dq, void* dk, void* dv,
-                                      void* dgate, void* stream);
+                                      int kv_heads, float scale, uint32_t flags, void* dq,
+                                      void* dk, void* dv, void* dgate, void* stream);
 
 /* Reads (after synchronising `stream`) and clears the index's device status word: OK, or
  * the first device-detected error (DUP_COORD, COORD_RANGE, TIMEOUT). */

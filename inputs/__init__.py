@@ -12,6 +12,9 @@ has two indices"; paper summary §3.1 and Table 9):
 
 Packings named on the pages: raster, Morton (Z-order), block-contiguous ("raster_block":
 blocks in raster order, raster order inside each block) and a seeded uniform random order.
+A workload may also leave lattice sites empty (`occupancy` < 1: a seeded subset of the sites
+holds tokens) and give k, v fewer heads than q (`kv_heads`); `pool2`, `summary_rope` and
+`spacing` describe its summary and RoPE plan and are passed through untouched.
 """
 from __future__ import annotations
 
@@ -58,10 +61,8 @@ def packing(kind, grid, block=(4, 4, 4), seed=1):
         return ids[np.argsort(_morton_code(unravel(ids, grid)), kind="stable")]
     if kind == "raster_block":
         bz, by, bx = (int(b) for b in block)
-        if gz % bz or gy % by or gx % bx:
-            raise ValueError("block-contiguous packing needs the grid divisible by the block")
         c = unravel(ids, grid).astype(np.int64)
-        nby, nbx = gy // by, gx // bx
+        nby, nbx = -(-gy // by), -(-gx // bx)  # blocks at the far edges may be partial
         blk = ((c[:, 0] // bz) * nby + c[:, 1] // by) * nbx + c[:, 2] // bx
         inner = ((c[:, 0] % bz) * by + c[:, 1] % by) * bx + c[:, 2] % bx
         key = blk * (bz * by * bx) + inner
@@ -74,6 +75,18 @@ def packing(kind, grid, block=(4, 4, 4), seed=1):
 
 def coords_of(perm, grid):
     return unravel(perm, grid)
+
+
+def occupied(perm, grid, occupancy, seed=3):
+    """Keep a seeded fraction of the lattice sites (the field's valid tokens): site r holds a
+    token when a uniform draw for r is below `occupancy`; memory order is kept."""
+    if occupancy >= 1.0:
+        return np.asarray(perm)
+    g = torch.Generator().manual_seed(int(seed))
+    keep = (torch.rand(grid_volume(grid), generator=g) < occupancy).numpy()
+    keep[np.asarray(perm)[0]] = True  # never empty
+    perm = np.asarray(perm)
+    return perm[keep[perm]]
 
 
 def field(batch, heads, grid, d, *, qkv_std=1.0, seed=0, gen_dtype=torch.float32):
@@ -113,8 +126,8 @@ def unpack(x, perm, token_dim=2):
 
 # --- named workloads -------------------------------------------------------------------------
 # Sizes follow the pages' workloads: the 8x8x8 / 2x2x2 field of the project page's "two-indices
-# lab" (Chapter 1), and 65,536- and 262,144-token fields (paper summary §4.3, project page
-# Chapter 3 Contract 2), with 4x4x4 blocks.
+# lab" (Chapter 1), 65,536- and 262,144-token fields (paper summary §4.3, project page
+# Chapter 3 Contract 2) with 4x4x4 blocks, and the 1M-token point of the latency sweep.
 WORKLOADS = {
     "tiny_8x8x8_fp32": dict(grid=(8, 8, 8), block=(2, 2, 2), batch=1, heads=1, d=48,
                             dtype="fp32", packing="raster", qkv_std=1.0, exclude_near=False),
@@ -130,6 +143,11 @@ WORKLOADS = {
     "field65k_fwdbwd_bf16": dict(grid=(32, 32, 64), block=(4, 4, 4), batch=2, heads=8, d=96,
                                  dtype="bf16", packing="raster_block", qkv_std=96 ** -0.5,
                                  exclude_near=False),
+    # the pages' high-token timing point (project page Ch.9: 1M tokens, 4,096 summaries per KV
+    # head): 4x4x4 blocks pooled again over 1x2x2 groups, 256 tokens per summary
+    "field1m_bf16": dict(grid=(64, 128, 128), block=(4, 4, 4), pool2=(1, 2, 2), batch=1,
+                         heads=8, d=96, dtype="bf16", packing="raster_block",
+                         qkv_std=96 ** -0.5, exclude_near=False),
 }
 
 
@@ -145,9 +163,15 @@ def make_workload(name_or_cfg, *, packing_kind=None, seed=0, perm_seed=1):
     grid, block = tuple(cfg["grid"]), tuple(cfg["block"])
     q, k, v, a = field(cfg["batch"], cfg["heads"], grid, cfg["d"], qkv_std=cfg["qkv_std"],
                        seed=seed)
+    hkv = cfg.get("kv_heads") or cfg["heads"]
+    k, v = k[:, :hkv].contiguous(), v[:, :hkv].contiguous()  # GQA: the KV heads' rows
     if cfg["dtype"] == "bf16":
         q, k, v, a = (t.to(torch.bfloat16).to(torch.float32) for t in (q, k, v, a))
-    perm = packing(kind, grid, block, seed=perm_seed)
+    perm = occupied(packing(kind, grid, block, seed=perm_seed), grid, cfg.get("occupancy", 1.0))
+    cfg.setdefault("pool2", (1, 1, 1))
+    cfg.setdefault("summary_rope", "token")
+    cfg.setdefault("spacing", (1.0, 1.0, 1.0))
+    cfg.setdefault("kv_heads", cfg["heads"])
     out = dict(cfg)
     out.update(packing=kind, perm=perm, coords=coords_of(perm, grid),
                q=pack(q, perm), k=pack(k, perm), v=pack(v, perm), a=pack(a, perm))

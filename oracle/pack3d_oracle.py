@@ -71,13 +71,15 @@ def _ceil_div(a, b):
     return -(-int(a) // int(b))
 
 
-def build_index(coords, grid, block, pool2=(1, 1, 1)):
+def build_index(coords, grid, block, pool2=(1, 1, 1), nbr_rows=None):
     """Index tables of a packed field, built by looping over tokens.
 
     coords: int [N, 3] -- (z, y, x) of the token at memory slot i; N may be smaller than the
     number of lattice sites (the sites without a token are empty). Blocks tile the grid from
     the origin; those at the far edges may stick out of it.
     pool2: extents of the second pooling stage's groups over the block grid ((1, 1, 1): none).
+    nbr_rows: fill the neighbour table for these memory slots only (the other rows stay -1),
+    for fields too large to loop over every token's neighbourhood in Python.
     Returns dict(inv, nbr, block_of, slot_of, members, count, n_blocks, block_volume,
     groups, count2, sum_of, n_summaries, summary_block).
     """
@@ -96,7 +98,7 @@ def build_index(coords, grid, block, pool2=(1, 1, 1)):
         inv[r] = i
 
     nbr = np.full((n, 27), -1, dtype=np.int64)
-    for i in range(n):
+    for i in (range(n) if nbr_rows is None else (int(r) for r in nbr_rows)):
         z, y, x = (int(t) for t in coords[i])
         for o, (dz, dy, dx) in enumerate(OFFSETS):
             zz, yy, xx = z + dz, y + dy, x + dx

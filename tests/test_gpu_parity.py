@@ -45,7 +45,9 @@ def tdtype(dt):
 
 def gpu_index(w, d, via="coords"):
     m = p3d()
-    geom = m.make_geom(w["grid"], w["block"], d)
+    geom = m.make_geom(w["grid"], w["block"], d, pool2=w.get("pool2", (1, 1, 1)),
+                       summary_rope=w.get("summary_rope", "token"),
+                       spacing=w.get("spacing", (1.0, 1.0, 1.0)))
     if via == "coords":
         return m.pack3d_build_index(geom, coords=torch.from_numpy(w["coords"]).cuda())
     return m.pack3d_build_index(geom, perm=torch.from_numpy(np.asarray(w["perm"])).cuda())
@@ -94,6 +96,16 @@ def compare_tables(ix, w, ref):
     assert np.array_equal(ix.table("slot_of", (n,)).cpu().numpy(), ref["slot_of"])
     assert np.array_equal(ix.table("members", (M, vol)).cpu().numpy(), ref["members"])
     assert np.array_equal(ix.table("count", (M,)).cpu().numpy(), ref["count"])
+    # summaries: the second pooling stage's groups, per-summary block counts and empty bits
+    S, gv = ref["groups"].shape
+    assert ix.m == S == ref["n_summaries"] and int(ix.struct.n_blocks) == M
+    assert np.array_equal(ix.table("sum_of", (n,)).cpu().numpy(), ref["sum_of"])
+    assert np.array_equal(ix.table("groups", (S, gv)).cpu().numpy(), ref["groups"])
+    assert np.array_equal(ix.table("count2", (S,)).cpu().numpy(), ref["count2"])
+    words = ix.table("empty", ((S + 31) // 32,)).cpu().numpy().view(np.uint32)
+    bits = (words[np.arange(S) // 32] >> (np.arange(S) % 32)) & 1
+    assert np.array_equal(bits == 1, ref["count2"] == 0)
+    assert int(ix.struct.n_empty) == int((ref["count2"] == 0).sum())
 
 
 @pytest.mark.parametrize("grid,block", [((8, 8, 8), (2, 2, 2)), ((6, 10, 12), (3, 2, 4)),
@@ -119,12 +131,14 @@ def test_index_tables_bit_exact_65k_field(kind):
 
 def test_rope_table_matches_theta_plan():
     w = small((4, 6, 9), (1, 1, 1), 1, 1, 96, "fp32", "raster")
+    w["spacing"] = (0.5, 1.0, 2.0)
     ix = gpu_index(w, 96)
-    tab = ix.rope_table().cpu().numpy().astype(np.float64)
+    tab = ix.rope_table().cpu().numpy().astype(np.float64)  # [axis, coordinate, pair, 2]
     theta = orc.rope_theta(96)
-    ang = np.arange(9)[:, None] * theta[None, :]
-    assert np.abs(tab[..., 0] - np.cos(ang)).max() < 1e-6
-    assert np.abs(tab[..., 1] - np.sin(ang)).max() < 1e-6
+    for a, sp in enumerate(w["spacing"]):
+        ang = sp * np.arange(9)[:, None] * theta[None, :]
+        assert np.abs(tab[a, ..., 0] - np.cos(ang)).max() < 1e-6
+        assert np.abs(tab[a, ..., 1] - np.sin(ang)).max() < 1e-6
 
 
 def test_index_errors_are_reported():
@@ -223,8 +237,8 @@ def sampled_compare(w, exclude_near, heads=((0, 0), (-1, -1)), count=96, rotated
         for key in ("o", "lse_loc", "lse_glob", "o_loc", "o_glob"):
             gv = g[key][b, h][rows] if key.startswith("o") else g[key][b, h][rows]
             assert_close(np64(gv), ref[key][0, 0], w["dtype"], f"{key}[{b},{h}]")
-        assert_close(np64(p3d().summary_rows(g["ksum"], idx["n_blocks"])[b, h]), ref["ksum"][0, 0],
-                     w["dtype"], "ksum")
+        assert_close(np64(p3d().summary_rows(g["ksum"], idx["n_summaries"])[b, h]),
+                     ref["ksum"][0, 0], w["dtype"], "ksum")
     return g
 
 

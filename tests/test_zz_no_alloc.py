@@ -56,11 +56,11 @@ def test_noalloc_backward_rejects_problems_beyond_its_buffer():
     buf = torch.empty(64, dtype=torch.float32, device="cuda")
     p = ctypes.c_void_p(buf.data_ptr())
     status = b.lib().pack3d_attn_bwd_noalloc(ctypes.byref(ix.struct), *([p] * 11), 0, 1, heads,
-                                             0.1, 0, p, p, p, p, None)
+                                             0, 0.1, 0, p, p, p, p, None)
     assert status == 8  # PACK3D_ERR_WORKSPACE, before any launch
     assert b.lib().pack3d_last_launch_count() == 0
     # an argument error is the one pack3d_attn_bwd reports (unsupported batch x heads here)
     status = b.lib().pack3d_attn_bwd_noalloc(ctypes.byref(ix.struct), *([p] * 11), 0, 1, 70000,
-                                             0.1, 0, p, p, p, p, None)
+                                             0, 0.1, 0, p, p, p, p, None)
     assert status == 2  # PACK3D_ERR_UNSUPPORTED
     assert b.lib().pack3d_last_launch_count() == 0
