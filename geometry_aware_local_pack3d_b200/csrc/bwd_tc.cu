@@ -56,6 +56,7 @@ struct Params {
   int64_t units, units_per_bh;  // dq: 128-query tiles
   int n_chunks;                 // dq: 64-summary chunks per (batch, head)
   int m_tiles, q_tiles, q_per_split;  // dsum: 128-summary tiles, 64-query tiles
+  int nsplit;                         // dsum: query ranges per (batch, head)
   int kv_group;                       // query heads per KV head (summaries per KV head)
   long long wait_budget;              // SM cycles of each bounded wait
 };
@@ -368,9 +369,9 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
   const int M = (int)P.ix.m;
   // work item: (batch*head, 128-summary tile, query range)
   const int64_t item = blockIdx.x;
-  const int split = (int)(item % kDsumSplit);
-  const int mt = (int)((item / kDsumSplit) % P.m_tiles);
-  const int64_t bh = item / ((int64_t)kDsumSplit * P.m_tiles);
+  const int split = (int)(item % P.nsplit);
+  const int mt = (int)((item / P.nsplit) % P.m_tiles);
+  const int64_t bh = item / ((int64_t)P.nsplit * P.m_tiles);
   const int qt0 = split * P.q_per_split;
   const int qt1 = min(P.q_tiles, qt0 + P.q_per_split);
   const int NT = max(qt1 - qt0, 0);
@@ -612,6 +613,39 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
   }
 }
 
+// Adds the per-query-range partials 1 .. nsplit-1 of the summary gradients, in range order,
+// into partial 0 (deterministic), so the un-pooling reads one.
+__global__ void __launch_bounds__(256) k_sum_splits(float* __restrict__ dks,
+                                                    float* __restrict__ dvs, int64_t elems,
+                                                    int nsplit) {
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= elems) return;
+  float sk = dks[e], sv = dvs[e];
+  for (int sp = 1; sp < nsplit; ++sp) {
+    sk += dks[sp * elems + e];
+    sv += dvs[sp * elems + e];
+  }
+  dks[e] = sk;
+  dvs[e] = sv;
+}
+
+// Query ranges per (batch, head) for the summary-gradient kernel (one CTA per SM): the count
+// in [1, kDsumSplitMax] whose CTAs fill the last wave best (fewer ranges on a tie).
+inline int dsum_splits(int64_t bh_tiles, int q_tiles, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= kDsumSplitMax && sp <= q_tiles; ++sp) {
+    const int64_t items = bh_tiles * sp;
+    const int64_t waves = (items + sms - 1) / sms;
+    const double eff = (double)items / (double)(waves * sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = sp;
+    }
+  }
+  return best;
+}
+
 // ------------------------------------------------------------------------------ host side
 template <int D>
 cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* ksum,
@@ -640,12 +674,18 @@ cudaError_t launch_bwd_tc(const pack3d_index& ix, const BwdWork& w, const void* 
   // summary gradients: (batch*head) x 128-summary tiles x query ranges
   p.m_tiles = (int)((ix.m + btc::kRows - 1) / btc::kRows);
   p.q_tiles = (int)((ix.n + btc::kChunk - 1) / btc::kChunk);
-  p.q_per_split = (p.q_tiles + kDsumSplit - 1) / kDsumSplit;
+  p.nsplit = dsum_splits(bh * p.m_tiles, p.q_tiles, sm_count());
+  p.q_per_split = (p.q_tiles + p.nsplit - 1) / p.nsplit;
   p.out0 = w.dks;
   p.out1 = w.dvs;
-  const int64_t items = bh * p.m_tiles * kDsumSplit;
+  const int64_t items = bh * p.m_tiles * p.nsplit;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   k_bwd_dsum_tc<D><<<(unsigned)items, bds::kThreads, bds::Smem<D>::kBytes, s>>>(p);
+  if (p.nsplit > 1) {
+    const int64_t elems = bh * ix.m * D;
+    k_sum_splits<<<(unsigned)((elems + 255) / 256), 256, 0, s>>>(w.dks, w.dvs, elems, p.nsplit);
+    count_launch();
+  }
   // dq~: persistent over 128-query tiles, two CTAs per SM
   p.units_per_bh = (ix.n + btc::kRows - 1) / btc::kRows;
   p.units = bh * p.units_per_bh;

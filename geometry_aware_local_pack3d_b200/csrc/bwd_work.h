@@ -9,9 +9,10 @@
 
 namespace p3d {
 
-// Query ranges the tensor-core summary-gradient kernel splits each (batch, head) into; their
-// partial sums are added, in split order, where the summary gradients are un-pooled.
-constexpr int kDsumSplit = 2;
+// Most query ranges the tensor-core summary-gradient kernel splits each (batch, head) into (the
+// launch picks the count that fills whole waves of SMs); the partial sums are added in split
+// order into the first range's slot before the summary gradients are un-pooled.
+constexpr int kDsumSplitMax = 8;
 
 struct BwdWork {
   void* qr;     // [BH, N, d]  rotated q, in the I/O type (bf16 or fp32)
@@ -20,7 +21,7 @@ struct BwdWork {
   float* Dg;    // [BH, N]     <(1 - g) dO, o_glob>
   float* dks;   // [nsplit][BH, M, d]  gradient of the key summaries (per query range)
   float* dvs;   // [nsplit][BH, M, d]  gradient of the value summaries
-  int nsplit;   // query ranges in dks / dvs (1: CUDA-core path)
+  int nsplit;   // partials the un-pooling adds (1: reduced in place, or the CUDA-core path)
   // tensor-core path only (null otherwise)
   __nv_bfloat16* qtb;   // [BH, N, d]  rotated q, bf16 (the qr array itself)
   __nv_bfloat16* dogb;  // [BH, N, d]  (1 - g) dO, bf16
@@ -39,7 +40,7 @@ inline size_t bwd_align(size_t x) { return (x + 255) & ~(size_t)255; }
 inline size_t bwd_workspace_bytes_for(const pack3d_index& ix, int64_t bh, size_t el, bool tc,
                                       int kv_group) {
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
-  const int ns = tc ? kDsumSplit : 1;
+  const int ns = tc ? kDsumSplitMax : 1;
   size_t b = 2 * bwd_align(el * rows * D) + 2 * bwd_align(sizeof(float) * rows) +
              2 * bwd_align(sizeof(float) * ns * sums * D);
   if (tc) b += bwd_align(sizeof(__nv_bfloat16) * rows * D) + bwd_align(sizeof(float) * rows * D);
@@ -52,13 +53,14 @@ inline BwdWork bwd_carve(const pack3d_index& ix, int64_t bh, void* ws, size_t el
   const size_t D = ix.geom.head_dim, rows = (size_t)bh * ix.n, sums = (size_t)bh * ix.m;
   char* p = static_cast<char*>(ws);
   BwdWork w;
-  w.nsplit = tc ? kDsumSplit : 1;
+  w.nsplit = 1;
+  const int ns = tc ? kDsumSplitMax : 1;
   w.qr = p; p += bwd_align(el * rows * D);
   w.kr = p; p += bwd_align(el * rows * D);
   w.Dl = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows);
   w.Dg = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * rows);
-  w.dks = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * w.nsplit * sums * D);
-  w.dvs = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * w.nsplit * sums * D);
+  w.dks = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * ns * sums * D);
+  w.dvs = reinterpret_cast<float*>(p); p += bwd_align(sizeof(float) * ns * sums * D);
   w.qtb = w.dogb = nullptr;
   w.dqg = nullptr;
   w.dkp = w.dvp = nullptr;

@@ -16,16 +16,16 @@
 //     map (x start rounded down to a 16-byte boundary: box 16x10x6 int32);
 //   * four producer warps fetch, per halo z-slice, the 100 key rows and value rows with one
 //     cp.async per 16-byte piece (rows off the grid or at empty sites are zero-filled) into the
-//     no-swizzle core-matrix layout, three stages deep. With rotated keys each thread's copies
+//     no-swizzle core-matrix layout, four stages deep. With rotated keys each thread's copies
 //     arrive on the stage's barrier by themselves when they land; with raw keys each thread
 //     waits for its copies of a slice (the next slice's copies already in flight), rotates its
 //     key pieces in place by the key's coordinate (known from the halo position) and then
 //     arrives;
-//   * the q tiles are double-buffered: softmax warps 0 and 1 of each tile, idle once their
-//     slices of a unit are done, load the next unit's q rows (64 rows each, one row per lane),
-//     rotate them in registers (axial RoPE by the row's coordinates) and store them into the
-//     tile's other q buffer, so the MMAs start a unit as soon as the previous one's last PV
-//     has been issued.
+//   * one q buffer per tile: softmax warps 0 and 1 of each tile, idle once their slices of a
+//     unit are done, load the next unit's q rows (64 rows each, one row per lane), rotate them
+//     in registers (axial RoPE by the row's coordinates) and store them into the tile's buffer
+//     as soon as the tile's last QK of the unit has completed, while the unit's last slices
+//     are still being worked on (a second q buffer would cost the fourth k/v stage).
 // Slice key order: halo row hy major, then halo column hx (row 10 hy + hx), so tile t's keys
 // (halo rows 4t .. 4t+5) are slice rows 40t .. 40t+59: each tile works on a 64-row window
 // starting at slice row 40 t (rows 100..103 of a stage are zero padding).
@@ -63,7 +63,7 @@ constexpr int kNK = 64;                // tile window (MMA N of QK, K of PV)
 constexpr int kNV = (TY + 2) * HX;     // 60 window columns that can hold a neighbour
 constexpr int kWin = TY * HX;          // 40: first slice row of tile 1's window
 constexpr int kRows = kWin + kNK;      // 104 rows per stage
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 // warps: softmax 0-7 (tile = warp / 4; warps 0, 1, 4, 5 also prepare q tiles), slot boxes 8
 // (warp 9 idle), k/v producers 10-13, MMA 14-15 (tile = warp - 14)
 constexpr int kThreads = 512;
@@ -94,7 +94,7 @@ template <int D> struct Smem {
   static constexpr int kChunkCol = kRows * 16 + 16;
   static constexpr int kStage = KC * kChunkCol;
   static constexpr int kQ = 0;                            // [2 buffers][2 tiles] q tiles
-  static constexpr int kK = kQ + 4 * kQBuf;               // [kStages] key chunks
+  static constexpr int kK = kQ + kTiles * kQBuf;          // [kStages] key chunks
   static constexpr int kV = kK + kStages * kStage;        // [kStages] value chunks
   static constexpr int kBox = (kV + kStages * kStage + 127) / 128 * 128;  // [2] slot boxes (TMA)
   static constexpr int kBar = kBox + 2 * kBoxPitch;
@@ -106,7 +106,7 @@ template <int D> struct Smem {
 };
 
 enum {
-  B_QFULL = 0, B_QEMPTY = 4,  // [q buffer][tile]
+  B_QFULL = 0, B_QEMPTY = 4,  // [tile] (slots 2, 3 and 6, 7 unused)
   B_KVFULL = 8, B_KVEMPTY = 12, B_BOX = 16, B_BOXFREE = 18,
   B_SFULL = 20,  // [tile][warp][buffer]
   B_PFULL = 36,  // [tile][warp][buffer]
@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     // coordinates (axial RoPE) and stored in the operand layout -- then publishes its share
     // (QFULL: 64 arrivals per tile). Row r of a tile holds brick position
     // (r / 32, 4 tile + (r / 8) % 4, r % 8); rows off the grid or at empty sites are zero.
-    auto prepare_q = [&](int64_t un, int nb, int qi) {
+    auto prepare_q = [&](int64_t un, int nb, int qi, int tix) {
+      if (lane == 0 && tile == 0) GTR(tix, 200 + w * 2);
       int64_t qbh;
       int qz0, qy0, qx0;
       origin(un, qbh, qz0, qy0, qx0);
@@ -321,6 +322,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars[B_QFULL + qi]);
+      if (lane == 0 && tile == 0) GTR(tix, 201 + w * 2);
     };
     int ti = 0;
     bool ok = true;
@@ -335,29 +337,37 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + bb], (ti >> 1) & 1))) break;
       const int64_t u = unit_of(bb);
       if (u < 0) break;
-      if (ti == 0 && w < 2) prepare_q(u, 0, tile);  // the first unit's q tile
+      if (ti == 0 && w < 2) prepare_q(u, 0, tile, 0);  // the first unit's q tile
       int64_t bh;
       int z0, y0, x0;
       origin(u, bh, z0, y0, x0);
       const int32_t* box = reinterpret_cast<const int32_t*>(smem + S::kBox + bb * kBoxPitch);
       const int cz = z0 + w, cy = y0 + qy, cx = x0 + qx;
       const bool valid = cz < g.gz && cy < g.gy && cx < g.gx;
-      // neighbour bits of the warp's three slices: bit slice_row(hy, hx) - 40 tile of slice
-      // w + i, i = 1 + dz (empty sites, with slot -1, are no neighbours)
-      uint64_t nb[3] = {0ull, 0ull, 0ull};
-      if (valid) {
+      // neighbour bits of the warp's three slices w + i (i = 1 + dz): bit c of the tile's
+      // window holds slice row 40 tile + c. The window's occupied keys (inside the grid, not an
+      // empty site) are one mask per slice, two window keys per lane and a ballot each; a row's
+      // 3x3 neighbours are the pattern 0b111 in three window rows, shifted to its position.
+      uint64_t nb[3];
 #pragma unroll
-        for (int o = 0; o < 27; ++o) {
-          const int ddz = o / 9 - 1, ddy = (o / 3) % 3 - 1, ddx = o % 3 - 1;
-          const int hy = qy + 1 + ddy, hx = qx + 1 + ddx;
-          const int hz = w + 1 + ddz;  // halo slice
-          if (!in_grid(cz + ddz, cy + ddy, cx + ddx)) continue;
-          if (box[(hz * kBoxY + hy) * kBoxX + hx + 3] < 0) continue;
-          const uint64_t bit = 1ull << (slice_row(hy, hx) - kWin * tile);
-          nb[0] |= ddz == -1 ? bit : 0ull;
-          nb[1] |= ddz == 0 ? bit : 0ull;
-          nb[2] |= ddz == 1 ? bit : 0ull;
+      for (int i = 0; i < 3; ++i) {
+        const int hz = w + i;  // halo slice
+        uint32_t half[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int c = hh * 32 + ln;  // window column
+          bool occ = false;
+          if (c < kNV) {
+            const int hy = TY * tile + c / HX, hx = c % HX;
+            occ = in_grid(z0 - 1 + hz, y0 - 1 + hy, x0 - 1 + hx) &&
+                  box[(hz * kBoxY + hy) * kBoxX + hx + 3] >= 0;
+          }
+          half[hh] = __ballot_sync(0xffffffffu, occ);
         }
+        const uint64_t occm = (uint64_t)half[0] | ((uint64_t)half[1] << 32);
+        const uint64_t row3 = 7ull << qx;  // halo x = qx .. qx + 2
+        const uint64_t pat = (row3 | (row3 << HX) | (row3 << (2 * HX))) << (HX * (qy - TY * tile));
+        nb[i] = valid ? (pat & occm) : 0ull;
       }
       // this warp's O rows start at zero (the previous unit's epilogue has read them)
       {
@@ -365,6 +375,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 16) tc::tmem_st16(tl + kOCol + c0, zr);
       }
+      if (ln == 0 && tile == 0) GTR(ti, 220 + w);  // preamble done
       uint64_t* sfull = &bars[B_SFULL + (tile * 4 + w) * 2];
       uint64_t* pfull = &bars[B_PFULL + (tile * 4 + w) * 2];
       float m_run = -INFINITY, l_run = 0.f;
@@ -476,16 +487,14 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           P.lse_loc[bh * N + slot] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
       if (w < 2) {
-        // the next unit's q tile, into the other q buffer once its slot box is in and the
-        // buffer's previous unit (ti - 1) has finished its QK MMAs
-        const int nb = (ti + 1) & 1, qi = nb * 2 + tile;
+        // the next unit's q tile, into the tile's q buffer once its slot box is in and this
+        // unit's last QK of the tile has completed
+        const int nb = (ti + 1) & 1;
         if (!__all_sync(0xffffffffu, ab.wait(&bars[B_BOX + nb], ((ti + 1) >> 1) & 1))) break;
         const int64_t un = unit_of(nb);
         if (un >= 0) {
-          if (ti >= 1 &&
-              !__all_sync(0xffffffffu, ab.wait(&bars[B_QEMPTY + qi], ((ti - 1) >> 1) & 1)))
-            break;
-          prepare_q(un, nb, qi);
+          if (!__all_sync(0xffffffffu, ab.wait(&bars[B_QEMPTY + tile], ti & 1))) break;
+          prepare_q(un, nb, tile, ti + 1);
         }
       }
     }
@@ -727,9 +736,9 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
     };
     for (; ok; ++ti) {
       if (!wwait(&bars[B_BOX + (ti & 1)], (ti >> 1) & 1) || unit_of(ti & 1) < 0) break;
-      const int qi = (ti & 1) * 2 + tile;
+      const int qi = tile;  // one q buffer per tile
       const uint64_t qd = qd0 + (uint64_t)((qi * S::kQBuf) >> 4);
-      if (!wwait(&bars[B_QFULL + qi], (ti >> 1) & 1)) break;
+      if (!wwait(&bars[B_QFULL + qi], ti & 1)) break;
       if (lane == 0 && tile == 0) GTR(ti, 50);
       if (lane == 0 && tile == 0) BRICK_T(ti);
       tc::tc_fence_after();

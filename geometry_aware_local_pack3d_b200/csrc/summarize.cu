@@ -28,7 +28,7 @@
 namespace p3d {
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __restrict__ k,
+__global__ void __launch_bounds__(128, 6) k_summarize(pack3d_index ix, const T* __restrict__ k,
                                                    const T* __restrict__ v, int64_t bh_count,
                                                    T* __restrict__ ksum, T* __restrict__ vsum,
                                                    T* __restrict__ krot) {
@@ -62,9 +62,10 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
     // itself, so no table lookup stands before the member loads
     const int blk = m < M ? (gv == 1 ? m : ix.groups[(int64_t)m * gv + t]) : -1;
     if (blk < 0) continue;
-    float bk[E], bv[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) bk[e] = bv[e] = 0.f;
+    // each member present carries 1 / (members present in the block): the sum over the
+    // block's members is then its mean (the count's load overlaps the member loads)
+    const int cnt = ix.count[blk];
+    const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.f;
     // Members are taken 32 at a time: lane l fetches the slot and coordinate of member b0 + l
     // once, and every lane then reads them by shuffle, so the 16-byte k/v loads of many
     // members are independent and in flight together (the loop body has no branch).
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
         const int32_t cc = __shfl_sync(0xffffffffu, cl, sl & 31);
         const bool use = active && sl < 32 && b0 + sl < vol && j >= 0;
         const int64_t row = use ? j : 0;
-        const float wgt = use ? 1.f : 0.f;
+        const float wgt = use ? inv : 0.f;
         const int cv = coord_axis(decode(cc), axis);
         float xk[E], xv[E], rk[E];
         Vec<T>::load(kb + row * D + c * E, xk);
@@ -93,20 +94,13 @@ __global__ void __launch_bounds__(128) k_summarize(pack3d_index ix, const T* __r
               rope_cs(ix.rope, ix.rope_rows, ix.rope_pairs, axis, use ? cv : 0, p0 + e / 2);
           rk[e] = xk[e] * cs.x - xk[e + 1] * cs.y;
           rk[e + 1] = xk[e] * cs.y + xk[e + 1] * cs.x;
-          bk[e] += wgt * (centre ? xk[e] : rk[e]);
-          bk[e + 1] += wgt * (centre ? xk[e + 1] : rk[e + 1]);
-          bv[e] += wgt * xv[e];
-          bv[e + 1] += wgt * xv[e + 1];
+          ak[e] = fmaf(wgt, centre ? xk[e] : rk[e], ak[e]);
+          ak[e + 1] = fmaf(wgt, centre ? xk[e + 1] : rk[e + 1], ak[e + 1]);
+          av[e] = fmaf(wgt, xv[e], av[e]);
+          av[e + 1] = fmaf(wgt, xv[e + 1], av[e + 1]);
         }
         if (krot && use) Vec<T>::store(krot + bh * ix.n * D + row * D + c * E, rk);
       }
-    }
-    const int cnt = ix.count[blk];  // an empty block added zeros: its weight is 0
-    const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.f;  // this lane's share of the block mean
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      ak[e] = fmaf(bk[e], inv, ak[e]);
-      av[e] = fmaf(bv[e], inv, av[e]);
     }
   }
   // combine the R partial sums in the fixed order r = 0, 1, ..., R-1 (each lane's own
