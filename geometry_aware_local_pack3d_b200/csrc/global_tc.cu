@@ -47,13 +47,6 @@ constexpr int kProd = 128;        // query producer threads
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kRopeSmemBytes = 24576;  // [3 axes][64 coordinates][16 pairs] (cos, sin)
-#ifndef P3D_POLY_EVERY
-#define P3D_POLY_EVERY 0
-#endif
-// softmax exponentials: one column pair in kPolyEvery computed on the FMA pipe (0: none). On
-// B200 the kernel measured 0.600 / 0.605 / 0.610 / 0.624 ms with none / 1 in 8 / 1 in 4 /
-// 1 in 2 at the 65,536-token field, so the MUFU pipe is not what bounds it: off by default.
-constexpr int kPolyEvery = P3D_POLY_EVERY;
 
 // TMEM columns: tile t uses [256 t, 256 t + 256): S buffers at +0 and +64, O at +128.
 __host__ __device__ constexpr uint32_t s_col(int t, int b) { return 256u * t + 64u * b; }
@@ -192,6 +185,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         }
         if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2);
         if (rin == 0 && pc == 1 && j < 10) P3D_TRACE_C(3400 + j * 4 + t * 2);
+        if (lane == 0 && pc == 1 && j < 16) P3D_TRACE(3730 + j * 8 + warp);
         tc::tc_fence_after();
         const int m0 = j * kChunk;
         const int ncol = min(kChunk, M - m0);
@@ -277,11 +271,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
           for (int k = 0; k < 32; k += 2) {
             const float2 x = tc::fma2(
                 make_float2(__uint_as_float(r[c0 + k]), __uint_as_float(r[c0 + k + 1])), sl2, nm2);
-            // one pair in kPolyEvery on the FMA pipe: the MUFU pipe bounds this loop otherwise
-            const float2 e = (kPolyEvery > 0 && (k >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1) ==
-                                                    kPolyEvery - 1)
-                                 ? tc::exp2_poly2(x)
-                                 : make_float2(ex2(x.x), ex2(x.y));
+            const float2 e = make_float2(ex2(x.x), ex2(x.y));
             ls[(k >> 1) & 3] = tc::add2(ls[(k >> 1) & 3], e);
             p[k >> 1] = tc::pack_bf16(e.x, e.y);
           }
@@ -294,6 +284,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         tc::tc_fence_before();
         tc::mbar_arrive(&bars[B_PFULL + 2 * t + b]);
         if (rin == 0 && pc < 3) P3D_TRACE(1000 + pc * 128 + t * 64 + j * 2 + 1);
+        if (lane == 0 && pc == 1 && j < 16) P3D_TRACE(3600 + j * 8 + warp);
         if (rin == 0 && pc == 1 && j < 10) P3D_TRACE_C(3400 + j * 4 + t * 2 + 1);
       }
       if (!ok) break;

@@ -93,7 +93,7 @@ template <int D> struct Smem {
   static constexpr int kQBuf = KC * kQCol;         // one q tile
   static constexpr int kChunkCol = kRows * 16 + 16;
   static constexpr int kStage = KC * kChunkCol;
-  static constexpr int kQ = 0;                            // [2 buffers][2 tiles] q tiles
+  static constexpr int kQ = 0;                            // [2 tiles] q tiles, one buffer each
   static constexpr int kK = kQ + kTiles * kQBuf;          // [kStages] key chunks
   static constexpr int kV = kK + kStages * kStage;        // [kStages] value chunks
   static constexpr int kBox = (kV + kStages * kStage + 127) / 128 * 128;  // [2] slot boxes (TMA)
@@ -130,7 +130,27 @@ struct Params {
   int64_t units;      // batch * heads * units per field
   int kv_group;       // query heads per KV head: k_rot and v rows of KV head bh / kv_group
   long long wait_budget;  // SM cycles of each bounded wait
+  // RoPE angle per unit coordinate of rotation pair p on axis a: spacing_a * base^(-2p / d_a)
+  float theta[3][16];
 };
+
+// (cos, sin) of the RoPE angle c * theta of integer coordinate c, computed in registers (the
+// q preparation would otherwise load the rotation table from global memory, two 16-byte loads
+// per 16-byte piece, on the path between units). The product is reduced to [-pi, pi] by the
+// two-constant Cody-Waite method (2 pi = kTwoPiHi + kTwoPiLo, kTwoPiHi the float nearest to
+// 2 pi) and the reduced angle goes to the fast sine and cosine. Absolute error about
+// 1e-7 * |c * theta| + 1e-6 against the float64 angle: far below the bf16 rounding of q~.
+__device__ __forceinline__ float2 rope_angle_cs(int c, float theta) {
+  constexpr float kInv2Pi = 0.159154943091895336f;
+  constexpr float kTwoPiHi = 6.28318548202514648f;
+  constexpr float kTwoPiLo = -1.74845560007448e-07f;
+  const float a = (float)c * theta;
+  const float n = rintf(a * kInv2Pi);
+  const float r = fmaf(-n, kTwoPiLo, fmaf(-n, kTwoPiHi, a));
+  float sn, cn;
+  __sincosf(r, &sn, &cn);
+  return make_float2(cn, sn);
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -284,7 +304,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       origin(un, qbh, qz0, qy0, qx0);
       const int32_t* qbox = reinterpret_cast<const int32_t*>(smem + S::kBox + nb * kBoxPitch);
       uint8_t* qd = smem + S::kQ + qi * S::kQBuf;
-      const int pairs = P.ix.rope_pairs, rmax = P.ix.rope_rows - 1;
+      const int rmax = P.ix.rope_rows - 1;
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
         const int r = 64 * w + 32 * pass + lane;
@@ -302,11 +322,14 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         for (int c = 0; c < KC; ++c) {
           const int axis = (c * 8) / DA, p0 = ((c * 8) % DA) / 2;
           const int cv = axis == 0 ? cz : (axis == 1 ? cy : cx);
-          // (cos, sin) of the piece's 4 rotation pairs: 32 contiguous bytes of the table
-          const float4* cs4 = reinterpret_cast<const float4*>(
-              P.ix.rope + 2 * rope_slot(P.ix.rope_rows, pairs, axis, cv, p0));
-          const float4 ca = __ldg(cs4), cbv = __ldg(cs4 + 1);
-          const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cbv.x, cbv.y, cbv.z, cbv.w};
+          // (cos, sin) of the piece's 4 rotation pairs
+          float cs[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 e = rope_angle_cs(cv, P.theta[axis][p0 + k]);
+            cs[2 * k] = e.x;
+            cs[2 * k + 1] = e.y;
+          }
           const uint32_t xin[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
           uint32_t xo[4];
 #pragma unroll
@@ -815,6 +838,12 @@ cudaError_t launch_local_tma(const pack3d_index& ix, const void* q, const void* 
   p.scale_log2 = scale * kLog2e;
   p.wait_budget = wait_budget_cycles();
   p.kv_group = kv_group;
+  for (int a = 0; a < 3; ++a)
+    for (int pp = 0; pp < 16; ++pp)
+      p.theta[a][pp] = pp < ix.rope_pairs
+                           ? (float)((double)ix.geom.spacing[a] *
+                                     pow((double)ix.geom.rope_base, -2.0 * pp / (2.0 * ix.rope_pairs)))
+                           : 0.f;
   p.nbz = (ix.geom.gz + BZ - 1) / BZ;
   p.nby = (ix.geom.gy + BY - 1) / BY;
   p.nbx = (ix.geom.gx + BX - 1) / BX;

@@ -88,10 +88,22 @@ __global__ void __launch_bounds__(128, 6) k_summarize(pack3d_index ix, const T* 
         float xk[E], xv[E], rk[E];
         Vec<T>::load(kb + row * D + c * E, xk);
         Vec<T>::load(vb + row * D + c * E, xv);
+        // (cos, sin) of the piece's E / 2 rotation pairs: E * 4 contiguous bytes of the table
+        // (p0 is a multiple of E / 2, so the 16-byte loads are aligned)
+        float2 csv[E / 2];
+        {
+          const float4* cs4 = reinterpret_cast<const float4*>(
+              ix.rope + 2 * rope_slot(ix.rope_rows, ix.rope_pairs, axis, use ? cv : 0, p0));
+#pragma unroll
+          for (int h = 0; h < E / 4; ++h) {
+            const float4 t4 = __ldg(cs4 + h);
+            csv[2 * h] = make_float2(t4.x, t4.y);
+            csv[2 * h + 1] = make_float2(t4.z, t4.w);
+          }
+        }
 #pragma unroll
         for (int e = 0; e < E; e += 2) {
-          const float2 cs =
-              rope_cs(ix.rope, ix.rope_rows, ix.rope_pairs, axis, use ? cv : 0, p0 + e / 2);
+          const float2 cs = csv[e / 2];
           rk[e] = xk[e] * cs.x - xk[e + 1] * cs.y;
           rk[e + 1] = xk[e] * cs.y + xk[e + 1] * cs.x;
           ak[e] = fmaf(wgt, centre ? xk[e] : rk[e], ak[e]);
