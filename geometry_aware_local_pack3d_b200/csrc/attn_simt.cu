@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(pack3d_index ix, const T* __re
 
 // dq = R(c)^T (sum_j dS_ij k~_j + global part); kGL lanes per query row.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __restrict__ v,
+__global__ void __launch_bounds__(128, 4) k_bwd_dq(pack3d_index ix, const T* __restrict__ v,
                                                 const T* __restrict__ ksum,
                                                 const T* __restrict__ vsum,
                                                 const T* __restrict__ gate,
@@ -544,7 +544,7 @@ __global__ void __launch_bounds__(128) k_bwd_dq(pack3d_index ix, const T* __rest
 // summary's rotation R(centre)^T and is added after the local part's inverse rotation. With
 // GQA each query head's dk, dv go to float32 partials that k_bwd_gqa_reduce sums.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) k_bwd_dkv(pack3d_index ix, const T* __restrict__ v,
+__global__ void __launch_bounds__(128, 4) k_bwd_dkv(pack3d_index ix, const T* __restrict__ v,
                                                  const T* __restrict__ gate,
                                                  const T* __restrict__ dO,
                                                  const float* __restrict__ lse_loc, float scale,
