@@ -654,6 +654,10 @@ size_t bwd_workspace_bytes(const pack3d_index& ix, int64_t bh, int dtype, bool t
 cudaError_t bwd_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* ksum,
                             const void* vsum, const float* lse_glob, int64_t bh, int kv_group,
                             float scale, int excl, cudaStream_t s);
+cudaError_t bwd_local_dq_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* v,
+                                     const void* dO, const void* gate, const float* lse_loc,
+                                     int64_t bh, int kv_group, float scale, void* dq,
+                                     cudaStream_t s);
 
 template <typename T, int D>
 cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
@@ -686,12 +690,20 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
     count_launch();
   }
   const unsigned gb = (unsigned)((rows + 128 / kGL - 1) / (128 / kGL));  // kGL lanes per row
-  k_bwd_dq<T, D><<<gb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
-                                     static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
-                                     scale, excl, rows, kv_group, w, static_cast<T*>(dq));
+  if (tc) {
+    // bf16: the local branch's part of dq~ on tensor cores, plus the global part, R(c)^T -> dq
+    const cudaError_t e =
+        bwd_local_dq_tc_dispatch(ix, w, v, dO, gate, lse_loc, bh, kv_group, scale, dq, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    k_bwd_dq<T, D><<<gb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
+                                       static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
+                                       scale, excl, rows, kv_group, w, static_cast<T*>(dq));
+    count_launch();
+  }
   k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, kv_group, w,
                                       static_cast<T*>(dk), static_cast<T*>(dv));
-  count_launch(2);
+  count_launch();
   if (kv_group > 1) {
     const int64_t kv_elems = rows / kv_group * D;
     k_bwd_gqa_reduce<T><<<(unsigned)((kv_elems + 255) / 256), 256, 0, s>>>(
