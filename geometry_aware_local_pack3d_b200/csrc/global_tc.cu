@@ -7,7 +7,8 @@
 //
 // Work unit: 256 consecutive memory rows of one (batch, head) = two 128-row query tiles that
 // share every summary chunk (halves the L2 reads of the summaries). Persistent CTAs walk the
-// units round-robin. Warp roles (480 threads):
+// units round-robin. Warp roles (with PW = 4 query-producer warps, 480 threads; PW = 2 when a
+// unit has 32 or more summary chunks, 416 threads, the later roles moving down by two):
 //   warps 0-3   softmax + epilogue of tile 0 (thread = row, TMEM lanes 0..127); the epilogue
 //               normalises O, writes lse, and parks o_glob in the tile's (by then consumed)
 //               q area
@@ -42,8 +43,15 @@ constexpr int kRows = 128;        // rows per tile
 constexpr int kTiles = 2;         // tiles per unit
 constexpr int kChunk = 64;        // summaries per chunk
 constexpr int kStages = 4;        // summary ring depth
-constexpr int kThreads = 480;
-constexpr int kProd = 128;        // query producer threads
+// Warp roles for PW query-producer warps (4, or 2 when a unit has many summary chunks: the
+// producers' per-unit work -- the mixer of one unit and the q tiles of the next -- is then
+// spread over a long unit, and fewer producer warps leave the softmax warps more of the SM)
+template <int PW> struct Roles {
+  static constexpr int kProd = 32 * PW;  // query producer threads
+  static constexpr int W_PROD = 8, W_MMA = W_PROD + PW, W_LOAD = W_MMA + kTiles;
+  static constexpr int kThreads = 32 * (W_LOAD + 1);
+};
+constexpr int kManyChunks = 32;  // 2 producer warps from this many 64-summary chunks up
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kRopeSmemBytes = 24576;  // [3 axes][64 coordinates][16 pairs] (cos, sin)
@@ -108,11 +116,13 @@ __device__ __forceinline__ float ex2(float x) {
 
 }  // namespace gtc
 
-template <int D>
-__global__ void __launch_bounds__(gtc::kThreads, 1)
+template <int D, int PW>
+__global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
     k_global_tc(const gtc::Params P) {
   using namespace gtc;
   using S = Smem<D>;
+  constexpr int kProd = Roles<PW>::kProd;
+  constexpr int W_PROD = Roles<PW>::W_PROD, W_MMA = Roles<PW>::W_MMA, W_LOAD = Roles<PW>::W_LOAD;
   constexpr int KC = D / 8;  // 16-byte chunks per row
   constexpr int CB = kChunk * 16;  // byte stride between 16-byte columns of a summary chunk
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     float* dst = reinterpret_cast<float*>(smem + S::kRope);
     for (int i = tid; i < n; i += blockDim.x) dst[i] = P.ix.rope[i];
   }
-  if (warp == 12) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == W_MMA) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -324,11 +334,11 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         P.lse_glob[bh * N + row] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       tc::mbar_arrive(&bars[B_QEMPTY + (pc & 1)]);  // o_glob of this unit is staged
     }
-  } else if (warp < 12) {
+  } else if (warp < W_MMA) {
     // ------------------------------------------------------------------ query producer
     // cp.async the unit's 256 q rows straight into the operand layout (every copy in flight at
     // once), then rotate each 16-byte piece in place with the row's coordinate.
-    const int ptid = tid - 256;
+    const int ptid = tid - 32 * W_PROD;
     constexpr int DA = D / 3;
     int32_t* coord_s = reinterpret_cast<int32_t*>(smem + S::kCoord);
     const float* rope = P.rope_in_smem ? reinterpret_cast<const float*>(smem + S::kRope) : P.ix.rope;
@@ -385,7 +395,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     // one thread waits for unit k's staging; the named barrier hands its verdict to all
     auto wait_staged = [&](int k) -> bool {
       if (ptid == 0) *prod_ok = ab.wait(&bars[B_QEMPTY + (k & 1)], (k >> 1) & 1) ? 1 : 0;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kProd) : "memory");
       return *prod_ok != 0;
     };
     int pc = 0;
@@ -396,7 +406,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         // q buffer b still holds unit pc-2's staged o_glob: mix it, then refill the buffer
         if (!wait_staged(pc - 2)) { pok = false; break; }
         mix(pc - 2);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kProd) : "memory");
       }
       if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4);
       const int64_t bh = u / P.units_per_bh;
@@ -415,7 +425,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       tc::cp_async_commit();
       for (int r = ptid; r < kRows * kTiles; r += kProd)
         coord_s[r] = row0 + r < N ? P.ix.coord[row0 + r] : 0;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(kProd) : "memory");
       tc::cp_async_wait_all();
       if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4 + 1);
 #pragma unroll 4
@@ -445,7 +455,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
         *ptr = make_uint4(xo[0], xo[1], xo[2], xo[3]);
       }
       tc::fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // coord_s is rewritten next unit
+      asm volatile("bar.sync 1, %0;" ::"n"(kProd) : "memory");  // coord_s is rewritten next unit
       tc::mbar_arrive(&bars[B_QFULL + b]);
       if (ptid == 0 && pc < 3) P3D_TRACE(2700 + pc * 4 + 2);
     }
@@ -454,7 +464,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
       if (!wait_staged(k)) break;
       mix(k);
     }
-  } else if (warp < 12 + kTiles) {
+  } else if (warp < W_LOAD) {
     // ------------------------------------------------------------------ MMA issuers
     // One warp per query tile (warp 12: tile 0, warp 13: tile 1), so each tile's chain
     // softmax(j) -> PV(j) -> QK(j+2) advances on its own and neither waits behind the other's
@@ -465,7 +475,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
     // start address is the low 14 bits and every offset keeps it in range); one elected lane
     // issues the MMAs and commits. A summary stage is released once both tiles' PVs of the
     // chunk have completed (KVEMPTY expects one commit from each issuer).
-    const int t = warp - 12;
+    const int t = warp - W_MMA;
     const uint32_t tb = __shfl_sync(0xffffffffu, tbase, 0);
     const uint32_t id_qk = tc::idesc_bf16_f32(128, kChunk, false, false);
     const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
@@ -583,7 +593,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == W_MMA) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, kTmemCols);
   }
@@ -591,14 +601,14 @@ __global__ void __launch_bounds__(gtc::kThreads, 1)
 
 // ------------------------------------------------------------------------------ host side
 
-template <int D>
+template <int D, int PW>
 cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* gate,
                              const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
                              int kv_group, float scale, int excl, void* o, float* lse_glob,
                              void* o_glob, cudaStream_t s) {
   using namespace gtc;
   static std::atomic<uint64_t> attr_done{0};
-  if (smem_attr_once(reinterpret_cast<const void*>(k_global_tc<D>), Smem<D>::kBytes, attr_done) !=
+  if (smem_attr_once(reinterpret_cast<const void*>(k_global_tc<D, PW>), Smem<D>::kBytes, attr_done) !=
       cudaSuccess)
     return cudaErrorInvalidValue;
   Params p;
@@ -621,7 +631,7 @@ cudaError_t launch_global_tc(const pack3d_index& ix, const void* q, const void* 
   p.kv_group = kv_group;
   p.has_empty = ix.n_empty > 0 ? 1 : 0;
   const int grid = (int)(p.units < sm_count() ? p.units : sm_count());
-  k_global_tc<D><<<grid, kThreads, Smem<D>::kBytes, s>>>(p);
+  k_global_tc<D, PW><<<grid, Roles<PW>::kThreads, Smem<D>::kBytes, s>>>(p);
   count_launch();
   return cudaGetLastError();
 }
@@ -630,11 +640,13 @@ cudaError_t global_tc_dispatch(const pack3d_index& ix, const void* q, const void
                                const void* ksum, const void* vsum, const void* o_loc, int64_t bh,
                                int kv_group, float scale, int excl, void* o, float* lse_glob,
                                void* o_glob, cudaStream_t s) {
-  if (ix.geom.head_dim == 96)
-    return launch_global_tc<96>(ix, q, gate, ksum, vsum, o_loc, bh, kv_group, scale, excl, o,
-                                lse_glob, o_glob, s);
-  return launch_global_tc<48>(ix, q, gate, ksum, vsum, o_loc, bh, kv_group, scale, excl, o,
-                              lse_glob, o_glob, s);
+  const bool many = (ix.m + gtc::kChunk - 1) / gtc::kChunk >= gtc::kManyChunks;
+#define P3D_GTC(D, PW)                                                                      \
+  launch_global_tc<D, PW>(ix, q, gate, ksum, vsum, o_loc, bh, kv_group, scale, excl, o, \
+                          lse_glob, o_glob, s)
+  if (ix.geom.head_dim == 96) return many ? P3D_GTC(96, 2) : P3D_GTC(96, 4);
+  return many ? P3D_GTC(48, 2) : P3D_GTC(48, 4);
+#undef P3D_GTC
 }
 
 }  // namespace p3d
