@@ -563,10 +563,11 @@ def main():
                                           "achieved": bflops / (bms / 1e3) / 1e12,
                                           "peak": peaks["bf16"], "unit": "TFLOP/s",
                                           "frac": bflops / (bms / 1e3) / 1e12 / peaks["bf16"]},
-                             "path": "global branch and the local branch's dq on tensor "
-                                     "cores (k_bwd_dsum_tc, k_bwd_dq_tc, k_bwd_local_dq_tc); row "
-                                     "prologue, the local branch's dk, dv, un-pooling and "
-                                     "inverse RoPE of dk on CUDA cores (k_bwd_prep, k_bwd_dkv)"}
+                             "path": "tensor cores: global branch (k_bwd_dsum_tc, "
+                                     "k_bwd_dq_tc) and local branch (k_bwd_local_dq_tc, "
+                                     "k_bwd_local_dkv_tc, with the un-pooling and inverse RoPE "
+                                     "in their epilogues); the row prologue on CUDA cores "
+                                     "(k_bwd_prep)"}
         extra["fwd_bwd"] = {"workload": "field65k_fwdbwd_bf16 (the headline field, forward "
                                         "saving o_loc, o_glob and both lse, then the backward)",
                             "ms": fms + bms, "fwd_ms": fms, "bwd_ms": bms,

@@ -658,6 +658,10 @@ cudaError_t bwd_local_dq_tc_dispatch(const pack3d_index& ix, const BwdWork& w, c
                                      const void* dO, const void* gate, const float* lse_loc,
                                      int64_t bh, int kv_group, float scale, void* dq,
                                      cudaStream_t s);
+cudaError_t bwd_local_dkv_tc_dispatch(const pack3d_index& ix, const BwdWork& w, const void* v,
+                                      const void* dO, const void* gate, const float* lse_loc,
+                                      int64_t bh, int kv_group, float scale, void* dk, void* dv,
+                                      cudaStream_t s);
 
 template <typename T, int D>
 cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const void* v,
@@ -691,19 +695,21 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
   }
   const unsigned gb = (unsigned)((rows + 128 / kGL - 1) / (128 / kGL));  // kGL lanes per row
   if (tc) {
-    // bf16: the local branch's part of dq~ on tensor cores, plus the global part, R(c)^T -> dq
-    const cudaError_t e =
+    // bf16: the local branch on tensor cores -- dq~ plus the global part, R(c)^T -> dq; dk~, dv
+    // plus the un-pooled summary gradients, R(c)^T -> dk
+    cudaError_t e =
         bwd_local_dq_tc_dispatch(ix, w, v, dO, gate, lse_loc, bh, kv_group, scale, dq, s);
+    if (e != cudaSuccess) return e;
+    e = bwd_local_dkv_tc_dispatch(ix, w, v, dO, gate, lse_loc, bh, kv_group, scale, dk, dv, s);
     if (e != cudaSuccess) return e;
   } else {
     k_bwd_dq<T, D><<<gb, 128, 0, s>>>(ix, tv, static_cast<const T*>(ksum),
                                        static_cast<const T*>(vsum), tg, tdo, lse_loc, lse_glob,
                                        scale, excl, rows, kv_group, w, static_cast<T*>(dq));
-    count_launch();
+    k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, kv_group, w,
+                                        static_cast<T*>(dk), static_cast<T*>(dv));
+    count_launch(2);
   }
-  k_bwd_dkv<T, D><<<gb, 128, 0, s>>>(ix, tv, tg, tdo, lse_loc, scale, rows, kv_group, w,
-                                      static_cast<T*>(dk), static_cast<T*>(dv));
-  count_launch();
   if (kv_group > 1) {
     const int64_t kv_elems = rows / kv_group * D;
     k_bwd_gqa_reduce<T><<<(unsigned)((kv_elems + 255) / 256), 256, 0, s>>>(
