@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(lk::kThreads, 1)
       }
       uint64_t* sfull = &bars[B_SFULL + w * 2];
       uint64_t* pfull = &bars[B_PFULL + w * 2];
-#pragma unroll
+#pragma unroll 1
       for (int i = 0; i < 3; ++i) {
         const int s = w + i, b = s & 1;
         const int st = (int)(((uint32_t)ti * kChunks + s) % kStages);
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(lk::kThreads, 1)
         }
         tc::tc_fence_after();
         const float* cv = reinterpret_cast<const float*>(smem + S::kCol) + st * 3 * 64;
-        const uint64_t win = nb[i];
+        const uint64_t win = i == 0 ? nb[0] : (i == 1 ? nb[1] : nb[2]);  // (no indexed array)
         // two halves of 32 query columns: P^T g packed over S^T and dS^T over dP^T, columns
         // 16 h .. 16 h + 15 (columns the first half has already read)
 #pragma unroll
@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(lk::kThreads, 1)
         const float* sk0 = P.dks + (bh * P.ix.m + t) * D;
         const float* sv0 = P.dvs + (bh * P.ix.m + t) * D;
         const float2* rc = reinterpret_cast<const float2*>(P.ix.rope_c) + (int64_t)t * (D / 2);
-#pragma unroll
+        // (once per unit: kept rolled, the kernel's code is large)
+#pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
           uint32_t ok16[16], ov16[16];
           tc::tmem_ld16(tl + kDkCol + c0, ok16);
