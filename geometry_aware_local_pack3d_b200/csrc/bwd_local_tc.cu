@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
       uint64_t* sfull = &bars[B_SFULL + tile * 4 + w];
       uint64_t* pfull = &bars[B_PFULL + tile * 4 + w];
-#pragma unroll
+#pragma unroll 1  // (rolled: the kernel's code is large; instruction fetch stalls otherwise)
       for (int i = 0; i < 3; ++i) {
         // S and dP of slice w + i (this warp's phase 3 ti + i)
         if (!__all_sync(0xffffffffu, ab.wait(sfull, (uint32_t)(3 * ti + i) & 1))) {
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
           break;
         }
         tc::tc_fence_after();
-        const uint64_t win = nb[i];
+        const uint64_t win = i == 0 ? nb[0] : (i == 1 ? nb[1] : nb[2]);  // (no indexed array)
         // two halves of 32 window columns: dS of half h packed over S columns 16 h .. 16 h + 15
         // (columns the first half has already read)
 #pragma unroll

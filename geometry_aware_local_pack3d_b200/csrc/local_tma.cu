@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
       uint64_t* sfull = &bars[B_SFULL + (tile * 4 + w) * 2];
       uint64_t* pfull = &bars[B_PFULL + (tile * 4 + w) * 2];
       float m_run = -INFINITY, l_run = 0.f;
-#pragma unroll
+#pragma unroll 1  // (rolled: the kernel's code is large; instruction fetch stalls otherwise)
       for (int i = 0; i < 3; ++i) {
         const int s = w + i, b = s & 1;
         const uint32_t gs = (uint32_t)ti * kChunks + s;
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
         lg::tmem_ld8(tl + s_col(b) + 48, &r[48]);
         lg::tmem_ld4(tl + s_col(b) + 56, &r[56]);
         tc::tmem_wait_ld();
-        const uint64_t win = nb[i];
+        const uint64_t win = i == 0 ? nb[0] : (i == 1 ? nb[1] : nb[2]);  // (no indexed array)
 #pragma unroll
         for (int k = 0; k < kNV; k += 2) {
           if (!((win >> k) & 1ull)) r[k] = 0xff800000u;
