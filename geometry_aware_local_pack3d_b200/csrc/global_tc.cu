@@ -402,6 +402,17 @@ __global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
     bool pok = true;
     for (int64_t u = blockIdx.x; u < P.units; u += gridDim.x, ++pc) {
       const int b = pc & 1;
+      if (ptid == 0) {
+        // this unit's o_loc rows (one contiguous run) and gates, read by its mixer two units
+        // from now: start bringing them into L2
+        const int64_t bhu = u / P.units_per_bh;
+        const int64_t r0 = (u % P.units_per_bh) * (kRows * kTiles);
+        const int64_t nr = min((int64_t)(kRows * kTiles), N - r0);
+        tc::prefetch_l2(P.o_loc + (bhu * N + r0) * D, (uint32_t)(nr * D * 2));
+        const __nv_bfloat16* gp0 = P.gate + bhu * N + r0;
+        const uint32_t gbytes = (uint32_t)(nr * 2) & ~15u;
+        if ((reinterpret_cast<uintptr_t>(gp0) & 15) == 0 && gbytes) tc::prefetch_l2(gp0, gbytes);
+      }
       if (pc >= 2) {
         // q buffer b still holds unit pc-2's staged o_glob: mix it, then refill the buffer
         if (!wait_staged(pc - 2)) { pok = false; break; }
