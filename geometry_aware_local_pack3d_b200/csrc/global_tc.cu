@@ -67,7 +67,8 @@ template <int D> struct Smem {
   static constexpr int kK = kQ + 2 * kTiles * kQTile;
   static constexpr int kV = kK + kStages * kCTile;
   static constexpr int kCoord = kV + kStages * kCTile;  // 256 packed coordinates
-  static constexpr int kRope = kCoord + kRows * kTiles * 4;
+  static constexpr int kGate = kCoord + kRows * kTiles * 4;  // [2 buffers][256] g = sigmoid(a)
+  static constexpr int kRope = kGate + 2 * kRows * kTiles * 4;
   static constexpr int kBar = kRope + kRopeSmemBytes;
   static constexpr int kBytes = kBar + 256;
 };
@@ -181,6 +182,8 @@ __global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
       const bool valid = row < N;
       // summaries excluded for this row: those whose box meets the cube [c-1, c+1]^3, kept as
       // summary-grid ranges [z0,z1] x [y0,y1] x [x0,x1] (empty when exclusion is off)
+      // the row's gate logit, loaded now and needed only by the epilogue
+      const float glogit = valid ? __bfloat162float(P.gate[bh * N + row]) : 0.f;
       const ExclBox xb = excl_box(P.ix, valid ? decode(P.ix.coord[row]) : Coord{0, 0, 0},
                                   P.exclude_near && valid);
       const int z0 = xb.z0, z1 = xb.z1, y0 = xb.y0, y1 = xb.y1, x0 = xb.x0, x1 = xb.x1;
@@ -332,6 +335,9 @@ __global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
             make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
       if (valid && P.lse_glob)
         P.lse_glob[bh * N + row] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      // the mixer's weight g = sigmoid(a) of the row, once per row
+      reinterpret_cast<float*>(smem + S::kGate)[(pc & 1) * kRows * kTiles + t * kRows + rin] =
+          1.f / (1.f + __expf(-glogit));
       tc::mbar_arrive(&bars[B_QEMPTY + (pc & 1)]);  // o_glob of this unit is staged
     }
   } else if (warp < W_MMA) {
@@ -343,30 +349,26 @@ __global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
     int32_t* coord_s = reinterpret_cast<int32_t*>(smem + S::kCoord);
     const float* rope = P.rope_in_smem ? reinterpret_cast<const float*>(smem + S::kRope) : P.ix.rope;
     // Mixer of unit k (the k-th unit of this CTA), once the softmax warps have staged its
-    // o_glob in q buffer k % 2: o = g o_loc + (1 - g) o_glob, g = sigmoid(a), over the unit's
-    // 256 rows with consecutive threads on consecutive 16 bytes. o_loc may alias o (in-place
+    // o_glob in q buffer k % 2 (and each row's g = sigmoid(a) beside it): o = g o_loc +
+    // (1 - g) o_glob over the unit's 256 rows with consecutive threads on consecutive 16 bytes. o_loc may alias o (in-place
     // mixing): every piece a thread stores is one it loaded itself, and loads come first.
     auto mix = [&](int k) {
       const int64_t uk = blockIdx.x + (int64_t)k * gridDim.x;
       const int64_t bh = uk / P.units_per_bh;
       const int64_t row0 = (uk % P.units_per_bh) * (kRows * kTiles);
       const uint8_t* stage = smem + S::kQ + (k & 1) * kTiles * S::kQTile;
+      const float* gsm = reinterpret_cast<const float*>(smem + S::kGate) + (k & 1) * kRows * kTiles;
       constexpr int G = D == 96 ? 12 : 6;  // pieces per thread in flight
       static_assert((kRows * kTiles * KC / kProd) % G == 0, "mixer groups");
 #pragma unroll 1
       for (int g0 = 0; g0 < kRows * kTiles * KC / kProd; g0 += G) {
         uint4 lv[G];
-        float gs[G];
 #pragma unroll
         for (int i = 0; i < G; ++i) {
           const int pidx = (g0 + i) * kProd + ptid, r = pidx / KC, c = pidx % KC;
           const int64_t grow = row0 + r;
           lv[i] = make_uint4(0u, 0u, 0u, 0u);
-          gs[i] = 0.f;
-          if (grow < N) {
-            lv[i] = reinterpret_cast<const uint4*>(P.o_loc + (bh * N + grow) * D)[c];
-            gs[i] = __bfloat162float(P.gate[bh * N + grow]);
-          }
+          if (grow < N) lv[i] = reinterpret_cast<const uint4*>(P.o_loc + (bh * N + grow) * D)[c];
         }
 #pragma unroll
         for (int i = 0; i < G; ++i) {
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(gtc::Roles<PW>::kThreads, 1)
           const int rin = r & (kRows - 1);
           const uint4 gv = *reinterpret_cast<const uint4*>(
               stage + (r >> 7) * S::kQTile + rin * (D * 2) + ((c + rin) % KC) * 16);
-          const float g = 1.f / (1.f + __expf(-gs[i]));
+          const float g = gsm[r];  // sigmoid(a) of the row, left by the epilogue
           const uint32_t lw[4] = {lv[i].x, lv[i].y, lv[i].z, lv[i].w};
           const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
           uint32_t outw[4];
