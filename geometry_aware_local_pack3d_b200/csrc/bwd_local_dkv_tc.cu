@@ -85,6 +85,7 @@ enum {
   B_DRAIN = 35,
   B_COUNT = 36
 };
+static_assert(B_KVEMPTY - B_KVFULL >= kStages && B_BOX - B_KVEMPTY >= kStages, "ring barriers");
 static_assert(8 * B_COUNT + 16 <= 1024, "barrier area");
 
 struct Params {

@@ -90,6 +90,7 @@ enum {
   B_DRAIN = 40,   // [tile]
   B_COUNT = 42
 };
+static_assert(B_KVEMPTY - B_KVFULL >= kStages && B_BOX - B_KVEMPTY >= kStages, "ring barriers");
 static_assert(8 * B_COUNT + 16 <= 1024, "barrier area");
 
 struct Params {

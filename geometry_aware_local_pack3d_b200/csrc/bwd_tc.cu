@@ -39,6 +39,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Asynchronous 4-byte global -> shared copy (through L1); zero-filled when `valid` is false.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(tc::smem_u32(smem_dst)),
+               "l"(gsrc), "r"(valid ? 4 : 0)
+               : "memory");
+}
+
 
 struct Params {
   pack3d_index ix;
@@ -325,7 +332,8 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
 
 // ======================================================================= dK, dV (summaries)
 namespace bds {
-constexpr int kStages = 3;
+constexpr int kStages = 4;
+constexpr int kLag = 1;  // a tile's row data is finalized this many tiles after its copies
 template <int D> struct Smem {
   static constexpr int kATile = btc::kRows * D * 2;    // K or V summaries, 128 rows
   static constexpr int kBTile = btc::kChunk * D * 2;   // q~ or dO_g, 64 rows
@@ -335,13 +343,16 @@ template <int D> struct Smem {
   static constexpr int kG = kQ + kStages * kBTile;     // [stages]
   static constexpr int kRowF = kG + kStages * kBTile;          // [stages][64] (nl, D)
   static constexpr int kRowX = kRowF + kStages * btc::kChunk * 8;  // [stages][64][6] ranges
-  static constexpr int kBar = kRowX + kStages * btc::kChunk * 24;
+  // [stages][3][64] raw lse, D and packed coordinate of the tile's queries, as copied
+  static constexpr int kRaw = kRowX + kStages * btc::kChunk * 24;
+  static constexpr int kBar = kRaw + kStages * 3 * btc::kChunk * 4;
   static constexpr int kBytes = kBar + 256;
 };
 enum {
-  B_QFULL = 0, B_QEMPTY = 3, B_AFULL = 6, B_SFULL = 7, B_PFULL = 9, B_DONE = 11, B_DRAIN = 13,
-  B_COUNT = 14
+  B_QFULL = 0, B_QEMPTY = B_QFULL + kStages, B_AFULL = B_QEMPTY + kStages, B_SFULL = B_AFULL + 1,
+  B_PFULL = B_SFULL + 2, B_DONE = B_PFULL + 2, B_DRAIN = B_DONE + 2, B_COUNT = B_DRAIN + 1
 };
+static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
 constexpr int kThreads = 288;  // elementwise 0-3, producer 4-7, MMA 8
 constexpr int kProd = 128;
 // TMEM columns: dK, dV accumulators; S^T and dP^T double-buffered (buffer b of tile i = i % 2)
@@ -510,37 +521,64 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
     tc::cp_async_wait_all();
     tc::fence_proxy_async_smem();
     tc::mbar_arrive(&bars[B_AFULL]);
-    for (int i = 0; i < NT; ++i) {
-      const int st = i % kStages;
-      if (i >= kStages && !pwait(&bars[B_QEMPTY + st], ((i / kStages) - 1) & 1)) break;
-      const int64_t row0 = (int64_t)(qt0 + i) * btc::kChunk;
-      for (int k = ptid; k < btc::kChunk * KC; k += kProd) {
-        int r, kc;
-        tc::PieceOrder<KC>::at(k, r, kc);
-        const int64_t row = row0 + r;
-        const bool ok = row < N;
-        const int64_t src = (bh * N + (ok ? row : 0)) * D + kc * 8;
-        const int off = st * S::kBTile + kc * CB + (r >> 3) * 128 + (r & 7) * 16;
-        tc::cp_async16(smem + S::kQ + off, P.qtb + src, ok);
-        tc::cp_async16(smem + S::kG + off, P.dogb + src, ok);
+    // Software pipeline: at step i the copies of tile i are issued (q~ and dO_g rows, and
+    // each query's lse, D and coordinate as raw 4-byte copies), and tile i - kLag, whose
+    // copies have landed, is finalized: its per-query (-lse log2(e), D) and exclusion ranges
+    // are formed in shared memory and the tile is handed to the MMA warp. No producer thread
+    // waits on a global load, and kLag + 1 tiles are in flight.
+    const float* raw = reinterpret_cast<const float*>(smem + S::kRaw);
+    bool pok = true;
+    for (int i = 0; i < NT + kLag && pok; ++i) {
+      if (i < NT) {
+        const int st = i % kStages;
+        if (i >= kStages && !pwait(&bars[B_QEMPTY + st], ((i / kStages) - 1) & 1)) {
+          pok = false;
+          break;
+        }
+        const int64_t row0 = (int64_t)(qt0 + i) * btc::kChunk;
+        for (int k = ptid; k < btc::kChunk * KC; k += kProd) {
+          int r, kc;
+          tc::PieceOrder<KC>::at(k, r, kc);
+          const int64_t row = row0 + r;
+          const bool ok = row < N;
+          const int64_t src = (bh * N + (ok ? row : 0)) * D + kc * 8;
+          const int off = st * S::kBTile + kc * CB + (r >> 3) * 128 + (r & 7) * 16;
+          tc::cp_async16(smem + S::kQ + off, P.qtb + src, ok);
+          tc::cp_async16(smem + S::kG + off, P.dogb + src, ok);
+        }
+        if (ptid < btc::kChunk) {
+          const int64_t row = row0 + ptid;
+          const bool ok = row < N;
+          const int64_t g = bh * N + (ok ? row : 0);
+          float* rw = reinterpret_cast<float*>(smem + S::kRaw) + st * 3 * btc::kChunk;
+          btc::cp_async4(rw + ptid, P.lse + g, ok);
+          btc::cp_async4(rw + btc::kChunk + ptid, P.Dg + g, ok);
+          if (P.exclude_near)
+            btc::cp_async4(rw + 2 * btc::kChunk + ptid, P.ix.coord + (ok ? row : 0), ok);
+        }
       }
+      tc::cp_async_commit();  // one group per step (empty past the last tile)
+      const int f = i - kLag;
+      if (f < 0) continue;
+      tc::cp_async_wait_group<kLag>();  // tile f's copies have landed
+      const int sf = f % kStages;
       if (ptid < btc::kChunk) {
-        const int64_t row = row0 + ptid;
+        const int64_t row = (int64_t)(qt0 + f) * btc::kChunk + ptid;
+        const float* rw = raw + sf * 3 * btc::kChunk;
         float2 rf = make_float2(-INFINITY, 0.f);
         ExclBox ex{0, -1, 0, -1, 0, -1};
         if (row < N) {
-          const float lse = P.lse[bh * N + row];
-          rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY, P.Dg[bh * N + row]);
-          ex = excl_box(P.ix, decode(P.ix.coord[row]), P.exclude_near != 0);
+          const float lse = rw[ptid];
+          rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY, rw[btc::kChunk + ptid]);
+          if (P.exclude_near)
+            ex = excl_box(P.ix, decode(__float_as_int(rw[2 * btc::kChunk + ptid])), true);
         }
-        reinterpret_cast<float2*>(smem + S::kRowF)[st * btc::kChunk + ptid] = rf;
-        int* x = reinterpret_cast<int*>(smem + S::kRowX) + (st * btc::kChunk + ptid) * 6;
+        reinterpret_cast<float2*>(smem + S::kRowF)[sf * btc::kChunk + ptid] = rf;
+        int* x = reinterpret_cast<int*>(smem + S::kRowX) + (sf * btc::kChunk + ptid) * 6;
         x[0] = ex.z0; x[1] = ex.z1; x[2] = ex.y0; x[3] = ex.y1; x[4] = ex.x0; x[5] = ex.x1;
       }
-      tc::cp_async_commit();
-      tc::cp_async_wait_all();
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[B_QFULL + st]);
+      tc::mbar_arrive(&bars[B_QFULL + sf]);
     }
     tc::cp_async_wait_all();
   } else {
