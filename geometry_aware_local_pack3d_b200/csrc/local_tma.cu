@@ -559,6 +559,8 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           tc::mbar_expect_tx(&bars[B_BOX + bb], kBoxBytes);
           tc::tma_load_3d(box, &mg, x0 - 4, y0 - 1, z0 - 1, &bars[B_BOX + bb]);
         }
+        // the box is read below (this phase of its barrier completes when it has landed)
+        if (!wwait(&bars[B_BOX + bb], (ti >> 1) & 1)) break;
       } else {
         for (int i = lane; i < kBoxX * kBoxY * kBoxZ; i += 32) {
           const int bx = i % kBoxX, by = (i / kBoxX) % kBoxY, bz = i / (kBoxX * kBoxY);
@@ -570,6 +572,15 @@ __global__ void __launch_bounds__(lg::kThreads, 1)
           ++box_phases[bb];
           tc::mbar_arrive(&bars[B_BOX + bb]);
         }
+      }
+      // The unit's q rows are read by two softmax warps per tile when the unit before it
+      // ends, between two units' MMA chains; start bringing them into L2 now, about one unit
+      // ahead (one bulk prefetch per present row of the 4 x 8 x 8 brick).
+      for (int i = lane; i < 4 * 8 * 8; i += 32) {
+        const int z = i >> 6, y = (i >> 3) & 7, x = i & 7;
+        if (!in_grid(z0 + z, y0 + y, x0 + x)) continue;
+        const int slot = box[((z + 1) * kBoxY + y + 1) * kBoxX + x + 4];
+        if (slot >= 0) tc::prefetch_l2(P.q + (bh * N + slot) * D, D * 2);
       }
     }
     // nothing may still be landing in shared memory when the CTA exits: wait for the latest
