@@ -22,6 +22,8 @@
 // Operands use the no-swizzle core-matrix layout; the summary tiles are already in it.
 #include <math.h>
 
+#include <type_traits>
+
 #include "bwd_work.h"
 #include "common.cuh"
 #include "launch.h"
@@ -37,6 +39,17 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// (a.x b.x, a.y b.y) in one instruction, round to nearest
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 // Asynchronous 4-byte global -> shared copy (through L1); zero-filled when `valid` is false.
@@ -147,6 +160,7 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
       const float Dg = valid ? P.Dg[grow] : 0.f;
       const bool live = lse != -INFINITY;  // every summary excluded: no global gradient
       const float nl = live ? -lse * kLog2e : 0.f;
+      const float Ds = Dg * P.scale;
       const ExclBox ex = excl_box(P.ix, decode(valid ? P.ix.coord[row] : 0),
                                   P.exclude_near != 0 && valid);
       for (int j = 0; j < NC; ++j, ++gc) {
@@ -164,9 +178,18 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
                 xm[1] |= (cidx >> 5) == 1 ? (1u << (cidx & 31)) : 0u;
               }
             }
-        // two halves of 32 columns: read S and dP, write dS (bf16) over S columns already read
+        // two halves of 32 columns: read S and dP, write dS (bf16) over S columns already read.
+        // Two columns per step with packed fp32: P = 2^(S tau log2(e) - lse log2(e)),
+        // dS = P (dP tau - D tau); the columns whose P is zero (no global gradient for the
+        // row, past the last summary, or excluded) are one bit mask per half.
+        const float2 sl2 = make_float2(P.scale_log2, P.scale_log2);
+        const float2 sc2 = make_float2(P.scale, P.scale);
+        const float2 nl2 = make_float2(nl, nl), nds2 = make_float2(-Ds, -Ds);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          const int lim = M - m0 - 32 * h;  // columns of this half with a summary
+          uint32_t zm = xm[h] | (live ? 0u : 0xffffffffu);
+          if (lim < 32) zm |= lim <= 0 ? 0xffffffffu : (0xffffffffu << lim);
           uint32_t sv[32], dv[32];
           tc::tmem_ld32(tl + kS + 32 * h, sv);
           tc::tmem_ld32(tl + kP + 32 * h, dv);
@@ -174,15 +197,15 @@ __global__ void __launch_bounds__(bdq::kThreads, 2) k_bwd_dq_tc(const btc::Param
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            float ds[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = 32 * h + k + e;
-              const bool use = live && m0 + col < M && !((xm[h] >> (k + e)) & 1u);
-              const float p = use ? btc::ex2(fmaf(__uint_as_float(sv[k + e]), P.scale_log2, nl)) : 0.f;
-              ds[e] = p * (__uint_as_float(dv[k + e]) - Dg) * P.scale;
-            }
-            pk[k >> 1] = tc::pack_bf16(ds[0], ds[1]);
+            const float2 x = tc::fma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
+                                      sl2, nl2);
+            float2 p = make_float2(btc::ex2(x.x), btc::ex2(x.y));
+            p.x = ((zm >> k) & 1u) ? 0.f : p.x;
+            p.y = ((zm >> (k + 1)) & 1u) ? 0.f : p.y;
+            const float2 t = tc::fma2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                      sc2, nds2);
+            const float2 ds = btc::mul2(p, t);
+            pk[k >> 1] = tc::pack_bf16(ds.x, ds.y);
           }
           tc::tmem_st16(tl + kS + 16 * h, pk);
         }
@@ -359,7 +382,7 @@ constexpr int kProd = 128;
 constexpr uint32_t kK = 0, kV = 128;
 __device__ __forceinline__ uint32_t s_col(int b) { return 256u + 128u * b; }
 __device__ __forceinline__ uint32_t p_col(int b) { return 320u + 128u * b; }
-// Per query of a tile (staged by the producer): (-lse log2(e), D) -- -inf in place of the
+// Per query of a tile (staged by the producer): (-lse log2(e), D tau) -- -inf in place of the
 // first term when the query has no global gradient, so that P = 0 -- and the block
 // coordinate ranges [z0, z1] x [y0, y1] x [x0, x1] of the summaries exclude_near drops.
 }  // namespace bds
@@ -424,37 +447,51 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
       tc::tc_fence_after();
       const float2* rf = rowf + st * btc::kChunk;
       const int* rx = rowx + st * btc::kChunk * 6;
-      // two halves of 32 query columns: P^T over S^T, dS^T over dP^T (columns already read)
+      // two halves of 32 query columns: P^T over S^T, dS^T over dP^T (columns already read).
+      // Two columns per step with packed fp32: P = 2^(S tau log2(e) - lse log2(e)),
+      // dS = P (dP tau - D tau); one 16-byte read brings both columns' row data.
+      const float4* rf4 = reinterpret_cast<const float4*>(rf);
+      const float2 sl2 = make_float2(P.scale_log2, P.scale_log2);
+      const float2 sc2 = make_float2(P.scale, P.scale);
+      auto pass = [&](auto excl_c) {
+        constexpr bool kExcl = decltype(excl_c)::value;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t sv[32], dv[32];
-        tc::tmem_ld32(tl + s_col(b) + 32 * h, sv);
-        tc::tmem_ld32(tl + p_col(b) + 32 * h, dv);
-        tc::tmem_wait_ld();
-        uint32_t pp[16], pd[16];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sv[32], dv[32];
+          tc::tmem_ld32(tl + s_col(b) + 32 * h, sv);
+          tc::tmem_ld32(tl + p_col(b) + 32 * h, dv);
+          tc::tmem_wait_ld();
+          uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float pv[2], dsv[2];
+          for (int k = 0; k < 32; k += 2) {
+            const int col = 32 * h + k;
+            const float4 r = rf4[col >> 1];  // broadcast: every thread reads the same
+            const float2 x = tc::fma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])),
+                                      sl2, make_float2(r.x, r.z));
+            float2 p = make_float2(btc::ex2(x.x), btc::ex2(x.y));
+            if constexpr (kExcl) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 32 * h + k + e;
-            const float2 r = rf[col];  // broadcast: every thread reads the same
-            float p = btc::ex2(fmaf(__uint_as_float(sv[k + e]), P.scale_log2, r.x));
-            if (excl) {
-              const int* x = rx + col * 6;
-              if (bz >= x[0] && bz <= x[1] && byy >= x[2] && byy <= x[3] && bxx >= x[4] &&
-                  bxx <= x[5])
-                p = 0.f;
+              for (int e = 0; e < 2; ++e) {
+                const int* xr = rx + (col + e) * 6;
+                if (bz >= xr[0] && bz <= xr[1] && byy >= xr[2] && byy <= xr[3] && bxx >= xr[4] &&
+                    bxx <= xr[5])
+                  (e == 0 ? p.x : p.y) = 0.f;
+              }
             }
-            pv[e] = p;
-            dsv[e] = p * (__uint_as_float(dv[k + e]) - r.y) * P.scale;
+            const float2 t = tc::fma2(make_float2(__uint_as_float(dv[k]), __uint_as_float(dv[k + 1])),
+                                      sc2, make_float2(-r.y, -r.w));
+            const float2 ds = btc::mul2(p, t);
+            pp[k >> 1] = tc::pack_bf16(p.x, p.y);
+            pd[k >> 1] = tc::pack_bf16(ds.x, ds.y);
           }
-          pp[k >> 1] = tc::pack_bf16(pv[0], pv[1]);
-          pd[k >> 1] = tc::pack_bf16(dsv[0], dsv[1]);
+          tc::tmem_st16(tl + s_col(b) + 16 * h, pp);
+          tc::tmem_st16(tl + p_col(b) + 16 * h, pd);
         }
-        tc::tmem_st16(tl + s_col(b) + 16 * h, pp);
-        tc::tmem_st16(tl + p_col(b) + 16 * h, pd);
-      }
+      };
+      if (excl)
+        pass(std::true_type{});
+      else
+        pass(std::false_type{});
       tc::tmem_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars[B_PFULL + b]);
@@ -569,7 +606,8 @@ __global__ void __launch_bounds__(bds::kThreads, 1) k_bwd_dsum_tc(const btc::Par
         ExclBox ex{0, -1, 0, -1, 0, -1};
         if (row < N) {
           const float lse = rw[ptid];
-          rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY, rw[btc::kChunk + ptid]);
+          rf = make_float2(lse != -INFINITY ? -lse * kLog2e : -INFINITY,
+                           rw[btc::kChunk + ptid] * P.scale);
           if (P.exclude_near)
             ex = excl_box(P.ix, decode(__float_as_int(rw[2 * btc::kChunk + ptid])), true);
         }

@@ -219,27 +219,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for two values on the FMA pipe instead of the MUFU pipe (x <= 126). Range reduction:
-// x is clamped below at -127 (so -inf gives +0 exactly), n = round(x) by adding 1.5 * 2^23
-// (n then sits in the low mantissa bits of t), f = x - n in [-1/2, 1/2]; 2^f is a cubic with
-// p(0) = 1 fitted in float64 to 2^f on [-1/2, 1/2] by iteratively reweighted least squares
-// toward the minimax relative error (max relative error 1.0e-4, well inside bf16's 2^-9), and
-// n is added to the exponent field.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  constexpr float c1 = 0.6932829022f, c2 = 0.2422109693f, c3 = 0.0550089329f;
-  x.x = fmaxf(x.x, -127.f);
-  x.y = fmaxf(x.y, -127.f);
-  const float2 t = add2(x, make_float2(kShift, kShift));
-  const float2 n = add2(t, make_float2(-kShift, -kShift));
-  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = fma2(f, make_float2(c3, c3), make_float2(c2, c2));
-  p = fma2(p, f, make_float2(c1, c1));
-  p = fma2(p, f, make_float2(1.f, 1.f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // One lane of a fully active warp (elect.sync): the lane that issues a warp's MMAs.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
