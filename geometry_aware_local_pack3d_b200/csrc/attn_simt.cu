@@ -371,54 +371,169 @@ __device__ __forceinline__ void gr_rotate(const pack3d_index& ix, const Coord& c
   }
 }
 
+// Row prologue, one pass over the rows of q, k, dO, o_loc and o_glob with 16-byte pieces: each
+// row is read by a group of G lanes (G = C rounded up to a power of two, C = 16-byte pieces
+// per row), a warp takes 32 / G rows at a time and the warps walk the rows persistently. The
+// rotation table, read at every row's coordinate, sits in shared memory when it fits (a grid
+// extent up to 170 at d = 96). The pair rotation is x0' = x0 c - x1 s, x1' = x0 s + x1 c with
+// one rounding of the product and one of the fma, and the row sums reduce over the group's
+// lanes with xor shuffles.
+template <typename T, int D> struct PrepShape {
+  static constexpr int kC = D / Vec<T>::E;
+  static constexpr int kG = kC <= 8 ? 8 : (kC <= 16 ? 16 : 32);
+};
+constexpr int kPrepThreads = 256;
+constexpr int kPrepTableMax = 65536;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128) k_bwd_prep(pack3d_index ix, const T* __restrict__ q,
-                                                  const T* __restrict__ k,
-                                                  const T* __restrict__ gate,
-                                                  const T* __restrict__ o_loc,
-                                                  const T* __restrict__ o_glob,
-                                                  const T* __restrict__ dO, int64_t rows,
-                                                  int kv_group, BwdWork w,
-                                                  T* __restrict__ dgate) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int64_t i = row % ix.n;
-  const int64_t kvrow = kv_of(row / ix.n, kv_group) * ix.n + i;  // the key of the KV head
-  const Coord c = decode(ix.coord[i]);
-  WarpRow<D> a, b, d;
-  wr_load<T, D>(q + row * D, a, lane);
-  wr_rotate<D>(ix, c, a, lane, 1.f);
-  wr_load<T, D>(k + kvrow * D, b, lane);
-  wr_rotate<D>(ix, c, b, lane, 1.f);
+__device__ __forceinline__ void prep_rotate(float (&x)[Vec<T>::E], const float2* cs) {
+#pragma unroll
+  for (int e = 0; e < Vec<T>::E; e += 2) {
+    const float2 r = cs[e / 2];
+    const float x0 = x[e], x1 = x[e + 1];
+    x[e] = fmaf(-x1, r.y, x0 * r.x);
+    x[e + 1] = fmaf(x0, r.y, x1 * r.x);
+  }
+}
+
+template <typename T, int D, bool kTab>
+__global__ void __launch_bounds__(kPrepThreads) k_bwd_prep(pack3d_index ix, const T* __restrict__ q,
+                                                           const T* __restrict__ k,
+                                                           const T* __restrict__ gate,
+                                                           const T* __restrict__ o_loc,
+                                                           const T* __restrict__ o_glob,
+                                                           const T* __restrict__ dO, int64_t rows,
+                                                           int kv_group, BwdWork w,
+                                                           T* __restrict__ dgate) {
+  constexpr int E = Vec<T>::E;
+  constexpr int C = PrepShape<T, D>::kC, G = PrepShape<T, D>::kG, RPW = 32 / G;
+  constexpr int DA = D / 3;
+  static_assert(DA % E == 0, "a 16-byte piece must stay inside one axis third");
+  extern __shared__ __align__(16) float prep_tab[];
+  const float* rope = ix.rope;
+  if constexpr (kTab) {
+    const int n16 = 6 * ix.rope_rows * ix.rope_pairs / 4;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x)
+      reinterpret_cast<float4*>(prep_tab)[i] = __ldg(reinterpret_cast<const float4*>(ix.rope) + i);
+    __syncthreads();
+    rope = prep_tab;
+  }
+  const int lane = threadIdx.x & 31, sub = lane / G, c = lane % G;
+  const bool active = c < C;
+  const int pc = active ? c : 0;  // an idle lane works on piece 0 and keeps nothing
+  const int axis = (pc * E) / DA, p0 = ((pc * E) % DA) / 2;
+  const float* tab_lane = rope + 2 * rope_slot(ix.rope_rows, ix.rope_pairs, axis, 0, p0);
+  const int tab_row = 2 * ix.rope_pairs, csh = 20 - 10 * axis;
+  const int64_t N = ix.n;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   T* qr = static_cast<T*>(w.qr);
   T* kr = static_cast<T*>(w.kr);
+  for (int64_t r0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+       r0 < rows; r0 += nwarps * RPW) {
+    const int64_t row = r0 + sub;
+    const bool live = row < rows;
+    const bool ok = active && live;
+    const int64_t i = live ? row % N : 0;
+    const int64_t kvrow = kv_of(live ? row / N : 0, kv_group) * N + i;  // the key of the KV head
+    float xq[E], xk[E], xd[E], xl[E], xg[E];
 #pragma unroll
-  for (int t = 0; t < WarpRow<D>::KT; ++t) {
-    const int e = lane + 32 * t;
-    if (e < D) {
-      qr[row * D + e] = from_f<T>(a.x[t]);
-      kr[row * D + e] = from_f<T>(b.x[t]);
+    for (int e = 0; e < E; ++e) xq[e] = xk[e] = xd[e] = xl[e] = xg[e] = 0.f;
+    const int64_t off = (live ? row : 0) * D + pc * E;
+    if (ok) {
+      Vec<T>::load(q + off, xq);
+      Vec<T>::load(k + kvrow * D + pc * E, xk);
+      Vec<T>::load(dO + off, xd);
+      Vec<T>::load(o_loc + off, xl);
+      Vec<T>::load(o_glob + off, xg);
+    }
+    const int32_t cc = live ? __ldg(ix.coord + i) : 0;
+    const float a = live ? to_f(gate[row]) : 0.f;
+    // (cos, sin) of the piece's E / 2 pairs at the row's coordinate on this lane's axis
+    float2 cs[E / 2];
+    {
+      const float4* cs4 = reinterpret_cast<const float4*>(tab_lane + tab_row * ((cc >> csh) & 1023));
+#pragma unroll
+      for (int h = 0; h < E / 4; ++h) {
+        const float4 t4 = kTab ? cs4[h] : __ldg(cs4 + h);
+        cs[2 * h] = make_float2(t4.x, t4.y);
+        cs[2 * h + 1] = make_float2(t4.z, t4.w);
+      }
+    }
+    prep_rotate<T, D>(xq, cs);
+    prep_rotate<T, D>(xk, cs);
+    const float g = 1.f / (1.f + expf(-a));
+    float dl = 0.f, dgl = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      dl = fmaf(xd[e], xl[e], dl);
+      dgl = fmaf(xd[e], xg[e], dgl);
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) {
+      dl += __shfl_xor_sync(0xffffffffu, dl, o);
+      dgl += __shfl_xor_sync(0xffffffffu, dgl, o);
+    }
+    if (ok) {
+      Vec<T>::store(qr + off, xq);
+      Vec<T>::store(kr + off, xk);
+      if (w.dogb) {
+        // tensor-core path: (1 - g) dO rows in bf16, an MMA operand (the rotated q is qr)
+        uint32_t pk[E / 2];
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn((1.f - g) * xd[e], (1.f - g) * xd[e + 1]);
+          pk[e / 2] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        if constexpr (E == 8)
+          *reinterpret_cast<uint4*>(w.dogb + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        else
+          *reinterpret_cast<uint2*>(w.dogb + off) = make_uint2(pk[0], pk[1]);
+      }
+    }
+    if (live && c == 0) {
+      dgate[row] = from_f<T>((dl - dgl) * g * (1.f - g));
+      w.Dl[row] = g * dl;
+      w.Dg[row] = (1.f - g) * dgl;
     }
   }
-  wr_load<T, D>(dO + row * D, d, lane);
-  const float g = 1.f / (1.f + expf(-to_f(gate[row])));
-  if (w.dogb) {
-    // tensor-core path: (1 - g) dO rows in bf16, an MMA operand (the rotated q is qr)
-#pragma unroll
-    for (int t = 0; t < WarpRow<D>::KT; ++t) {
-      const int e = lane + 32 * t;
-      if (e < D) w.dogb[row * D + e] = __float2bfloat16_rn((1.f - g) * d.x[t]);
-    }
-  }
-  wr_load<T, D>(o_loc + row * D, a, lane);
-  wr_load<T, D>(o_glob + row * D, b, lane);
-  const float dl = wr_dot<D>(d, a), dgl = wr_dot<D>(d, b);
-  if (lane == 0) {
-    dgate[row] = from_f<T>((dl - dgl) * g * (1.f - g));
-    w.Dl[row] = g * dl;
-    w.Dg[row] = (1.f - g) * dgl;
-  }
+}
+
+template <typename T, int D, bool kTab>
+cudaError_t launch_bwd_prep_as(const pack3d_index& ix, const T* q, const T* k, const T* gate,
+                               const T* o_loc, const T* o_glob, const T* dO, int64_t rows,
+                               int kv_group, const BwdWork& w, T* dgate, int smem,
+                               cudaStream_t s) {
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e =
+      smem_attr_once(reinterpret_cast<const void*>(k_bwd_prep<T, D, kTab>), kPrepTableMax, attr_done);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_bwd_prep<T, D, kTab>, kPrepThreads,
+                                                    smem);
+  if (e != cudaSuccess) return e;
+  occ = occ > 0 ? occ : 1;
+  constexpr int RPW = 32 / PrepShape<T, D>::kG;
+  const int64_t per_cta = (int64_t)(kPrepThreads / 32) * RPW;
+  const int64_t need = (rows + per_cta - 1) / per_cta;
+  const int64_t resident = (int64_t)occ * sm_count();
+  const unsigned grid = (unsigned)(need < resident ? need : resident);
+  if (grid == 0) return cudaSuccess;
+  k_bwd_prep<T, D, kTab><<<grid, kPrepThreads, smem, s>>>(ix, q, k, gate, o_loc, o_glob, dO, rows,
+                                                          kv_group, w, dgate);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd_prep(const pack3d_index& ix, const T* q, const T* k, const T* gate,
+                            const T* o_loc, const T* o_glob, const T* dO, int64_t rows,
+                            int kv_group, const BwdWork& w, T* dgate, cudaStream_t s) {
+  const int tab = 24 * ix.rope_rows * ix.rope_pairs;  // bytes: [3, rows, pairs] x (cos, sin)
+  if (tab <= kPrepTableMax)
+    return launch_bwd_prep_as<T, D, true>(ix, q, k, gate, o_loc, o_glob, dO, rows, kv_group, w,
+                                          dgate, tab, s);
+  return launch_bwd_prep_as<T, D, false>(ix, q, k, gate, o_loc, o_glob, dO, rows, kv_group, w,
+                                         dgate, 0, s);
 }
 
 template <typename T, int D>
@@ -671,17 +786,18 @@ cudaError_t bwd_simt(const pack3d_index& ix, const void* q, const void* k, const
                      void* dk, void* dv, void* dgate, void* ws, bool tc, cudaStream_t s) {
   const BwdWork w = bwd_carve(ix, bh, ws, sizeof(T), tc, kv_group);
   const int64_t rows = bh * ix.n;
-  const unsigned rb = (unsigned)((rows + 3) / 4);
   const unsigned mb = (unsigned)((bh * ix.m + 3) / 4);
   const T* tq = static_cast<const T*>(q);
   const T* tk = static_cast<const T*>(k);
   const T* tv = static_cast<const T*>(v);
   const T* tg = static_cast<const T*>(gate);
   const T* tdo = static_cast<const T*>(dO);
-  k_bwd_prep<T, D><<<rb, 128, 0, s>>>(ix, tq, tk, tg, static_cast<const T*>(o_loc),
-                                       static_cast<const T*>(o_glob), tdo, rows, kv_group, w,
-                                       static_cast<T*>(dgate));
-  count_launch();
+  {
+    const cudaError_t e = launch_bwd_prep<T, D>(ix, tq, tk, tg, static_cast<const T*>(o_loc),
+                                                static_cast<const T*>(o_glob), tdo, rows,
+                                                kv_group, w, static_cast<T*>(dgate), s);
+    if (e != cudaSuccess) return e;
+  }
   if (tc) {
     // the global branch's summary gradients and its part of dq on tensor cores
     const cudaError_t e =
