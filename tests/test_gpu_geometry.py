@@ -76,6 +76,12 @@ CASES = {
                       "raster", True),
     "mqa_centre_sparse": ((6, 6, 10), (2, 3, 2), 1, 3, 1, 96, 0.7, (1, 2, 1), "centre",
                           (1.0, 0.25, 2.0), "raster_block", True),
+    # a long axis: the rotation table (3 x extent x d/6 pairs of (cos, sin)) is larger than
+    # 64 KB, so the kernels that otherwise keep it in shared memory read it from L1 / L2
+    "long_axis_d96": ((2, 3, 200), (2, 2, 4), 1, 2, 2, 96, 0.9, (1, 1, 1), "token", None,
+                      "morton", False),
+    "long_axis_d48_centre": ((2, 2, 400), (1, 2, 8), 1, 2, 1, 48, 1.0, (1, 1, 2), "centre",
+                             None, "raster", True),
 }
 
 
