@@ -541,6 +541,19 @@ __global__ void __launch_bounds__(lk::kThreads, 1)
       int z0, y0, x0;
       origin(u, bh, z0, y0, x0);
       const int64_t qbase = bh * N;
+      // per piece, fixed for the unit: the box index of its (hy, hx) column in slice 0 (-1 when
+      // the column is off the grid in y or x)
+      int bidx[NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf;
+        const int y = y0 - 1 + hy, x = x0 - 1 + hx;
+        bidx[j] = (pc[j] != 0xffffffffu && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
+                      ? hy * kBoxX + hx + 3
+                      : -1;
+      }
+      const __nv_bfloat16* qgb = P.qr + qbase * D;
+      const __nv_bfloat16* ggb = P.dO + qbase * D;
       for (int s = 0; s < kChunks; ++s, ++gs) {
         const int st = gs % kStages;
         if (gs >= (uint32_t)kStages && !pwait(&bars[B_KVEMPTY + st], ((gs / kStages) - 1) & 1)) {
@@ -550,18 +563,15 @@ __global__ void __launch_bounds__(lk::kThreads, 1)
         uint8_t* qd = smem + S::kQ + st * S::kStage;
         uint8_t* gd = smem + S::kG + st * S::kStage;
         const bool zin = z0 - 1 + s >= 0 && z0 - 1 + s < g.gz;
+        const int32_t* sbox = box + s * kBoxY * kBoxX;
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
           if (pc[j] == 0xffffffffu) continue;
-          const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf, c = pc[j] >> 24;
-          const int y = y0 - 1 + hy, x = x0 - 1 + hx;
-          int slot = -1;
-          if (zin && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
-            slot = box[(s * kBoxY + hy) * kBoxX + hx + 3];
-          const int64_t src = (qbase + (slot >= 0 ? slot : 0)) * D + c * 8;
+          const int slot = (zin && bidx[j] >= 0) ? sbox[bidx[j]] : -1;
+          const int64_t src = (int64_t)(slot >= 0 ? slot : 0) * D + (int)(pc[j] >> 24) * 8;
           const uint32_t off = (pc[j] & 0xffffu) << 4;
-          tc::cp_async16(qd + off, P.qr + src, slot >= 0);
-          tc::cp_async16(gd + off, P.dO + src, slot >= 0);
+          tc::cp_async16(qd + off, qgb + src, slot >= 0);
+          tc::cp_async16(gd + off, ggb + src, slot >= 0);
         }
         tc::cp_async_arrive_noinc(&bars[B_KVFULL + st]);
         if (pt < kNK) {

@@ -479,6 +479,19 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       origin(u, bh, z0, y0, x0);
       const int64_t kbase = bh * N;                       // k~ rows of the query head
       const int64_t vbase = kv_of(bh, P.kv_group) * N;    // v rows of the KV head
+      // per piece, fixed for the unit: the box index of its (hy, hx) column in slice 0 (-1 when
+      // the column is off the grid in y or x)
+      int bidx[NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf;
+        const int y = y0 - 1 + hy, x = x0 - 1 + hx;
+        bidx[j] = (pc[j] != 0xffffffffu && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
+                      ? hy * kBoxX + hx + 3
+                      : -1;
+      }
+      const __nv_bfloat16* kgb = P.kr + kbase * D;
+      const __nv_bfloat16* vgb = P.v + vbase * D;
       for (int s = 0; s < kChunks; ++s, ++gs) {
         const int st = gs % kStages;
         if (gs >= (uint32_t)kStages && !pwait(&bars[B_KVEMPTY + st], ((gs / kStages) - 1) & 1)) {
@@ -488,18 +501,15 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
         uint8_t* kd = smem + S::kK + st * S::kStage;
         uint8_t* vd = smem + S::kV + st * S::kStage;
         const bool zin = z0 - 1 + s >= 0 && z0 - 1 + s < g.gz;
+        const int32_t* sbox = box + s * kBoxY * kBoxX;
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
           if (pc[j] == 0xffffffffu) continue;
-          const int hy = (pc[j] >> 16) & 0xf, hx = (pc[j] >> 20) & 0xf, c = pc[j] >> 24;
-          const int y = y0 - 1 + hy, x = x0 - 1 + hx;
-          int slot = -1;
-          if (zin && y >= 0 && y < g.gy && x >= 0 && x < g.gx)
-            slot = box[(s * kBoxY + hy) * kBoxX + hx + 3];
-          const int sl = slot >= 0 ? slot : 0;
+          const int slot = (zin && bidx[j] >= 0) ? sbox[bidx[j]] : -1;
+          const int64_t src = (int64_t)(slot >= 0 ? slot : 0) * D + (int)(pc[j] >> 24) * 8;
           const uint32_t off = (pc[j] & 0xffffu) << 4;
-          tc::cp_async16(kd + off, P.kr + (kbase + sl) * D + c * 8, slot >= 0);
-          tc::cp_async16(vd + off, P.v + (vbase + sl) * D + c * 8, slot >= 0);
+          tc::cp_async16(kd + off, kgb + src, slot >= 0);
+          tc::cp_async16(vd + off, vgb + src, slot >= 0);
         }
         tc::cp_async_arrive_noinc(&bars[B_KVFULL + st]);
       }
