@@ -127,6 +127,10 @@ class ClockSampler:
 
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
+            # the sampler is live before the caller's timed region starts (up to 1 s)
+            t_end = time.time() + 1.0
+            while not self.rows and time.time() < t_end and self.thread.is_alive():
+                time.sleep(0.001)
             self.source = "nvml, 2 ms"
             return
         except Exception:
