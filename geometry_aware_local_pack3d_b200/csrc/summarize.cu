@@ -23,7 +23,8 @@
 // without a read), double-buffered: while the warp sums chunk f the rows of chunk f + 1 are in
 // flight, and the table lookups of chunks f + 2 (member slots) and f + 3 (group slot) are issued
 // ahead, so no load sits on the warp's path. The rotation table, read for every member row,
-// is copied into shared memory once per CTA. The sum itself: lane l handles 16-byte piece
+// is copied into shared memory once per CTA when it fits (up to 64 KB; a larger table is read
+// through L1). The sum itself: lane l handles 16-byte piece
 // (l % C) of member rows s = l / C, l / C + R, ... (C pieces per row, R = 32 / C rows per pass);
 // the R partial sums are then combined in fixed order with warp shuffles. Absent members (and
 // the zero padding of the last summary tile) are zero rows. The summation order depends on
